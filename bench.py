@@ -1,0 +1,385 @@
+"""Benchmark of one SparsePR attention call (all seven steps) on B200 GPUs.
+
+`python bench.py --gpus N --steps K --warmup W` times K calls of
+sparsepr_attention on the HunyuanVideo-shaped 720p workload (B=1, 24 heads,
+d=128, N=118800, rho_exec=22%) per GPU and prints one JSON line. Each rank
+processes its own call on its own seeded inputs (weak scaling, no data-path
+collective); the time is the max over ranks of CUDA-event time.
+
+`--impl reference` times the CPU oracle instead (the reference arm of this
+build): a bounded sample of the same workload, scaled to the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SparsePR attn ms/call & dense-equiv TFLOPS at N=118800, 24 heads, rho=22%"
+UNIT = "TFLOPS (dense-equivalent)"
+DEFAULT_WORKLOAD = "hunyuan720p_n118800"
+
+
+# ----------------------------------------------------------------------------- distributed helpers
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def dist_init(backend: str, timeout_s: int = 300):
+    import datetime
+
+    import torch.distributed as dist
+
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a scalar over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def whole_job_value(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Dense-equivalent TFLOPS of the whole job: all ranks' work over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        under = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(under), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- peaks
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"bf16_tflops": d["bf16_tflops"], "bf16_tflops_sustained": d["bf16_tflops_sustained"],
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) sample
+
+def oracle_sample_seconds(w, n_groups: int = 4):
+    """Time the CPU oracle on one KV head of workload w and scale to one whole call.
+
+    The sample: the full partition and route of KV head 0 (all N rows), then exact
+    sparse attention for `n_groups` query groups, the M dense probe rows, the
+    ridge fit and the correction of those groups. Per call = Hkv * (partition +
+    route + fit + attention_sample * Gq / n_groups) for each of the g query heads.
+    """
+    import oracle
+    from synthetic import bf16_bits_to_f64, video_qkv
+
+    one = w.replace(B=1, Hq=w.g, Hkv=1)
+    Qb, Kb, Vb = video_qkv(one)
+    Q, K, V = (bf16_bits_to_f64(x) for x in (Qb, Kb, Vb))
+    Qg, Kh, Vh = Q[0], K[0, 0], V[0, 0]
+    t0 = time.perf_counter()
+    part = oracle.partition_head(Qg, Kh, one)
+    t1 = time.perf_counter()
+    rt = oracle.route_head(Qg, part, one)
+    t2 = time.perf_counter()
+    groups = np.unique(part.qgroup)[:n_groups]
+    rows = np.nonzero(np.isin(part.qgroup, groups))[0]
+    t_attn = t_fit = 0.0
+    for j in range(w.g):
+        ta = time.perf_counter()
+        o, _ = oracle.sparse_attention(Qg[j], Kh, Vh, part.qgroup, part.kgroup, rt.sel,
+                                       rows=np.union1d(rows, part.probe))
+        tb = time.perf_counter()
+        fit = oracle.fit_head(Qg[j], Kh, Vh, o[part.probe], part, one)
+        oracle.correction(o[rows], fit.U, fit.A, fit.obar, fit.Rbar)
+        tc = time.perf_counter()
+        t_attn += tb - ta
+        t_fit += tc - tb
+    sample_s = tc - t0
+    frac = len(rows) / float(w.N)
+    per_head = (t1 - t0) + (t2 - t1) + t_fit + t_attn / max(frac, 1e-12)
+    per_call = per_head * w.Hkv * w.B
+    desc = (f"KV head 0 of {w.name}: full partition + route, exact attention/fit/correction for "
+            f"{len(groups)} of {w.Gq} query groups ({len(rows)} rows) on each of its {w.g} query heads; "
+            f"scaled by rows and by {w.B * w.Hkv} KV heads")
+    return per_call, sample_s, desc
+
+
+def cpu_cores_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    """The oracle on the host cores: the reference arm (rank 0 only under torchrun)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from synthetic import get_workload
+
+    w = get_workload(args.workload)
+    vals = []
+    sample_desc = ""
+    for i in range(args.warmup + args.steps):
+        per_call, sample_s, sample_desc = oracle_sample_seconds(w, n_groups=2)
+        if i >= args.warmup:
+            vals.append(per_call)
+    per_call = statistics.mean(vals)
+    value = w.dense_equiv_flops() / per_call / 1e12
+    cores = cpu_cores_used()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_call * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, world=1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample_desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "grid_thw": [w.T, w.Hg, w.Wg],
+            "d": w.d, "Gk": w.Gk, "Gq": w.Gq, "block": w.block, "rho_exec_target": w.rho, "rK": w.rK,
+            "rQ": w.rQ, "M": w.M, "r": w.r, "lambda": w.lam, "kmeans_iters": w.kmeans_iters,
+            "parallelism": f"independent calls on {world} GPU(s), one per rank (no collective)",
+            "l2": "inputs larger than L2 (Q, K, V are 730 MB each; no flush needed)"}
+
+
+def run_ours(args):
+    import torch
+
+    import free_block_sparse_sparsepr_b200 as spr
+    from synthetic import get_workload, video_qkv
+
+    rank, world = dist_init("nccl" if torch.cuda.is_available() else "gloo")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = get_workload(args.workload)
+
+    # seeded inputs of this rank's call, resident in HBM
+    Qb, Kb, Vb = video_qkv(w, layer=rank)
+    host = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) for x in (Qb, Kb, Vb)]
+    q, k, v = (t.to(dev) for t in host)
+    O = torch.empty_like(q)
+    h = spr.SparsePR.from_workload(w)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        h.attention(q, k, v, O)
+    torch.cuda.synchronize()
+    launches = h.last_launch_count()
+    st = h.stats()
+
+    # timed region: K calls, per-stage events of every call on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            h.set_stage_events(evs[i])
+            h.attention(q, k, v, O)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    h.set_stage_events(None)
+    ms = start.elapsed_time(end) / args.steps
+    ms_max = reduce_max(ms, dev)
+    stage_names = ["partition", "route", "permute", "attention", "probe_fit", "writeback"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(stage_names)}
+    st = h.stats()
+    flops = w.dense_equiv_flops()
+    value = whole_job_value(flops, world, ms_max)
+
+    # roofline of the dominant kernel: block-sparse attention on the routed cells
+    peaks = measured_peaks()
+    routed_pairs = st["route_density"] * float(w.N) ** 2 * w.B * w.Hq
+    attn_flops = 4.0 * w.d * routed_pairs
+    achieved = attn_flops / (stage_ms["attention"] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "kernel": "block-sparse attention (routed cells)", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_kind": f"bf16 sustained ({peaks['source']})",
+                "useful_flops_per_launch": attn_flops}
+
+    # end to end through the public API with HOST buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pin = [t.pin_memory() for t in host]
+        Oh = torch.empty_like(pin[0]).pin_memory()
+        h.attention_host(*pin, Oh)
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nsteps = max(1, min(args.steps, 3))
+        barrier()
+        torch.cuda.synchronize()
+        e_start.record(stream)
+        for _ in range(nsteps):
+            h.attention_host(*pin, Oh)
+        e_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = reduce_max(e_start.elapsed_time(e_end) / nsteps, dev)
+        h2d = sum(t.numel() * t.element_size() for t in pin)
+        e2e = {"value": whole_job_value(flops, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": Oh.numel() * Oh.element_size()}
+
+    # dense baseline of the same library on the same shapes
+    dense = None
+    if not args.no_dense:
+        Od = torch.empty_like(q)
+        h.dense_attn(q, k, v, Od)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        h.dense_attn(q, k, v, Od)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = reduce_max(d0.elapsed_time(d1), dev)
+        dense = {"ms_per_call": dms, "tflops": flops / (dms * 1e-3) / 1e12, "speedup_vs_dense": dms / ms_max,
+                 "frac_of_peak": flops / (dms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        per_call, sample_s, desc = oracle_sample_seconds(w)
+        cpu = {"value": flops / per_call / 1e12, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
+               "sample": desc, "sample_seconds": sample_s, "ms_per_call_extrapolated": per_call * 1e3}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, world),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches * args.steps,
+            "clocks": clk.summary(),
+            "stage_ms": stage_ms,
+            "realised": {"route_density": st["route_density"], "rho_exec": st["rho_exec"]},
+            "dense_baseline": dense,
+            "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

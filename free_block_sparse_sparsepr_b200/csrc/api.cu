@@ -1,0 +1,604 @@
+// C ABI of the SparsePR library: argument validation, workspace, and the
+// orchestration of the seven steps on one CUDA stream (no host synchronisation
+// inside the call).
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "sparsepr.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using spr::bf16;
+
+namespace {
+
+constexpr int kMaxGroups = 1024;
+constexpr int kProbeSplits = 32;
+constexpr int kSortChunk = 256;
+constexpr unsigned kSupportedFlags =
+    SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_STAGE_TIMING;
+
+inline int pad16(int v) { return (v + 15) / 16 * 16; }
+inline int pad64(int v) { return (v + 63) / 64 * 64; }
+
+enum Stage { kStPartition = 0, kStRoute, kStPermute, kStAttn, kStProbeFit, kStWriteback, kStUnused, kStTotal, kNumStages };
+
+}  // namespace
+
+struct sparsepr_handle_s {
+    sparsepr_config cfg;
+    int P = 0, Hp = 0, g = 0, M = 0;     // M = probes actually used (0 under hard drop)
+    int DPk = 0, Dy = 0, DPy = 0, Gkp = 0, nch = 0, Gmax = 0;
+    bool proj = false;
+    size_t bytes = 0;
+    std::vector<void*> allocs;
+    // partition
+    int32_t *kgroup = nullptr, *qgroup = nullptr, *kperm = nullptr, *koff = nullptr, *qperm = nullptr,
+            *qoff = nullptr, *probe = nullptr, *probe_pos = nullptr, *probe_seq = nullptr;
+    float *kcent = nullptr, *radial = nullptr, *weights = nullptr, *features = nullptr, *ycoord = nullptr,
+          *kdist = nullptr, *kmC = nullptr;
+    int *counts = nullptr, *bases = nullptr, *km_changed = nullptr, *km_done = nullptr;
+    bf16 *Qs = nullptr, *chi = nullptr, *clo = nullptr, *uhi = nullptr, *ulo = nullptr, *projT = nullptr;
+    float *u = nullptr, *ulse = nullptr;
+    // route
+    float* scores = nullptr;
+    int32_t *rowptr = nullptr, *kg = nullptr, *tile_off = nullptr;
+    int64_t* pairs = nullptr;
+    // permuted tensors and sparse output
+    bf16 *Qp = nullptr, *Kp = nullptr, *Vp = nullptr, *Osp = nullptr;
+    float* lse = nullptr;
+    // probes and fit
+    float *Opart = nullptr, *mpart = nullptr, *lpart = nullptr, *Odense = nullptr, *R = nullptr,
+          *Xprobe = nullptr, *obar = nullptr, *Rbar = nullptr, *A = nullptr, *U = nullptr, *Bm = nullptr,
+          *c0 = nullptr;
+    int32_t* rank = nullptr;
+    int* dev_status = nullptr;
+    // host-buffer variant staging (allocated on first use)
+    bf16 *sQ = nullptr, *sK = nullptr, *sV = nullptr, *sO = nullptr;
+    // timing
+    cudaEvent_t ev[kNumStages + 1] = {};
+    cudaEvent_t done_ev = nullptr;
+    cudaEvent_t user_ev[7] = {};
+    bool user_events = false;
+    bool timing = false, timed_call = false;
+    int launches = 0;
+    int device = 0;
+};
+
+namespace {
+
+#define SPR_TRY(expr)                                   \
+    do {                                                \
+        cudaError_t e_ = (expr);                        \
+        if (e_ != cudaSuccess) return SPARSEPR_ERR_CUDA; \
+        ++h->launches;                                  \
+    } while (0)
+
+template <typename T>
+sparsepr_status alloc(sparsepr_handle h, T** p, size_t count) {
+    if (count == 0) count = 1;
+    void* q = nullptr;
+    if (cudaMalloc(&q, count * sizeof(T)) != cudaSuccess) return SPARSEPR_ERR_WORKSPACE;
+    h->allocs.push_back(q);
+    h->bytes += count * sizeof(T);
+    *p = static_cast<T*>(q);
+    return SPARSEPR_OK;
+}
+
+void free_all(sparsepr_handle h) {
+    for (void* p : h->allocs) cudaFree(p);
+    h->allocs.clear();
+    for (auto& e : h->ev)
+        if (e) cudaEventDestroy(e);
+    if (h->done_ev) cudaEventDestroy(h->done_ev);
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sparsepr_status validate(const sparsepr_config* c) {
+    if (!c) return SPARSEPR_ERR_INVALID_ARG;
+    if (c->B < 1 || c->Hq < 1 || c->Hkv < 1 || c->Hq % c->Hkv != 0 || c->N < 1) return SPARSEPR_ERR_INVALID_ARG;
+    if (c->d != 64 && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
+    if (c->block != 64 && c->block != 128) return SPARSEPR_ERR_INVALID_ARG;
+    if (c->Gk < 1 || c->Gq < 1 || c->Gk > c->N || c->Gq > c->N) return SPARSEPR_ERR_INVALID_ARG;
+    if (c->Gk > kMaxGroups || c->Gq > kMaxGroups) return SPARSEPR_ERR_UNSUPPORTED;
+    if ((long long)c->Gq * c->Gk > (1ll << 20)) return SPARSEPR_ERR_UNSUPPORTED;
+    if (c->rK < 1 || c->rK > 64 || c->rQ < 1 || c->rQ > 64) return SPARSEPR_ERR_INVALID_ARG;
+    if (c->kmeans_iters < 0 || c->kmeans_iters > 64) return SPARSEPR_ERR_INVALID_ARG;
+    if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return SPARSEPR_ERR_INVALID_ARG;
+    if (!(c->rho_exec > 0.f) || !isfinite(c->rho_exec)) return SPARSEPR_ERR_INVALID_ARG;
+    if (c->flags & ~(kSupportedFlags | SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED))
+        return SPARSEPR_ERR_INVALID_ARG;
+    if (c->flags & (SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED)) return SPARSEPR_ERR_UNSUPPORTED;
+    if (!(c->flags & SPARSEPR_FLAG_HARD_DROP_ONLY)) {
+        if (c->M < 1 || c->M > c->N) return SPARSEPR_ERR_INVALID_ARG;
+        if (c->M > 64) return SPARSEPR_ERR_UNSUPPORTED;
+        if (c->r < 1 || c->r > c->M || c->r > 32) return SPARSEPR_ERR_INVALID_ARG;
+    }
+    if ((long long)c->N * c->Gk > (1ll << 31) || (long long)c->N * 128 > (1ll << 31))
+        return SPARSEPR_ERR_UNSUPPORTED;
+    return SPARSEPR_OK;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+void mark(sparsepr_handle h, int stage, cudaStream_t s) {
+    if (h->user_events) cudaEventRecord(h->user_ev[stage], s);
+    else if (h->timing) cudaEventRecord(h->ev[stage], s);
+}
+
+long long budget_pairs(const sparsepr_config& c, int M) {
+    const double nn = (double)((long long)c.N * c.N);
+    return (long long)floor((double)c.rho_exec * nn) - (long long)M * c.N;
+}
+
+// Lloyd k-means on X [P][n][DP] into G groups, then the stable group-major order.
+sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t* labels, float* dist,
+                       int32_t* perm, int32_t* off, cudaStream_t s) {
+    const int P = h->P, n = h->cfg.N;
+    SPR_TRY(spr::launch_km_reset(h->km_changed, h->km_done, P, s));
+    SPR_TRY(spr::launch_km_seed(X, h->kmC, P, n, G, DP, s));
+    SPR_TRY(spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, nullptr, P, n, G, DP, true, s));
+    for (int it = 0; it < h->cfg.kmeans_iters; ++it) {
+        SPR_TRY(spr::launch_group_sort(labels, perm, off, h->counts, h->bases, h->km_done, P, n, G, s));
+        h->launches += 2;  // histogram, scan and scatter kernels
+        SPR_TRY(spr::launch_km_update(X, perm, off, h->kmC, h->km_done, P, n, G, DP, s));
+        SPR_TRY(spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, h->km_done, P, n, G, DP, false, s));
+        SPR_TRY(spr::launch_km_check(h->km_changed, h->km_done, P, s));
+    }
+    SPR_TRY(spr::launch_group_sort(labels, perm, off, h->counts, h->bases, nullptr, P, n, G, s));
+    h->launches += 2;
+    return SPARSEPR_OK;
+}
+
+// u[x] = Q[x] . kcent[z]^T / sqrt(d) with kcent split into bf16 hi + lo.
+sparsepr_status query_logits(sparsepr_handle h, const bf16* Q, const bf16* chi, const bf16* clo, cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    spr::GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.A1 = Q; a.A2 = nullptr; a.sA = (long long)c.N * c.d; a.lda = c.d;
+    a.B1 = chi; a.B2 = clo; a.sB = (long long)c.Gk * c.d; a.ldb = c.d; a.bdiv = h->g;
+    a.C = h->u; a.sC = (long long)c.N * c.Gk; a.ldc = c.Gk;
+    a.M = c.N; a.N = c.Gk; a.K = c.d; a.batch = h->Hp;
+    a.alpha = (float)(1.0 / sqrt((double)c.d));
+    SPR_TRY(spr::launch_gemm_bf16(a, s));
+    return SPARSEPR_OK;
+}
+
+sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    const int P = h->P, N = c.N, d = c.d;
+    // (1) sampled responses: F[z] = K[z] . Qs[z]^T / sqrt(d)
+    SPR_TRY(spr::launch_gather_samples(Q, h->Qs, c.B, c.Hq, c.Hkv, N, d, c.rK, h->DPk, s));
+    spr::GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.A1 = K; a.sA = (long long)N * d; a.lda = d;
+    a.B1 = h->Qs; a.sB = (long long)h->DPk * d; a.ldb = d; a.bdiv = 1;
+    a.C = h->features; a.sC = (long long)N * h->DPk; a.ldc = h->DPk;
+    a.M = N; a.N = h->DPk; a.K = d; a.batch = P;
+    a.alpha = (float)(1.0 / sqrt((double)d));
+    SPR_TRY(spr::launch_gemm_bf16(a, s));
+    // (2a) key groups and their means in the original key space
+    sparsepr_status st = kmeans(h, h->features, h->DPk, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s);
+    if (st) return st;
+    SPR_TRY(spr::launch_group_mean_bf16(K, h->kperm, h->koff, h->kcent, h->chi, h->clo, P, N, c.Gk, d, s));
+    // (2b) query coordinates and query groups
+    st = query_logits(h, Q, h->chi, h->clo, s);
+    if (st) return st;
+    SPR_TRY(spr::launch_coords_center(h->u, h->uhi, h->ulo, h->ycoord, P, h->g, N, c.Gk, h->Gkp, h->DPy, h->proj, s));
+    if (h->proj) {
+        spr::GemmArgs b;
+        memset(&b, 0, sizeof(b));
+        b.A1 = h->uhi; b.A2 = h->ulo; b.sA = (long long)N * h->Gkp; b.lda = h->Gkp;
+        b.B1 = h->projT; b.B2 = nullptr; b.sB = 0; b.ldb = h->Gkp; b.bdiv = 1;
+        b.C = h->ycoord; b.sC = (long long)N * h->DPy; b.ldc = h->DPy;
+        b.M = N; b.N = h->DPy; b.K = h->Gkp; b.batch = P; b.alpha = 1.f;
+        SPR_TRY(spr::launch_gemm_bf16(b, s));
+        SPR_TRY(spr::launch_rows_normalize(h->ycoord, P * N, h->DPy, s));
+    }
+    st = kmeans(h, h->ycoord, h->DPy, c.Gq, h->qgroup, h->radial, h->qperm, h->qoff, s);
+    if (st) return st;
+    // probe rows (stratified, radial order) and their coverage weights
+    if (h->M) {
+        SPR_TRY(spr::launch_probe_select(h->qperm, h->qoff, h->radial, h->probe, h->probe_pos, h->probe_seq,
+                                         P, N, c.Gq, h->M, s));
+        SPR_TRY(spr::launch_probe_weights(h->qoff, h->probe_seq, h->weights, P, N, c.Gq, h->M,
+                                          (c.flags & SPARSEPR_FLAG_UNIFORM_WEIGHTS) != 0, s));
+    }
+    return SPARSEPR_OK;
+}
+
+void fill_partition(sparsepr_handle h, sparsepr_partition_t* p) {
+    p->kgroup = h->kgroup; p->qgroup = h->qgroup; p->kperm = h->kperm; p->koff = h->koff;
+    p->qperm = h->qperm; p->qoff = h->qoff; p->kcent = h->kcent; p->radial = h->radial;
+    p->probe = h->probe; p->probe_pos = h->probe_pos; p->weights = h->weights; p->features = h->features;
+}
+
+void fill_route(sparsepr_handle h, sparsepr_route_t* r) {
+    r->rowptr = h->rowptr; r->kg = h->kg; r->scores = h->scores; r->pairs = h->pairs;
+}
+
+void fill_fit(sparsepr_handle h, sparsepr_fit_t* f) {
+    f->obar = h->obar; f->Rbar = h->Rbar; f->A = h->A; f->U = h->U; f->Bm = h->Bm; f->c0 = h->c0;
+    f->rank = h->rank; f->R = h->R; f->Odense = h->Odense; f->Osp = h->Xprobe;
+}
+
+sparsepr_status check_partition(const sparsepr_partition_t* p, bool need_probe) {
+    if (!p || !p->kperm || !p->koff || !p->qperm || !p->qoff || !p->kcent) return SPARSEPR_ERR_INVALID_ARG;
+    if (need_probe && (!p->probe || !p->probe_pos || !p->weights)) return SPARSEPR_ERR_INVALID_ARG;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status route_impl(sparsepr_handle h, const bf16* Q, const sparsepr_partition_t* p, bool logits_ready,
+                           cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    if (!logits_ready) {
+        SPR_TRY(spr::launch_split_bf16(p->kcent, h->chi, h->clo, (long long)h->P * c.Gk * c.d, s));
+        sparsepr_status st = query_logits(h, Q, h->chi, h->clo, s);
+        if (st) return st;
+    }
+    SPR_TRY(spr::launch_row_lse(h->u, p->koff, h->ulse, h->Hp, h->g, c.N, c.Gk, s));
+    SPR_TRY(spr::launch_cell_scores(h->u, h->ulse, p->qperm, p->qoff, p->koff, h->scores, h->P, h->g, c.N,
+                                    c.Gq, c.Gk, s));
+    SPR_TRY(spr::launch_route_select(h->scores, p->qoff, p->koff, h->rowptr, h->kg, h->pairs, h->P, c.Gq, c.Gk,
+                                     budget_pairs(c, h->M), c.rho_exec >= 1.0f, s));
+    return SPARSEPR_OK;
+}
+
+sparsepr_status permute_impl(sparsepr_handle h, const bf16* Q, const bf16* K, const bf16* V,
+                             const sparsepr_partition_t* p, bf16* Qp, bf16* Kp, bf16* Vp, cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    if (Qp) SPR_TRY(spr::launch_permute_rows(Q, Qp, p->qperm, h->Hp, h->g, c.N, c.d, s));
+    if (Kp) SPR_TRY(spr::launch_permute_rows(K, Kp, p->kperm, h->P, 1, c.N, c.d, s));
+    if (Vp) SPR_TRY(spr::launch_permute_rows(V, Vp, p->kperm, h->P, 1, c.N, c.d, s));
+    return SPARSEPR_OK;
+}
+
+sparsepr_status attn_impl(sparsepr_handle h, const bf16* Qp, const bf16* Kp, const bf16* Vp,
+                          const sparsepr_partition_t* p, const sparsepr_route_t* r, bf16* Osp, float* lse,
+                          cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, 64, s));
+    SPR_TRY(spr::launch_attn_sparse(Qp, Kp, Vp, p->qoff, p->koff, h->tile_off, r->rowptr, r->kg, Osp, lse,
+                                    c.B, c.Hq, c.Hkv, c.N, c.d, c.Gq, c.Gk, s));
+    return SPARSEPR_OK;
+}
+
+sparsepr_status probe_fit_impl(sparsepr_handle h, const bf16* Q, const bf16* K, const bf16* V,
+                               const sparsepr_partition_t* p, const bf16* Osp, cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    if (!h->M) return SPARSEPR_OK;
+    SPR_TRY(spr::launch_attn_probe(Q, K, V, p->probe, h->Opart, h->mpart, h->lpart, h->Odense, c.B, c.Hq, c.Hkv,
+                                   c.N, c.d, h->M, kProbeSplits, s));
+    ++h->launches;  // combine kernel
+    SPR_TRY(spr::launch_probe_residual(h->Odense, Osp, p->probe_pos, h->R, h->Xprobe, h->Hp, h->g, c.N, c.d,
+                                       h->M, s));
+    SPR_TRY(spr::launch_fit(h->R, h->Xprobe, p->weights, c.lambda, h->obar, h->Rbar, h->A, h->U, h->Bm, h->c0,
+                            h->rank, h->Hp, h->g, c.d, h->M, c.r, h->dev_status, s));
+    return SPARSEPR_OK;
+}
+
+sparsepr_status writeback_impl(sparsepr_handle h, const sparsepr_partition_t* p, const bf16* Osp,
+                               const float* U, const float* Bm, const float* c0, const float* Odense, bf16* O,
+                               cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    const bool correct = h->M > 0;
+    SPR_TRY(spr::launch_writeback(Osp, p->qperm, U, Bm, c0, O, h->Hp, h->g, c.N, c.d, correct ? c.r : 1,
+                                  correct, s));
+    if (correct) SPR_TRY(spr::launch_probe_override(Odense, p->probe, O, h->Hp, h->g, c.N, c.d, h->M, s));
+    return SPARSEPR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sparsepr_status_string(sparsepr_status s) {
+    switch (s) {
+        case SPARSEPR_OK: return "ok";
+        case SPARSEPR_ERR_INVALID_ARG: return "invalid argument";
+        case SPARSEPR_ERR_UNSUPPORTED: return "unsupported configuration";
+        case SPARSEPR_ERR_WORKSPACE: return "workspace allocation failed";
+        case SPARSEPR_ERR_CUDA: return "CUDA error";
+        case SPARSEPR_ERR_TIMEOUT: return "device wait timed out";
+        case SPARSEPR_ERR_DEVICE: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+int sparsepr_version(void) { return 100; }
+
+sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out) {
+    if (!out) return SPARSEPR_ERR_INVALID_ARG;
+    *out = nullptr;
+    sparsepr_status st = validate(cfg);
+    if (st) return st;
+    sparsepr_handle h = new (std::nothrow) sparsepr_handle_s();
+    if (!h) return SPARSEPR_ERR_WORKSPACE;
+    h->cfg = *cfg;
+    const sparsepr_config& c = h->cfg;
+    cudaGetDevice(&h->device);
+    h->P = c.B * c.Hkv;
+    h->Hp = c.B * c.Hq;
+    h->g = c.Hq / c.Hkv;
+    h->M = (c.flags & SPARSEPR_FLAG_HARD_DROP_ONLY) ? 0 : c.M;
+    h->DPk = pad16(c.rK);
+    h->proj = c.Gk > c.rQ;
+    h->Dy = h->proj ? c.rQ : c.Gk;
+    h->DPy = pad16(h->Dy);
+    h->Gkp = pad64(c.Gk);
+    h->nch = (c.N + kSortChunk - 1) / kSortChunk;
+    h->Gmax = c.Gk > c.Gq ? c.Gk : c.Gq;
+    h->timing = (c.flags & SPARSEPR_FLAG_STAGE_TIMING) != 0;
+    const size_t P = h->P, Hp = h->Hp, N = c.N, d = c.d, M = h->M > 0 ? h->M : 1, r = c.r > 0 ? c.r : 1;
+    const size_t Gk = c.Gk, Gq = c.Gq;
+#define A_(ptr, n)                                 \
+    do {                                           \
+        if ((st = alloc(h, &h->ptr, (n)))) {       \
+            free_all(h);                           \
+            delete h;                              \
+            return st;                             \
+        }                                          \
+    } while (0)
+    A_(kgroup, P * N); A_(qgroup, P * N); A_(kperm, P * N); A_(koff, P * (Gk + 1));
+    A_(qperm, P * N); A_(qoff, P * (Gq + 1)); A_(probe, P * M); A_(probe_pos, P * M); A_(probe_seq, P * M);
+    A_(kcent, P * Gk * d); A_(radial, P * N); A_(weights, P * M); A_(features, P * N * h->DPk);
+    A_(ycoord, P * N * h->DPy); A_(kdist, P * N); A_(kmC, P * h->Gmax * 64);
+    A_(counts, P * h->nch * h->Gmax); A_(bases, P * h->nch * h->Gmax); A_(km_changed, P); A_(km_done, P);
+    A_(Qs, P * h->DPk * d); A_(chi, P * Gk * d); A_(clo, P * Gk * d);
+    A_(u, Hp * N * Gk); A_(ulse, Hp * N);
+    if (h->proj) {
+        A_(uhi, P * N * h->Gkp); A_(ulo, P * N * h->Gkp); A_(projT, (size_t)h->DPy * h->Gkp);
+    }
+    A_(scores, P * Gq * Gk); A_(rowptr, P * (Gq + 1)); A_(kg, P * Gq * Gk); A_(tile_off, P * (Gq + 1));
+    A_(pairs, P);
+    A_(Qp, Hp * N * d); A_(Kp, P * N * d); A_(Vp, P * N * d); A_(Osp, Hp * N * d); A_(lse, Hp * N);
+    A_(Opart, Hp * kProbeSplits * M * d); A_(mpart, Hp * kProbeSplits * M); A_(lpart, Hp * kProbeSplits * M);
+    A_(Odense, Hp * M * d); A_(R, Hp * M * d); A_(Xprobe, Hp * M * d);
+    A_(obar, Hp * d); A_(Rbar, Hp * d); A_(A, Hp * d * d); A_(U, Hp * d * r); A_(Bm, Hp * r * d); A_(c0, Hp * r);
+    A_(rank, Hp); A_(dev_status, 1);
+#undef A_
+    bool ok = cudaMemset(h->dev_status, 0, sizeof(int)) == cudaSuccess;
+    if (h->proj) {
+        ok = ok && cudaMemset(h->uhi, 0, P * N * h->Gkp * sizeof(bf16)) == cudaSuccess;
+        ok = ok && cudaMemset(h->ulo, 0, P * N * h->Gkp * sizeof(bf16)) == cudaSuccess;
+        ok = ok && spr::launch_make_projection(h->projT, c.Gk, h->Gkp, c.rQ, h->DPy, c.seed, 0) == cudaSuccess;
+    }
+    ok = ok && cudaMemset(h->ycoord, 0, P * N * h->DPy * sizeof(float)) == cudaSuccess;
+    for (auto& e : h->ev) ok = ok && cudaEventCreate(&e) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&h->done_ev, cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    if (!ok) {
+        free_all(h);
+        delete h;
+        return SPARSEPR_ERR_CUDA;
+    }
+    *out = h;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_destroy(sparsepr_handle h) {
+    if (!h) return SPARSEPR_OK;
+    cudaDeviceSynchronize();
+    if (h->sQ) { cudaFree(h->sQ); cudaFree(h->sK); cudaFree(h->sV); cudaFree(h->sO); }
+    free_all(h);
+    delete h;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_workspace_bytes(sparsepr_handle h, size_t* out) {
+    if (!h || !out) return SPARSEPR_ERR_INVALID_ARG;
+    *out = h->bytes;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_partition(sparsepr_handle h, const void* Q, const void* K, sparsepr_partition_t* out,
+                                   void* stream) {
+    if (!h || !aligned16(Q) || !aligned16(K) || !out) return SPARSEPR_ERR_INVALID_ARG;
+    h->launches = 0;
+    cudaStream_t s = as_stream(stream);
+    sparsepr_status st = partition_impl(h, static_cast<const bf16*>(Q), static_cast<const bf16*>(K), s);
+    if (st) return st;
+    fill_partition(h, out);
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_route(sparsepr_handle h, const void* Q, const sparsepr_partition_t* part,
+                               sparsepr_route_t* out, void* stream) {
+    if (!h || !aligned16(Q) || !out) return SPARSEPR_ERR_INVALID_ARG;
+    sparsepr_status st = check_partition(part, false);
+    if (st) return st;
+    h->launches = 0;
+    cudaStream_t s = as_stream(stream);
+    st = route_impl(h, static_cast<const bf16*>(Q), part, false, s);
+    if (st) return st;
+    cudaEventRecord(h->done_ev, s);
+    h->timed_call = false;
+    fill_route(h, out);
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_permute(sparsepr_handle h, const void* Q, const void* K, const void* V,
+                                 const sparsepr_partition_t* part, void* Qp, void* Kp, void* Vp, void* stream) {
+    if (!h) return SPARSEPR_ERR_INVALID_ARG;
+    sparsepr_status st = check_partition(part, false);
+    if (st) return st;
+    if ((Qp && (!aligned16(Q) || !aligned16(Qp))) || (Kp && (!aligned16(K) || !aligned16(Kp))) ||
+        (Vp && (!aligned16(V) || !aligned16(Vp))))
+        return SPARSEPR_ERR_INVALID_ARG;
+    h->launches = 0;
+    return permute_impl(h, static_cast<const bf16*>(Q), static_cast<const bf16*>(K), static_cast<const bf16*>(V),
+                        part, static_cast<bf16*>(Qp), static_cast<bf16*>(Kp), static_cast<bf16*>(Vp),
+                        as_stream(stream));
+}
+
+sparsepr_status sparsepr_blocksparse_attn(sparsepr_handle h, const void* Qp, const void* Kp, const void* Vp,
+                                          const sparsepr_partition_t* part, const sparsepr_route_t* route, void* Osp,
+                                          float* lse, void* stream) {
+    if (!h || !aligned16(Qp) || !aligned16(Kp) || !aligned16(Vp) || !aligned16(Osp)) return SPARSEPR_ERR_INVALID_ARG;
+    sparsepr_status st = check_partition(part, false);
+    if (st) return st;
+    if (!route || !route->rowptr || !route->kg) return SPARSEPR_ERR_INVALID_ARG;
+    h->launches = 0;
+    return attn_impl(h, static_cast<const bf16*>(Qp), static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp),
+                     part, route, static_cast<bf16*>(Osp), lse, as_stream(stream));
+}
+
+sparsepr_status sparsepr_probe_fit(sparsepr_handle h, const void* Q, const void* K, const void* V,
+                                   const sparsepr_partition_t* part, const void* Osp, sparsepr_fit_t* out,
+                                   void* stream) {
+    if (!h || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Osp) || !out)
+        return SPARSEPR_ERR_INVALID_ARG;
+    sparsepr_status st = check_partition(part, true);
+    if (st) return st;
+    if (!h->M) return SPARSEPR_ERR_INVALID_ARG;
+    h->launches = 0;
+    st = probe_fit_impl(h, static_cast<const bf16*>(Q), static_cast<const bf16*>(K), static_cast<const bf16*>(V),
+                        part, static_cast<const bf16*>(Osp), as_stream(stream));
+    if (st) return st;
+    fill_fit(h, out);
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_writeback(sparsepr_handle h, const sparsepr_partition_t* part, const void* Osp,
+                                   const sparsepr_fit_t* fit, void* O, void* stream) {
+    if (!h || !aligned16(Osp) || !aligned16(O)) return SPARSEPR_ERR_INVALID_ARG;
+    sparsepr_status st = check_partition(part, h->M > 0);
+    if (st) return st;
+    if (h->M && (!fit || !fit->U || !fit->Bm || !fit->c0 || !fit->Odense)) return SPARSEPR_ERR_INVALID_ARG;
+    h->launches = 0;
+    return writeback_impl(h, part, static_cast<const bf16*>(Osp), fit ? fit->U : nullptr, fit ? fit->Bm : nullptr,
+                          fit ? fit->c0 : nullptr, fit ? fit->Odense : nullptr, static_cast<bf16*>(O),
+                          as_stream(stream));
+}
+
+sparsepr_status sparsepr_attention(sparsepr_handle h, const void* Q, const void* K, const void* V, void* O,
+                                   void* stream) {
+    if (!h || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARSEPR_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    const bf16* q = static_cast<const bf16*>(Q);
+    const bf16* k = static_cast<const bf16*>(K);
+    const bf16* v = static_cast<const bf16*>(V);
+    h->launches = 0;
+    sparsepr_partition_t part;
+    sparsepr_route_t route;
+    fill_partition(h, &part);
+    fill_route(h, &route);
+    mark(h, 0, s);
+    sparsepr_status st = partition_impl(h, q, k, s);
+    if (st) return st;
+    mark(h, 1, s);
+    if ((st = route_impl(h, q, &part, true, s))) return st;
+    mark(h, 2, s);
+    if ((st = permute_impl(h, q, k, v, &part, h->Qp, h->Kp, h->Vp, s))) return st;
+    mark(h, 3, s);
+    if ((st = attn_impl(h, h->Qp, h->Kp, h->Vp, &part, &route, h->Osp, h->lse, s))) return st;
+    mark(h, 4, s);
+    if ((st = probe_fit_impl(h, q, k, v, &part, h->Osp, s))) return st;
+    mark(h, 5, s);
+    if ((st = writeback_impl(h, &part, h->Osp, h->U, h->Bm, h->c0, h->Odense, static_cast<bf16*>(O), s)))
+        return st;
+    mark(h, 6, s);
+    cudaEventRecord(h->done_ev, s);
+    h->timed_call = h->timing && !h->user_events;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const void* K, const void* V, void* O,
+                                        void* stream) {
+    if (!h || !Q || !K || !V || !O) return SPARSEPR_ERR_INVALID_ARG;
+    const sparsepr_config& c = h->cfg;
+    const size_t qb = (size_t)c.B * c.Hq * c.N * c.d * sizeof(bf16);
+    const size_t kb = (size_t)c.B * c.Hkv * c.N * c.d * sizeof(bf16);
+    if (!h->sQ) {
+        void *a = nullptr, *b = nullptr, *cc = nullptr, *dd = nullptr;
+        if (cudaMalloc(&a, qb) || cudaMalloc(&b, kb) || cudaMalloc(&cc, kb) || cudaMalloc(&dd, qb)) {
+            if (a) cudaFree(a);
+            if (b) cudaFree(b);
+            if (cc) cudaFree(cc);
+            if (dd) cudaFree(dd);
+            return SPARSEPR_ERR_WORKSPACE;
+        }
+        h->sQ = static_cast<bf16*>(a); h->sK = static_cast<bf16*>(b);
+        h->sV = static_cast<bf16*>(cc); h->sO = static_cast<bf16*>(dd);
+    }
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(h->sQ, Q, qb, cudaMemcpyHostToDevice, s) || cudaMemcpyAsync(h->sK, K, kb, cudaMemcpyHostToDevice, s) ||
+        cudaMemcpyAsync(h->sV, V, kb, cudaMemcpyHostToDevice, s))
+        return SPARSEPR_ERR_CUDA;
+    sparsepr_status st = sparsepr_attention(h, h->sQ, h->sK, h->sV, h->sO, stream);
+    if (st) return st;
+    if (cudaMemcpyAsync(O, h->sO, qb, cudaMemcpyDeviceToHost, s)) return SPARSEPR_ERR_CUDA;
+    if (cudaStreamSynchronize(s)) return SPARSEPR_ERR_CUDA;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_dense_attn(sparsepr_handle h, const void* Q, const void* K, const void* V, void* O,
+                                    void* stream) {
+    if (!h || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARSEPR_ERR_INVALID_ARG;
+    const sparsepr_config& c = h->cfg;
+    h->launches = 0;
+    SPR_TRY(spr::launch_attn_dense(static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
+                                   static_cast<const bf16*>(V), static_cast<bf16*>(O), nullptr, c.B, c.Hq, c.Hkv,
+                                   c.N, c.d, as_stream(stream)));
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_get_stats(sparsepr_handle h, sparsepr_stats* out) {
+    if (!h || !out) return SPARSEPR_ERR_INVALID_ARG;
+    memset(out, 0, sizeof(*out));
+    if (cudaEventSynchronize(h->done_ev) != cudaSuccess) return SPARSEPR_ERR_CUDA;
+    const sparsepr_config& c = h->cfg;
+    std::vector<int64_t> pairs(h->P);
+    if (cudaMemcpy(pairs.data(), h->pairs, h->P * sizeof(int64_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SPARSEPR_ERR_CUDA;
+    const double nn = (double)c.N * (double)c.N;
+    double dens = 0.0, useful = 0.0;
+    for (int z = 0; z < h->P; ++z) {
+        dens += (double)pairs[z] / nn;
+        useful += (double)h->g * ((double)pairs[z] + (double)h->M * c.N);
+    }
+    out->route_density = dens / h->P;
+    out->rho_exec = out->route_density + (double)h->M / c.N;
+    out->useful_pairs = useful;
+    if (h->timed_call) {
+        for (int i = 0; i < 6; ++i) cudaEventElapsedTime(&out->stage_ms[i], h->ev[i], h->ev[i + 1]);
+        cudaEventElapsedTime(&out->stage_ms[kStTotal], h->ev[0], h->ev[6]);
+    }
+    int ds = 0;
+    if (cudaMemcpy(&ds, h->dev_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SPARSEPR_ERR_CUDA;
+    out->device_status = ds;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_device_status(sparsepr_handle h, int* out) {
+    if (!h || !out) return SPARSEPR_ERR_INVALID_ARG;
+    if (cudaMemcpy(out, h->dev_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SPARSEPR_ERR_CUDA;
+    if (cudaMemset(h->dev_status, 0, sizeof(int)) != cudaSuccess) return SPARSEPR_ERR_CUDA;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_set_stage_events(sparsepr_handle h, void* const* events) {
+    if (!h) return SPARSEPR_ERR_INVALID_ARG;
+    if (!events) {
+        h->user_events = false;
+        return SPARSEPR_OK;
+    }
+    for (int i = 0; i < 7; ++i)
+        if (!events[i]) return SPARSEPR_ERR_INVALID_ARG;
+    for (int i = 0; i < 7; ++i) h->user_ev[i] = static_cast<cudaEvent_t>(events[i]);
+    h->user_events = true;
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_last_launch_count(sparsepr_handle h, int* out) {
+    if (!h || !out) return SPARSEPR_ERR_INVALID_ARG;
+    *out = h->launches;
+    return SPARSEPR_OK;
+}
+
+}  // extern "C"

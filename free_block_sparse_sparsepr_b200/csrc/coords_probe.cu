@@ -1,0 +1,227 @@
+// Sampled query rows, query coordinates against the key-group centroids, and
+// the stratified radial probe rows with their group-coverage weights.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spr {
+namespace {
+
+// Qs[z][s] = Q[b][h*g + s%g][floor((s+1/2)N/S)] (bf16 rows), zero rows for S <= s < DP.
+__global__ void gather_samples_kernel(const bf16* __restrict__ Q, bf16* Qs, int Hq, int Hkv, int N,
+                                      int d, int S, int DP) {
+    const int z = blockIdx.x, b = z / Hkv, h = z % Hkv, g = Hq / Hkv;
+    const int vpr = d / 8;  // 16-byte vectors per row
+    for (int t = threadIdx.x; t < DP * vpr; t += blockDim.x) {
+        int sidx = t / vpr, c = t % vpr;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (sidx < S) {
+            long long row = sample_pos(sidx, N, S);
+            int head = h * g + sidx % g;
+            v = reinterpret_cast<const uint4*>(Q + (((long long)b * Hq + head) * N + row) * d)[c];
+        }
+        reinterpret_cast<uint4*>(Qs + ((long long)z * DP + sidx) * d)[c] = v;
+    }
+}
+
+// One warp per query row of a KV head: mean of the g heads' logits, centred over the groups.
+__global__ void coords_center_kernel(const float* __restrict__ u, bf16* uhi, bf16* ulo, float* y,
+                                     int g, int N, int Gk, int Gkp, int DPy, int proj) {
+    const int z = blockIdx.y;
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (i >= N) return;
+    const float invg = 1.f / (float)g;
+    float v[32];
+    float s = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        int gk = lane + 32 * t;
+        float a = 0.f;
+        if (gk < Gk) {
+            for (int j = 0; j < g; ++j) a += u[(((long long)z * g + j) * N + i) * Gk + gk];
+            a *= invg;
+        }
+        v[t] = a;
+        s += a;
+    }
+    const float mean = warp_sum(s) / (float)Gk;
+    float ss = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+        int gk = lane + 32 * t;
+        v[t] = gk < Gk ? v[t] - mean : 0.f;
+        ss = fmaf(v[t], v[t], ss);
+    }
+    if (proj) {
+        bf16* hr = uhi + ((long long)z * N + i) * Gkp;
+        bf16* lr = ulo + ((long long)z * N + i) * Gkp;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            int gk = lane + 32 * t;
+            if (gk < Gkp) {
+                bf16 hh = __float2bfloat16_rn(v[t]);
+                hr[gk] = hh;
+                lr[gk] = __float2bfloat16_rn(v[t] - __bfloat162float(hh));
+            }
+        }
+    } else {
+        const float nrm = sqrtf(warp_sum(ss));
+        float* yr = y + ((long long)z * N + i) * DPy;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            int gk = lane + 32 * t;
+            if (gk < DPy) yr[gk] = (gk < Gk && nrm > 0.f) ? v[t] / nrm : 0.f;
+        }
+    }
+}
+
+__global__ void rows_normalize_kernel(float* y, int rows, int DP) {
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= rows) return;
+    float* r = y + i * DP;
+    float ss = 0.f;
+    for (int k = 0; k < DP; ++k) ss = fmaf(r[k], r[k], ss);
+    const float nrm = sqrtf(ss);
+    for (int k = 0; k < DP; ++k) r[k] = nrm > 0.f ? r[k] / nrm : 0.f;
+}
+
+__global__ void make_projection_kernel(bf16* projT, int Gk, int Gkp, int rQ, int DPy,
+                                       unsigned long long seed) {
+    long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= (long long)DPy * Gkp) return;
+    int row = (int)(t / Gkp), gk = (int)(t % Gkp);
+    float v = 0.f;
+    if (row < rQ && gk < Gk) {
+        unsigned long long bit = splitmix64(seed ^ (unsigned long long)((long long)gk * rQ + row)) & 1ull;
+        v = bit ? -1.f : 1.f;
+    }
+    projT[t] = __float2bfloat16_rn(v);
+}
+
+// Probe m of a KV head: position p = floor((m+1/2)N/M) of the sequence ordered by
+// (group, radial distance, original index). Rank counting inside the group.
+constexpr int kProbeSmem = 4096;
+__global__ void __launch_bounds__(256) probe_select_kernel(const int32_t* __restrict__ qperm,
+                                                           const int32_t* __restrict__ qoff,
+                                                           const float* __restrict__ radial,
+                                                           int32_t* probe, int32_t* probe_pos,
+                                                           int32_t* probe_seq, int N, int Gq, int M) {
+    const int z = blockIdx.y, m = blockIdx.x;
+    const int32_t* off = qoff + (long long)z * (Gq + 1);
+    const long long p = sample_pos(m, N, M);
+    const int a = upper_index(off, Gq, p);
+    const int lo = off[a], cnt = off[a + 1] - lo;
+    const int k = (int)(p - lo);
+    __shared__ float sr[kProbeSmem];
+    __shared__ int si[kProbeSmem];
+    const int32_t* perm = qperm + (long long)z * N + lo;
+    const float* rad = radial + (long long)z * N;
+    const bool staged = cnt <= kProbeSmem;
+    if (staged) {
+        for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
+            int idx = perm[j];
+            si[j] = idx;
+            sr[j] = rad[idx];
+        }
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
+        const int ij = staged ? si[j] : perm[j];
+        const float rj = staged ? sr[j] : rad[ij];
+        int rank = 0;
+        for (int e = 0; e < cnt; ++e) {
+            const int ie = staged ? si[e] : perm[e];
+            const float re = staged ? sr[e] : rad[ie];
+            rank += (re < rj || (re == rj && ie < ij)) ? 1 : 0;
+        }
+        if (rank == k) {
+            probe[(long long)z * M + m] = ij;
+            probe_pos[(long long)z * M + m] = lo + j;
+            probe_seq[(long long)z * M + m] = (int)p;
+        }
+    }
+}
+
+// Coverage weight of probe m: its group's size split over the group's probes, plus the
+// sizes of probe-less groups whose nearest probe (sequence distance, ties -> lower m) is m.
+__global__ void probe_weights_kernel(const int32_t* __restrict__ qoff,
+                                     const int32_t* __restrict__ probe_seq, float* w, int N,
+                                     int Gq, int M, int uniform) {
+    const int z = blockIdx.x;
+    const int32_t* off = qoff + (long long)z * (Gq + 1);
+    const int32_t* ps = probe_seq + (long long)z * M;
+    for (int m = threadIdx.x; m < M; m += blockDim.x) {
+        if (uniform) { w[(long long)z * M + m] = 1.f; continue; }
+        const int pm = ps[m];
+        const int am = upper_index(off, Gq, pm);
+        const int lo = off[am], hi = off[am + 1];
+        int count = 0;
+        for (int t = 0; t < M; ++t) count += (ps[t] >= lo && ps[t] < hi) ? 1 : 0;
+        float raw = (float)(hi - lo) / (float)count;
+        // probe-less groups before a_m (after the previous probe's group)
+        const int abeg = m > 0 ? upper_index(off, Gq, ps[m - 1]) + 1 : 0;
+        for (int a = abeg; a < am; ++a) {
+            const int glo = off[a], ghi = off[a + 1];
+            if (ghi <= glo) continue;
+            const long long dm = (long long)pm - (ghi - 1);
+            const long long dprev = m > 0 ? (long long)glo - ps[m - 1] : LLONG_MAX;
+            if (dm < dprev) raw += (float)(ghi - glo);
+        }
+        // probe-less groups after a_m (before the next probe's group)
+        const int aend = m + 1 < M ? upper_index(off, Gq, ps[m + 1]) : Gq;
+        for (int a = am + 1; a < aend; ++a) {
+            const int glo = off[a], ghi = off[a + 1];
+            if (ghi <= glo) continue;
+            const long long dm = (long long)glo - pm;
+            const long long dnext = m + 1 < M ? (long long)ps[m + 1] - (ghi - 1) : LLONG_MAX;
+            if (dm <= dnext) raw += (float)(ghi - glo);
+        }
+        w[(long long)z * M + m] = raw * (float)M / (float)N;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gather_samples(const bf16* Q, bf16* Qs, int B, int Hq, int Hkv, int N, int d,
+                                  int S, int DP, cudaStream_t s) {
+    gather_samples_kernel<<<B * Hkv, 256, 0, s>>>(Q, Qs, Hq, Hkv, N, d, S, DP);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_coords_center(const float* u, bf16* uhi, bf16* ulo, float* y, int P, int g,
+                                 int N, int Gk, int Gkp, int DPy, bool proj, cudaStream_t s) {
+    dim3 grid((N + 7) / 8, P);
+    coords_center_kernel<<<grid, 256, 0, s>>>(u, uhi, ulo, y, g, N, Gk, Gkp, DPy, proj ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rows_normalize(float* y, int rows, int DP, cudaStream_t s) {
+    rows_normalize_kernel<<<(rows + 255) / 256, 256, 0, s>>>(y, rows, DP);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_make_projection(bf16* projT, int Gk, int Gkp, int rQ, int DPy,
+                                   unsigned long long seed, cudaStream_t s) {
+    long long tot = (long long)DPy * Gkp;
+    make_projection_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(projT, Gk, Gkp, rQ, DPy, seed);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_probe_select(const int32_t* qperm, const int32_t* qoff, const float* radial,
+                                int32_t* probe, int32_t* probe_pos, int32_t* probe_seq, int P,
+                                int N, int Gq, int M, cudaStream_t s) {
+    if (M <= 0) return cudaSuccess;
+    probe_select_kernel<<<dim3(M, P), 256, 0, s>>>(qperm, qoff, radial, probe, probe_pos, probe_seq, N, Gq, M);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_probe_weights(const int32_t* qoff, const int32_t* probe_seq, float* w, int P,
+                                 int N, int Gq, int M, bool uniform, cudaStream_t s) {
+    if (M <= 0) return cudaSuccess;
+    probe_weights_kernel<<<P, 128, 0, s>>>(qoff, probe_seq, w, N, Gq, M, uniform ? 1 : 0);
+    return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -1,0 +1,114 @@
+// Internal host-side launchers of the SparsePR kernels. Every launcher only
+// enqueues work on `s` and returns the launch error (cudaSuccess on success).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace spr {
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------- dense bf16 GEMM
+// C[z][m][n] = alpha * sum_k (A1[z][m][k] B1[zb][n][k] + A2[z][m][k] B2[zb][n][k]),
+// zb = z / bdiv. A2/B2 may be null (single term). K % 8 == 0, lda/ldb % 8 == 0.
+struct GemmArgs {
+    const bf16* A1; const bf16* A2; long long sA; int lda;
+    const bf16* B1; const bf16* B2; long long sB; int ldb; int bdiv;
+    float* C; long long sC; int ldc;
+    int M, N, K, batch;
+    float alpha;
+};
+cudaError_t launch_gemm_bf16(const GemmArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- k-means + group-major order
+// X: [P][n][DP] fp32 rows (DP in {16,32,48,64}); C: [P][G][DP]; labels/dist: [P][n].
+cudaError_t launch_km_seed(const float* X, float* C, int P, int n, int G, int DP, cudaStream_t s);
+cudaError_t launch_km_assign(const float* X, const float* C, int32_t* labels, float* dist,
+                             int* changed, const int* done, int P, int n, int G, int DP, bool first,
+                             cudaStream_t s);
+cudaError_t launch_km_update(const float* X, const int32_t* perm, const int32_t* off, float* C,
+                             const int* done, int P, int n, int G, int DP, cudaStream_t s);
+cudaError_t launch_km_check(int* changed, int* done, int P, cudaStream_t s);
+cudaError_t launch_km_reset(int* changed, int* done, int P, cudaStream_t s);
+// Stable counting sort of labels [P][n] into perm [P][n] and off [P][G+1].
+// counts/bases: [P][ceil(n/256)][G] scratch. done may be null (always run).
+cudaError_t launch_group_sort(const int32_t* labels, int32_t* perm, int32_t* off, int* counts,
+                              int* bases, const int* done, int P, int n, int G, cudaStream_t s);
+// Mean of the bf16 rows Y [P][n][d] per group (perm/off order); empty -> 0. Also writes a
+// bf16 hi/lo split of the means (hi = bf16(c), lo = bf16(c - hi)) when chi/clo are non-null.
+cudaError_t launch_group_mean_bf16(const bf16* Y, const int32_t* perm, const int32_t* off,
+                                   float* cent, bf16* chi, bf16* clo, int P, int n, int G, int d,
+                                   cudaStream_t s);
+// Split fp32 group means into bf16 hi/lo (used when the partition is handed in).
+cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long count, cudaStream_t s);
+
+// ---------------------------------------------------------------- responses and coordinates
+// Qs[z][s][:] = Q[b][h*g + s%g][floor((s+1/2)N/S)][:] for s < S, zero rows up to DP.
+cudaError_t launch_gather_samples(const bf16* Q, bf16* Qs, int B, int Hq, int Hkv, int N, int d,
+                                  int S, int DP, cudaStream_t s);
+// Mean over the g query heads of u, centred over the Gk groups. If proj: write bf16 hi/lo
+// [P][N][Gkp]; else write the L2-normalised rows into y [P][N][DPy].
+cudaError_t launch_coords_center(const float* u, bf16* uhi, bf16* ulo, float* y, int P, int g,
+                                 int N, int Gk, int Gkp, int DPy, bool proj, cudaStream_t s);
+cudaError_t launch_rows_normalize(float* y, int rows, int DP, cudaStream_t s);
+// projT [DPy][Gkp] bf16 = +-1 with the sign of bit 0 of splitmix64(seed ^ (g*rQ + t)).
+cudaError_t launch_make_projection(bf16* projT, int Gk, int Gkp, int rQ, int DPy,
+                                   unsigned long long seed, cudaStream_t s);
+
+// ---------------------------------------------------------------- probes
+// Probe rows: systematic positions of the radial-ordered group-major sequence.
+cudaError_t launch_probe_select(const int32_t* qperm, const int32_t* qoff, const float* radial,
+                                int32_t* probe, int32_t* probe_pos, int32_t* probe_seq, int P,
+                                int N, int Gq, int M, cudaStream_t s);
+cudaError_t launch_probe_weights(const int32_t* qoff, const int32_t* probe_seq, float* w, int P,
+                                 int N, int Gq, int M, bool uniform, cudaStream_t s);
+
+// ---------------------------------------------------------------- routing
+cudaError_t launch_row_lse(const float* u, const int32_t* koff, float* lse, int Hp, int g, int N,
+                           int Gk, cudaStream_t s);
+cudaError_t launch_cell_scores(const float* u, const float* lse, const int32_t* qperm,
+                               const int32_t* qoff, const int32_t* koff, float* scores, int P,
+                               int g, int N, int Gq, int Gk, cudaStream_t s);
+cudaError_t launch_route_select(const float* scores, const int32_t* qoff, const int32_t* koff,
+                                int32_t* rowptr, int32_t* kg, int64_t* pairs, int P, int Gq,
+                                int Gk, long long budget, bool keep_all, cudaStream_t s);
+
+// ---------------------------------------------------------------- permutation
+// dst[z][p][:] = src[z][perm[z / div][p]][:] for rows of d bf16 (d % 8 == 0).
+cudaError_t launch_permute_rows(const bf16* src, bf16* dst, const int32_t* perm, int Z, int div,
+                                int N, int d, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+// Per-pair tile offsets of the query groups: tile_off[z][a] = sum_{a'<a} ceil(|Q_a'| / bm).
+cudaError_t launch_tile_offsets(const int32_t* qoff, int32_t* tile_off, int P, int Gq, int bm,
+                                cudaStream_t s);
+// Block-sparse attention over group-major Qp/Kp/Vp with the route CSR.
+cudaError_t launch_attn_sparse(const bf16* Qp, const bf16* Kp, const bf16* Vp,
+                               const int32_t* qoff, const int32_t* koff, const int32_t* tile_off,
+                               const int32_t* rowptr, const int32_t* kg, bf16* O, float* lse,
+                               int B, int Hq, int Hkv, int N, int d, int Gq, int Gk,
+                               cudaStream_t s);
+// Dense attention of every query over all keys.
+cudaError_t launch_attn_dense(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse,
+                              int B, int Hq, int Hkv, int N, int d, cudaStream_t s);
+// Dense attention of gathered probe rows, split over ns key chunks, then combined.
+cudaError_t launch_attn_probe(const bf16* Q, const bf16* K, const bf16* V, const int32_t* probe,
+                              float* Opart, float* mpart, float* lpart, float* Odense, int B,
+                              int Hq, int Hkv, int N, int d, int M, int ns, cudaStream_t s);
+
+// ---------------------------------------------------------------- probe fit + write-back
+cudaError_t launch_probe_residual(const float* Odense, const bf16* Osp, const int32_t* probe_pos,
+                                  float* R, float* Osp_probe, int Hp, int g, int N, int d, int M,
+                                  cudaStream_t s);
+cudaError_t launch_fit(const float* R, const float* Xp, const float* w, float lambda, float* obar,
+                       float* Rbar, float* A, float* U, float* Bm, float* c0, int32_t* rank,
+                       int Hp, int g, int d, int M, int r, int* status, cudaStream_t s);
+cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float* U,
+                             const float* Bm, const float* c0, bf16* O, int Hp, int g, int N,
+                             int d, int r, bool correct, cudaStream_t s);
+cudaError_t launch_probe_override(const float* Odense, const int32_t* probe, bf16* O, int Hp,
+                                  int g, int N, int d, int M, cudaStream_t s);
+
+}  // namespace spr

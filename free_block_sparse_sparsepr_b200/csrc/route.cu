@@ -1,0 +1,261 @@
+// Routing of (query group, key group) cells to the execution-density budget:
+// per-row log-normaliser over the key groups, cell scores (estimated softmax
+// weight of one key of group g for a query of group a, averaged over the
+// group's queries and the KV head's query heads), then whole-cell selection.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spr {
+namespace {
+
+// lse[x][i] = log sum_{g: |K_g| > 0} |K_g| exp(u[x][i][g]); one warp per row.
+__global__ void row_lse_kernel(const float* __restrict__ u, const int32_t* __restrict__ koff,
+                               float* lse, int g, int N, int Gk) {
+    const int x = blockIdx.y, z = x / g;
+    const int lane = threadIdx.x & 31;
+    const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (i >= N) return;
+    const float* ur = u + ((long long)x * N + i) * Gk;
+    const int32_t* ko = koff + (long long)z * (Gk + 1);
+    float m = -FLT_MAX;
+    for (int gk = lane; gk < Gk; gk += 32)
+        if (ko[gk + 1] > ko[gk]) m = fmaxf(m, ur[gk]);
+    m = warp_max(m);
+    float s = 0.f;
+    for (int gk = lane; gk < Gk; gk += 32) {
+        int sz = ko[gk + 1] - ko[gk];
+        if (sz > 0) s += (float)sz * expf(ur[gk] - m);
+    }
+    s = warp_sum(s);
+    if (lane == 0) lse[(long long)x * N + i] = m + logf(s);
+}
+
+// scores[z][a][g] = mean over the g heads and the queries of group a of exp(u - lse).
+__global__ void cell_scores_kernel(const float* __restrict__ u, const float* __restrict__ lse,
+                                   const int32_t* __restrict__ qperm, const int32_t* __restrict__ qoff,
+                                   const int32_t* __restrict__ koff, float* scores, int g, int N,
+                                   int Gq, int Gk) {
+    const int z = blockIdx.y, a = blockIdx.x;
+    const int lo = qoff[(long long)z * (Gq + 1) + a], hi = qoff[(long long)z * (Gq + 1) + a + 1];
+    const int32_t* ko = koff + (long long)z * (Gk + 1);
+    const int32_t* perm = qperm + (long long)z * N;
+    for (int gk = threadIdx.x; gk < Gk; gk += blockDim.x) {
+        float acc = 0.f;
+        const bool ok = hi > lo && ko[gk + 1] > ko[gk];
+        if (ok) {
+            for (int j = 0; j < g; ++j) {
+                const long long x = (long long)z * g + j;
+                const float* ux = u + x * N * Gk;
+                const float* lx = lse + x * N;
+                for (int p = lo; p < hi; ++p) {
+                    int i = perm[p];
+                    acc += expf(ux[(long long)i * Gk + gk] - lx[i]);
+                }
+            }
+        }
+        scores[((long long)z * Gq + a) * Gk + gk] = ok ? acc / ((float)g * (float)(hi - lo)) : 0.f;
+    }
+}
+
+// One CTA per (batch, KV head). Each non-empty query group keeps its top cell; the other
+// eligible cells are ordered by key = (~score_bits << 32 | a*Gk + g) (descending score, then
+// ascending a, g) and a cost-weighted radix select finds the first cell whose inclusion would
+// exceed the remaining budget; it is kept iff its overshoot < the remaining undershoot.
+constexpr int kSelThreads = 1024;
+__global__ void __launch_bounds__(kSelThreads) route_select_kernel(
+    const float* __restrict__ scores, const int32_t* __restrict__ qoff, const int32_t* __restrict__ koff,
+    int32_t* rowptr, int32_t* kg, int64_t* pairs, int Gq, int Gk, long long budget, int keep_all) {
+    const int z = blockIdx.x;
+    extern __shared__ int sm[];
+    int* qs = sm;             // [Gq]
+    int* ks = qs + Gq;        // [Gk]
+    int* mand = ks + Gk;      // [Gq]
+    int* rowcnt = mand + Gq;  // [Gq]
+    __shared__ unsigned long long hist[256];
+    __shared__ long long red[32];
+    __shared__ long long s_rem;
+    __shared__ unsigned long long s_prefix, s_mask;
+    __shared__ int s_found;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const float* S = scores + (long long)z * Gq * Gk;
+    for (int a = tid; a < Gq; a += blockDim.x)
+        qs[a] = qoff[(long long)z * (Gq + 1) + a + 1] - qoff[(long long)z * (Gq + 1) + a];
+    for (int gk = tid; gk < Gk; gk += blockDim.x)
+        ks[gk] = koff[(long long)z * (Gk + 1) + gk + 1] - koff[(long long)z * (Gk + 1) + gk];
+    __syncthreads();
+
+    // Mandatory cell per query group: argmax score over eligible key groups, ties -> lowest g.
+    for (int a = warp; a < Gq; a += nw) {
+        float best = -FLT_MAX;
+        int bg = -1;
+        if (qs[a] > 0) {
+            for (int gk = lane; gk < Gk; gk += 32) {
+                if (ks[gk] > 0) {
+                    float v = S[(long long)a * Gk + gk];
+                    if (bg < 0 || v > best) { best = v; bg = gk; }
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(kFull, best, o);
+            int og = __shfl_xor_sync(kFull, bg, o);
+            if (og >= 0 && (bg < 0 || ov > best || (ov == best && og < bg))) { best = ov; bg = og; }
+        }
+        if (lane == 0) mand[a] = bg;
+    }
+    __syncthreads();
+
+    // Cost of the mandatory cells.
+    long long loc = 0;
+    for (int a = tid; a < Gq; a += blockDim.x)
+        if (mand[a] >= 0) loc += (long long)qs[a] * ks[mand[a]];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) loc += __shfl_xor_sync(kFull, loc, o);
+    if (lane == 0) red[warp] = loc;
+    __syncthreads();
+    if (tid == 0) {
+        long long b = 0;
+        for (int w = 0; w < nw; ++w) b += red[w];
+        s_rem = budget - b;
+        s_prefix = 0ull;
+        s_mask = 0ull;
+        s_found = keep_all ? 0 : 1;
+    }
+    __syncthreads();
+
+    const long long ncell = (long long)Gq * Gk;
+    if (!keep_all) {
+        for (int shift = 56; shift >= 0; shift -= 8) {
+            for (int t = tid; t < 256; t += blockDim.x) hist[t] = 0ull;
+            __syncthreads();
+            const unsigned long long prefix = s_prefix, mask = s_mask;
+            for (long long c = tid; c < ncell; c += blockDim.x) {
+                const int a = (int)(c / Gk), gk = (int)(c % Gk);
+                if (qs[a] == 0 || ks[gk] == 0 || mand[a] == gk) continue;
+                const unsigned long long key =
+                    ((unsigned long long)(~__float_as_uint(S[c])) << 32) | (unsigned long long)c;
+                if ((key & mask) != prefix) continue;
+                atomicAdd(&hist[(key >> shift) & 255ull], (unsigned long long)((long long)qs[a] * ks[gk]));
+            }
+            __syncthreads();
+            if (tid == 0) {
+                long long cum = 0;
+                int dsel = -1;
+                for (int dg = 0; dg < 256; ++dg) {
+                    long long h = (long long)hist[dg];
+                    if (h > 0 && cum + h > s_rem) { dsel = dg; break; }
+                    cum += h;
+                }
+                if (dsel < 0) {
+                    s_found = 0;  // every remaining candidate fits in the budget
+                } else {
+                    s_rem -= cum;
+                    s_prefix |= (unsigned long long)dsel << shift;
+                    s_mask |= 255ull << shift;
+                }
+            }
+            __syncthreads();
+            if (!s_found) break;
+        }
+    }
+    const int found = s_found;
+    const unsigned long long kstar = s_prefix;
+    const long long under = s_rem;
+    bool take_star = false;
+    if (found) {
+        const long long cstar = (long long)(kstar & 0xffffffffull);
+        const long long cost = (long long)qs[cstar / Gk] * ks[cstar % Gk];
+        take_star = (cost - under) < under;
+    }
+
+    // Row counts, then CSR in ascending key-group order.
+    long long psum = 0;
+    for (int a = warp; a < Gq; a += nw) {
+        int cnt = 0;
+        for (int g0 = 0; g0 < Gk; g0 += 32) {
+            const int gk = g0 + lane;
+            bool sel = false;
+            if (gk < Gk && qs[a] > 0 && ks[gk] > 0) {
+                const long long c = (long long)a * Gk + gk;
+                if (keep_all || mand[a] == gk || !found) {
+                    sel = true;
+                } else {
+                    const unsigned long long key =
+                        ((unsigned long long)(~__float_as_uint(S[c])) << 32) | (unsigned long long)c;
+                    sel = key < kstar || (key == kstar && take_star);
+                }
+            }
+            const unsigned b = __ballot_sync(kFull, sel);
+            cnt += __popc(b);
+            if (sel) psum += (long long)qs[a] * ks[gk];
+        }
+        if (lane == 0) rowcnt[a] = cnt;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(kFull, psum, o);
+    __syncthreads();
+    if (lane == 0) red[warp] = psum;
+    __syncthreads();
+    if (tid == 0) {
+        long long tot = 0;
+        for (int w = 0; w < nw; ++w) tot += red[w];
+        pairs[z] = tot;
+        int s = 0;
+        int32_t* rp = rowptr + (long long)z * (Gq + 1);
+        for (int a = 0; a < Gq; ++a) { int v = rowcnt[a]; rp[a] = s; rowcnt[a] = s; s += v; }
+        rp[Gq] = s;
+    }
+    __syncthreads();
+    int32_t* kz = kg + (long long)z * Gq * Gk;
+    for (int a = warp; a < Gq; a += nw) {
+        int base = rowcnt[a];
+        for (int g0 = 0; g0 < Gk; g0 += 32) {
+            const int gk = g0 + lane;
+            bool sel = false;
+            if (gk < Gk && qs[a] > 0 && ks[gk] > 0) {
+                const long long c = (long long)a * Gk + gk;
+                if (keep_all || mand[a] == gk || !found) {
+                    sel = true;
+                } else {
+                    const unsigned long long key =
+                        ((unsigned long long)(~__float_as_uint(S[c])) << 32) | (unsigned long long)c;
+                    sel = key < kstar || (key == kstar && take_star);
+                }
+            }
+            const unsigned b = __ballot_sync(kFull, sel);
+            if (sel) kz[base + __popc(b & ((1u << lane) - 1u))] = gk;
+            base += __popc(b);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_row_lse(const float* u, const int32_t* koff, float* lse, int Hp, int g, int N,
+                           int Gk, cudaStream_t s) {
+    dim3 grid((N + 7) / 8, Hp);
+    row_lse_kernel<<<grid, 256, 0, s>>>(u, koff, lse, g, N, Gk);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cell_scores(const float* u, const float* lse, const int32_t* qperm,
+                               const int32_t* qoff, const int32_t* koff, float* scores, int P,
+                               int g, int N, int Gq, int Gk, cudaStream_t s) {
+    cell_scores_kernel<<<dim3(Gq, P), 256, 0, s>>>(u, lse, qperm, qoff, koff, scores, g, N, Gq, Gk);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_select(const float* scores, const int32_t* qoff, const int32_t* koff,
+                                int32_t* rowptr, int32_t* kg, int64_t* pairs, int P, int Gq,
+                                int Gk, long long budget, bool keep_all, cudaStream_t s) {
+    size_t smem = (size_t)(3 * Gq + Gk) * sizeof(int);
+    route_select_kernel<<<P, kSelThreads, smem, s>>>(scores, qoff, koff, rowptr, kg, pairs, Gq, Gk,
+                                                     budget, keep_all ? 1 : 0);
+    return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -1,0 +1,281 @@
+"""GPU parity: every step of the CUDA path against the CPU oracle on the same
+seeded inputs, through the C ABI. Tolerances: bf16 outputs with fp32
+accumulation match within max-abs 2e-2 and mean-abs 2e-3; permutations,
+offsets and (where the oracle's partition is handed in) selected cells are
+exact; end-to-end partitions agree on >= 99% of rows whose k-means margin
+exceeds 1e-3."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import free_block_sparse_sparsepr_b200 as spr  # noqa: E402
+from synthetic import Workload, get_workload  # noqa: E402
+from gpu_helpers import (MAX_ABS, MEAN_ABS, assert_close, bf16_to_f64, err, inputs, kmeans_margin,  # noqa: E402
+                         partition_tensors, route_tensors, selected_from_csr, to_group_major)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny_n1024": get_workload("tiny_n1024"),
+    "mid_n16384_h4": get_workload("mid_n16384").replace(Hq=4, Hkv=4),
+    # ragged: N=1000 (not a multiple of any tile), GQA 4 query heads on 2 KV heads, B=2
+    "ragged_gqa_n1000": Workload("ragged_gqa_n1000", B=2, Hq=4, Hkv=2, T=5, Hg=10, Wg=20, d=128, Gk=13, Gq=7,
+                                 block=64, rho=0.3, M=40, r=8, locality=0.8, noise=0.4),
+    # ragged d=64: N=777, more query groups than key groups
+    "ragged_d64_n777": Workload("ragged_d64_n777", B=1, Hq=3, Hkv=3, T=3, Hg=7, Wg=37, d=64, Gk=20, Gq=24,
+                                block=64, rho=0.35, M=32, r=12),
+    # Gk > rQ: the query coordinates go through the +-1 projection
+    "proj_n4096": Workload("proj_n4096", B=1, Hq=2, Hkv=2, T=4, Hg=32, Wg=32, d=128, Gk=96, Gq=80, block=128,
+                           rho=0.25, locality=1.2),
+}
+
+_cache = {}
+
+
+def _setup(name):
+    if name not in _cache:
+        w = CASES[name]
+        host, dev = inputs(w)
+        res = oracle.sparsepr_attention(*host, w)
+        _cache[name] = (w, host, dev, res)
+    return _cache[name]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    spr.load_library()
+    yield
+    _cache.clear()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_dense_attention_matches_oracle(name):
+    w, (Q, K, V), (q, k, v), _ = _setup(name)
+    with spr.SparsePR.from_workload(w) as h:
+        O = h.dense_attn(q, k, v)
+        torch.cuda.synchronize()
+        rows = np.arange(w.N) if w.N <= 4096 else np.unique(oracle.sample_rows(w.N, 512))
+        ref = oracle.dense_attention(Q, K, V, rows=rows)
+        assert_close(bf16_to_f64(O)[:, :, rows], ref, "dense attention")
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_handed_in_partition_and_route(name):
+    """Steps 4-7 with the oracle's partition and route handed in."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    pt = partition_tensors(res, w)
+    rt = route_tensors(res, w)
+    part = spr.partition_from_tensors(pt)
+    route = spr.route_from_tensors(rt)
+    with spr.SparsePR.from_workload(w) as h:
+        Qp, Kp, Vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        h.permute(q, k, v, part, Qp, Kp, Vp)
+        # (4) permutation: bit-exact gathers
+        kperm = pt["kperm"].long()
+        qperm = pt["qperm"].long()
+        for b in range(w.B):
+            for hq in range(w.Hq):
+                z = b * w.Hkv + hq // w.g
+                assert torch.equal(Qp[b, hq], q[b, hq][qperm[z]])
+            for hk in range(w.Hkv):
+                z = b * w.Hkv + hk
+                assert torch.equal(Kp[b, hk], k[b, hk][kperm[z]])
+                assert torch.equal(Vp[b, hk], v[b, hk][kperm[z]])
+        # (5) block-sparse attention, group-major order
+        Osp = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+        h.blocksparse_attn(Qp, Kp, Vp, part, route, Osp, lse)
+        torch.cuda.synchronize()
+        ref_s = to_group_major(res["O_sparse"], res, w)
+        assert_close(bf16_to_f64(Osp), ref_s, "sparse output")
+        ref_lse = to_group_major(res["lse"][..., None], res, w)[..., 0]
+        assert np.abs(lse.cpu().numpy() - ref_lse).max() < 1e-3
+        # (6) probes, residuals, fit
+        fit = h.probe_fit(q, k, v, part, Osp)
+        torch.cuda.synchronize()
+        fv = h.fit_views(fit)
+        R = fv["R"].cpu().numpy().reshape(w.B, w.Hq, w.M, w.d)
+        Od = fv["Odense"].cpu().numpy().reshape(w.B, w.Hq, w.M, w.d)
+        for b in range(w.B):
+            for hq in range(w.Hq):
+                f = res["fits"][(b, hq)]
+                assert_close(Od[b, hq], f.Odense, "probe dense rows", max_abs=2e-3, mean_abs=2e-4)
+                assert_close(R[b, hq], f.R, "probe residual")
+                x = b * w.Hq + hq
+                assert_close(fv["obar"][x].cpu().numpy(), f.obar, "obar", 1e-2, 1e-3)
+                assert_close(fv["Rbar"][x].cpu().numpy(), f.Rbar, "Rbar", 1e-2, 1e-3)
+                s = f.sing
+                rk = int(fv["rank"][x])
+                assert rk == min(w.r, f.U.shape[1]) or rk == w.r
+                if len(s) > w.r and s[w.r - 1] > 1.2 * s[w.r]:       # projector well defined
+                    Ug = fv["U"][x].cpu().numpy().astype(np.float64)
+                    assert np.abs(Ug @ Ug.T - f.U @ f.U.T).max() < 5e-2
+        # (7) correction and write-back
+        O = torch.empty_like(q)
+        h.writeback(part, Osp, fit, O)
+        torch.cuda.synchronize()
+        assert_close(bf16_to_f64(O), res["O"], "corrected output")
+        Of = bf16_to_f64(O)
+        for b in range(w.B):
+            for hq in range(w.Hq):
+                p = res["partitions"][(b, hq // w.g)].probe
+                assert_close(Of[b, hq, p], res["fits"][(b, hq)].Odense, "probe rows = dense rows", 8e-3, 2e-3)
+        assert h.device_status() == 0
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_route_with_oracle_partition(name):
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    part = spr.partition_from_tensors(partition_tensors(res, w))
+    with spr.SparsePR.from_workload(w) as h:
+        route = h.route(q, part)
+        torch.cuda.synchronize()
+        rv = h.route_views(route)
+        for b in range(w.B):
+            for hk in range(w.Hkv):
+                z = b * w.Hkv + hk
+                ro = res["routes"][(b, hk)]
+                S = rv["scores"][z].cpu().numpy()
+                nz = ro.scores > 0
+                rel = np.abs(S.astype(np.float64) - ro.scores) / np.maximum(ro.scores, 1e-30)
+                assert rel[nz].max() < 2e-4, f"scores rel err {rel[nz].max()}"
+                assert np.all(S[~nz] == 0)
+                sel = selected_from_csr(rv["rowptr"][z].cpu().numpy(), rv["kg"][z].cpu().numpy(), w.Gq, w.Gk)
+                diff = sel ^ ro.sel
+                if diff.any():
+                    # only cells at the budget cut whose scores tie within fp32 rounding may differ
+                    free = ~ro.mandatory & (np.outer(np.diff(res["partitions"][(b, hk)].qoff),
+                                                     np.diff(res["partitions"][(b, hk)].koff)) > 0)
+                    cut = ro.scores[ro.sel & free].min() if (ro.sel & free).any() else 0.0
+                    assert np.all(np.abs(ro.scores[diff] - cut) <= 2e-4 * cut), "selected cells differ"
+                else:
+                    assert int(rv["pairs"][z]) == ro.pairs
+                # CSR rows ascending
+                rp = rv["rowptr"][z].cpu().numpy()
+                kgz = rv["kg"][z].cpu().numpy()
+                for a in range(w.Gq):
+                    assert np.all(np.diff(kgz[rp[a]:rp[a + 1]]) > 0)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_partition_end_to_end(name):
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    with spr.SparsePR.from_workload(w) as h:
+        part = h.partition(q, k)
+        torch.cuda.synchronize()
+        pv = {n: t.cpu().numpy() for n, t in h.partition_views(part).items()}
+    for b in range(w.B):
+        for hk in range(w.Hkv):
+            z = b * w.Hkv + hk
+            po = res["partitions"][(b, hk)]
+            # (1) response features, fp32
+            F = pv["features"][z][:, : w.rK]
+            scale = np.abs(po.features).max()
+            assert np.abs(F - po.features).max() <= 1e-5 * scale
+            # (2a) key groups: agreement where the oracle's margin is clear
+            _, Ck, _ = oracle.kmeans(po.features, w.Gk, w.kmeans_iters)
+            mk = kmeans_margin(po.features, Ck) > 1e-3
+            agree_k = (pv["kgroup"][z] == po.kgroup)[mk].mean()
+            assert agree_k >= 0.99, f"key-group agreement {agree_k:.4f}"
+            # (2b) query groups
+            _, Cq, _ = oracle.kmeans(po.ycoord, w.Gq, w.kmeans_iters)
+            mq = kmeans_margin(po.ycoord, Cq) > 1e-3
+            agree_q = (pv["qgroup"][z] == po.qgroup)[mq].mean()
+            assert agree_q >= 0.99, f"query-group agreement {agree_q:.4f}"
+            # (4) group-major orders: the stable sort of the GPU's own labels, bit-exact
+            for lab, perm, off, G in ((pv["kgroup"][z], pv["kperm"][z], pv["koff"][z], w.Gk),
+                                      (pv["qgroup"][z], pv["qperm"][z], pv["qoff"][z], w.Gq)):
+                assert np.array_equal(perm, np.argsort(lab, kind="stable"))
+                assert np.array_equal(off, np.concatenate([[0], np.cumsum(np.bincount(lab, minlength=G))]))
+            if np.array_equal(pv["kgroup"][z], po.kgroup):
+                assert np.array_equal(pv["kperm"][z], po.kperm)
+                assert np.abs(pv["kcent"][z] - po.kcent).max() < 1e-5
+            if np.array_equal(pv["qgroup"][z], po.qgroup):
+                assert np.array_equal(pv["qperm"][z], po.qperm)
+                # probe rows follow from the radial order; equal up to radial near-ties
+                same = (pv["probe"][z] == po.probe).mean()
+                assert same >= 0.9, f"probe rows agree on {same:.2f}"
+            # probe rows: distinct, M of them, systematic positions of the radial sequence
+            pr = pv["probe"][z]
+            assert len(np.unique(pr)) == w.M
+            assert abs(pv["weights"][z].sum() - w.M) < 1e-3
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attention_end_to_end(name):
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    with spr.SparsePR.from_workload(w, flags=spr.FLAG_STAGE_TIMING) as h:
+        O = h.attention(q, k, v)
+        st = h.stats()
+        O2 = h.attention(q, k, v)
+        torch.cuda.synchronize()
+        assert torch.equal(O, O2), "two calls on the same input differ"
+        assert st["device_status"] == 0
+        assert h.last_launch_count() > 10
+        Of = bf16_to_f64(O)
+        # realised density follows the rho_exec formula; whole cells keep it near the target
+        assert abs(st["rho_exec"] - (st["route_density"] + w.M / w.N)) < 1e-12
+        assert abs(st["rho_exec"] - res["rho_exec"]) < 0.02
+        assert st["stage_ms"]["total"] > 0
+        # probe rows of the output are the exact dense rows
+        probes = h.partition_views(h.partition(q, k))["probe"].cpu().numpy()
+        torch.cuda.synchronize()
+        for b in range(w.B):
+            for hq in range(w.Hq):
+                p = probes[b * w.Hkv + hq // w.g]
+                ref, _ = oracle.dense_attention_rows(Q[b, hq, p], K[b, hq // w.g], V[b, hq // w.g])
+                assert_close(Of[b, hq, p], ref, "probe rows = dense rows", 8e-3, 2e-3)
+        # quality relative to dense attention is the oracle's, within rounding
+        D = oracle.dense_attention(Q, K, V) if w.N <= 4096 else None
+        if D is not None:
+            e_gpu = np.abs(Of - D).mean()
+            e_orc = np.abs(res["O"] - D).mean()
+            assert e_gpu <= 1.1 * e_orc + 1e-3, (e_gpu, e_orc)
+        mx, mn = err(Of, res["O"])
+        assert mn <= 5 * MEAN_ABS, f"end-to-end mean-abs {mn}"
+
+
+def test_full_density_equals_dense():
+    w = CASES["ragged_gqa_n1000"].replace(rho=1.0)
+    (Q, K, V), (q, k, v) = inputs(w)
+    with spr.SparsePR.from_workload(w) as h:
+        O = h.attention(q, k, v)
+        Od = h.dense_attn(q, k, v)
+        torch.cuda.synchronize()
+        st = h.stats()
+    assert abs(st["route_density"] - 1.0) < 1e-12
+    D = oracle.dense_attention(Q, K, V)
+    assert_close(bf16_to_f64(O), D, "rho=1 output vs dense")
+    assert_close(bf16_to_f64(Od), D, "dense kernel")
+
+
+def test_hard_drop_only_flag():
+    w = CASES["tiny_n1024"]
+    (Q, K, V), (q, k, v) = inputs(w)
+
+    class Cfg:
+        pass
+
+    cfg = Cfg()
+    for f in ("rK", "Gk", "Gq", "rQ", "M", "r", "lam", "rho", "kmeans_iters", "seed"):
+        setattr(cfg, f, getattr(w, f))
+    cfg.flags = oracle.FLAG_HARD_DROP_ONLY
+    res = oracle.sparsepr_attention(Q, K, V, cfg)
+    pt = partition_tensors(res, w.replace(M=0))
+    rt = route_tensors(res, w)
+    with spr.SparsePR.from_workload(w, flags=spr.FLAG_HARD_DROP_ONLY) as h:
+        part, route = spr.partition_from_tensors(pt), spr.route_from_tensors(rt)
+        Qp, Kp, Vp, Osp, O = (torch.empty_like(t) for t in (q, k, v, q, q))
+        h.permute(q, k, v, part, Qp, Kp, Vp)
+        h.blocksparse_attn(Qp, Kp, Vp, part, route, Osp)
+        h.writeback(part, Osp, None, O)
+        torch.cuda.synchronize()
+        assert_close(bf16_to_f64(O), res["O"], "hard-drop output")
+        O2 = h.attention(q, k, v)
+        torch.cuda.synchronize()
+        st = h.stats()
+        assert abs(st["rho_exec"] - st["route_density"]) < 1e-12
