@@ -268,6 +268,9 @@ def run_ours(args):
 
     # timed region: K calls, per-stage events of every call on the launching stream
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for row in evs:            # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()

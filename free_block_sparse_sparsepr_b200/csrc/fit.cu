@@ -275,24 +275,31 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     if (tid == 0) rank_out[x] = rank;
 }
 
-// O[qperm[p]] = Osp[p] + U (c0 + Bm Osp[p]); one warp per group-major row.
-template <int D>
+// O[qperm[p]] = Osp[p] + U (c0 + Bm Osp[p]); one warp per group-major row. Each lane holds
+// EPL consecutive elements; Bm and U^T are staged row-major in shared memory so every
+// vector load is conflict-free. The RP partial dot products are reduced by recursive
+// halving (RP/2 + ... + 1 + 1 shuffles); afterwards lane 2k holds t_k.
+template <int D, int RP>
 __global__ void __launch_bounds__(256) writeback_kernel(const bf16* __restrict__ Osp,
                                                         const int32_t* __restrict__ qperm,
                                                         const float* __restrict__ U,
                                                         const float* __restrict__ Bm,
                                                         const float* __restrict__ c0, bf16* O,
                                                         int g, int N, int r, int correct) {
-    constexpr int EPL = D / 32;   // elements per lane
+    constexpr int EPL = D / 32;
+    static_assert(RP == 16 || RP == 32, "RP");
     const int x = blockIdx.y, z = x / g;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __shared__ float sU[D * 32];
-    __shared__ float sB[32 * D];
-    __shared__ float sc[32];
+    __shared__ __align__(16) float sB[RP * D];    // Bm[k][c]
+    __shared__ __align__(16) float sUt[RP * D];   // U[c][k] transposed to [k][c]
+    __shared__ float sc[RP];
     if (correct) {
-        for (int t = threadIdx.x; t < D * r; t += blockDim.x) sU[t] = U[(long long)x * D * r + t];
-        for (int t = threadIdx.x; t < r * D; t += blockDim.x) sB[t] = Bm[(long long)x * r * D + t];
-        for (int t = threadIdx.x; t < r; t += blockDim.x) sc[t] = c0[(long long)x * r + t];
+        for (int t = threadIdx.x; t < RP * D; t += blockDim.x) {
+            const int k = t / D, c = t % D;
+            sB[t] = k < r ? Bm[((long long)x * r + k) * D + c] : 0.f;
+            sUt[t] = k < r ? U[((long long)x * D + c) * r + k] : 0.f;
+        }
+        for (int t = threadIdx.x; t < RP; t += blockDim.x) sc[t] = t < r ? c0[(long long)x * r + t] : 0.f;
     }
     __syncthreads();
     const int32_t* perm = qperm + (long long)z * N;
@@ -300,27 +307,42 @@ __global__ void __launch_bounds__(256) writeback_kernel(const bf16* __restrict__
         const bf16* src = Osp + ((long long)x * N + p) * D + lane * EPL;
         float o[EPL];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) o[e] = __bfloat162float(src[e]);
+        for (int e = 0; e < EPL; e += 2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + e));
+            o[e] = f.x;
+            o[e + 1] = f.y;
+        }
         if (correct) {
-            float t[32];
+            float a[RP];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                float a = 0.f;
-                if (k < r) {
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) a = fmaf(sB[k * D + lane * EPL + e], o[e], a);
-                    a = warp_sum(a) + sc[k];
-                }
-                t[k] = a;
-            }
-            float delta[EPL];
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) {
+            for (int k = 0; k < RP; ++k) {
                 float acc = 0.f;
 #pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    if (k < r) acc = fmaf(sU[(lane * EPL + e) * r + k], t[k], acc);
-                delta[e] = acc;
+                for (int e = 0; e < EPL; ++e) acc = fmaf(sB[k * D + lane * EPL + e], o[e], acc);
+                a[k] = acc;
+            }
+            // Step with lane bit b: lanes with b set keep the upper half of the remaining
+            // partials (adding the partner's upper half), the others the lower half.
+#pragma unroll
+            for (int n = RP, bit = 16; n > 1; n >>= 1, bit >>= 1) {
+                const bool up = (lane & bit) != 0;
+#pragma unroll
+                for (int i = 0; i < n / 2; ++i) {
+                    const float send = up ? a[i] : a[i + n / 2];
+                    const float keep = up ? a[i + n / 2] : a[i];
+                    a[i] = keep + __shfl_xor_sync(kFull, send, bit);
+                }
+            }
+            if (RP == 16) a[0] += __shfl_xor_sync(kFull, a[0], 1);   // lanes 2k, 2k+1 held halves of t_k
+            const float tk = a[0];
+            float delta[EPL];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) delta[e] = 0.f;
+#pragma unroll
+            for (int k = 0; k < RP; ++k) {
+                const float t = __shfl_sync(kFull, tk, (RP == 16) ? 2 * k : k) + sc[k];
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) delta[e] = fmaf(sUt[k * D + lane * EPL + e], t, delta[e]);
             }
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o[e] += delta[e];
@@ -372,9 +394,16 @@ cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float*
                              int d, int r, bool correct, cudaStream_t s) {
     const int blocks = (N + 8 * 16 - 1) / (8 * 16);   // 16 rows per warp
     dim3 grid(blocks, Hp);
-    if (d == 64) writeback_kernel<64><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, correct ? 1 : 0);
-    else if (d == 128) writeback_kernel<128><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, correct ? 1 : 0);
-    else return cudaErrorInvalidValue;
+    const int cf = correct ? 1 : 0;
+    if (r <= 16) {
+        if (d == 64) writeback_kernel<64, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
+        else if (d == 128) writeback_kernel<128, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
+        else return cudaErrorInvalidValue;
+    } else {
+        if (d == 64) writeback_kernel<64, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
+        else if (d == 128) writeback_kernel<128, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
+        else return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 

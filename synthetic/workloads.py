@@ -90,6 +90,10 @@ def stack_layer_locality(layer: int, seed: int = 0) -> float:
 
 
 def get_workload(name: str) -> Workload:
+    """A named workload, or a sweep point named sweep_n<N>_rho<percent>."""
     if name in WORKLOADS:
         return WORKLOADS[name]
-    raise KeyError(f"unknown workload {name!r}; known: {sorted(WORKLOADS)}")
+    if name.startswith("sweep_n") and "_rho" in name:
+        n_part, rho_part = name[len("sweep_n"):].split("_rho")
+        return sweep_workload(int(n_part), int(rho_part) / 100.0)
+    raise KeyError(f"unknown workload {name!r}; known: {sorted(WORKLOADS)} or sweep_n<N>_rho<pct>")
