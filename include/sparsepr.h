@@ -302,6 +302,32 @@ sparsepr_status sparsepr_device_status(sparsepr_handle h, int* out);
  */
 sparsepr_status sparsepr_set_stage_events(sparsepr_handle h, void* const* events);
 
+/*
+ * Allocation-free dense attention of given query rows (the probe-row pass of
+ * sparsepr_probe_fit without a handle). The paper has no counterpart: this
+ * entry point exists for callers that cannot call cudaMalloc -- code inside a
+ * framework whose memory manager owns every device allocation, code that runs
+ * while an allocator lock is held, or a process that reserves its device
+ * memory up front. It allocates nothing: the caller passes inputs and outputs,
+ * and the split-key partial results go to a fixed 8 MiB array compiled into the
+ * library (every GPU that loads the library holds it until the process exits).
+ *   Q        bf16 [B][Hq][N][d], K and V bf16 [B][Hkv][N][d] (device, 16-byte aligned)
+ *   rows     int32 [B*Hkv][M]: original query rows, shared by the KV head's query heads
+ *   O        fp32 [B*Hq][M][d] (device, caller-owned): softmax(q K^T / sqrt(d)) V per row
+ *   d in {64, 128}, 1 <= M <= min(N, 64)
+ * Limit: B*Hq*M*(d+2)*4 bytes must fit in the 8 MiB array (e.g. 24 heads x 64
+ * rows x d=128 uses 0.8 MB per key split, so 10 splits); larger requests return
+ * SPARSEPR_ERR_UNSUPPORTED without touching the device. The first call on a
+ * device looks up the array's device address on that device (cudaGetSymbolAddress,
+ * with the device current), so make that first call before any stream capture.
+ * Every call uses the same array: calls whose work overlaps on a GPU (two streams,
+ * two threads) race on it and must be serialised by the caller. No part of the
+ * array needs to start at zero: each call writes every slot it later reads.
+ */
+sparsepr_status sparsepr_probe_attention_noalloc(const void* Q, const void* K, const void* V,
+                                                 const int32_t* rows, float* O, int B, int Hq, int Hkv,
+                                                 int N, int d, int M, void* stream);
+
 /* Number of kernel launches the last sparsepr_attention call enqueued. */
 sparsepr_status sparsepr_last_launch_count(sparsepr_handle h, int* out);
 
