@@ -262,6 +262,12 @@ sparsepr_status attn_impl(sparsepr_handle h, const bf16* Qp, const bf16* Kp, con
                           const sparsepr_partition_t* p, const sparsepr_route_t* r, bf16* Osp, float* lse,
                           cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
+    if (spr::attn_tc_supported(c.d)) {
+        SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, 128, s));
+        SPR_TRY(spr::launch_attn_sparse_tc(Qp, Kp, Vp, p->qoff, p->koff, h->tile_off, r->rowptr, r->kg, Osp, lse,
+                                           c.B, c.Hq, c.Hkv, c.N, c.Gq, c.Gk, h->dev_status, s));
+        return SPARSEPR_OK;
+    }
     SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, 64, s));
     SPR_TRY(spr::launch_attn_sparse(Qp, Kp, Vp, p->qoff, p->koff, h->tile_off, r->rowptr, r->kg, Osp, lse,
                                     c.B, c.Hq, c.Hkv, c.N, c.d, c.Gq, c.Gk, s));
@@ -542,6 +548,12 @@ sparsepr_status sparsepr_dense_attn(sparsepr_handle h, const void* Q, const void
     if (!h || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARSEPR_ERR_INVALID_ARG;
     const sparsepr_config& c = h->cfg;
     h->launches = 0;
+    if (spr::attn_tc_supported(c.d)) {
+        SPR_TRY(spr::launch_attn_dense_tc(static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
+                                          static_cast<const bf16*>(V), static_cast<bf16*>(O), nullptr, c.B, c.Hq,
+                                          c.Hkv, c.N, h->dev_status, as_stream(stream)));
+        return SPARSEPR_OK;
+    }
     SPR_TRY(spr::launch_attn_dense(static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
                                    static_cast<const bf16*>(V), static_cast<bf16*>(O), nullptr, c.B, c.Hq, c.Hkv,
                                    c.N, c.d, as_stream(stream)));

@@ -93,6 +93,14 @@ cudaError_t launch_attn_sparse(const bf16* Qp, const bf16* Kp, const bf16* Vp,
 // Dense attention of every query over all keys.
 cudaError_t launch_attn_dense(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse,
                               int B, int Hq, int Hkv, int N, int d, cudaStream_t s);
+// tcgen05/TMEM versions (head dimension 128): 128-row query tiles, 128-key tiles.
+bool attn_tc_supported(int d);
+cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp, const int32_t* qoff,
+                                  const int32_t* koff, const int32_t* tile_off, const int32_t* rowptr,
+                                  const int32_t* kg, bf16* O, float* lse, int B, int Hq, int Hkv, int N, int Gq,
+                                  int Gk, int* status, cudaStream_t s);
+cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
+                                 int Hkv, int N, int* status, cudaStream_t s);
 // Dense attention of gathered probe rows, split over ns key chunks, then combined.
 cudaError_t launch_attn_probe(const bf16* Q, const bf16* K, const bf16* V, const int32_t* probe,
                               float* Opart, float* mpart, float* lpart, float* Odense, int B,
