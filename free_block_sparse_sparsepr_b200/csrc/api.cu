@@ -65,8 +65,12 @@ struct sparsepr_handle_s {
     cudaEvent_t user_ev[7] = {};
     bool user_events = false;
     bool timing = false, timed_call = false;
+    // tensor-core k-means operands
+    bf16 *kmX3 = nullptr, *kmC3 = nullptr;
+    float *kmxx = nullptr, *kmcc = nullptr;
     int launches = 0;
     int device = 0;
+    int num_sms = 148;
 };
 
 namespace {
@@ -136,18 +140,29 @@ long long budget_pairs(const sparsepr_config& c, int M) {
     return (long long)floor((double)c.rho_exec * nn) - (long long)M * c.N;
 }
 
-// Lloyd k-means on X [P][n][DP] into G groups, then the stable group-major order.
+// Lloyd k-means on X [P][n][DP] into G groups, then the stable group-major order. With
+// G <= 256 the assignment runs on tensor cores (bf16 hi/lo split operands).
 sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t* labels, float* dist,
                        int32_t* perm, int32_t* off, cudaStream_t s) {
     const int P = h->P, n = h->cfg.N;
+    const bool tc = spr::km_tc_supported(G);
+    auto assign = [&](bool first, const int* done) -> cudaError_t {
+        if (!tc) return spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, done, P, n, G, DP, first, s);
+        cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC3, h->kmcc, P, G, DP, s);
+        if (e != cudaSuccess) return e;
+        ++h->launches;
+        return spr::launch_km_assign_tc(h->kmX3, h->kmxx, h->kmC3, h->kmcc, labels, dist, h->km_changed, done,
+                                        h->dev_status, P, n, G, DP, first, h->num_sms, s);
+    };
     SPR_TRY(spr::launch_km_reset(h->km_changed, h->km_done, P, s));
+    if (tc) SPR_TRY(spr::launch_km_split_rows(X, h->kmX3, h->kmxx, P, n, DP, s));
     SPR_TRY(spr::launch_km_seed(X, h->kmC, P, n, G, DP, s));
-    SPR_TRY(spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, nullptr, P, n, G, DP, true, s));
+    SPR_TRY(assign(true, nullptr));
     for (int it = 0; it < h->cfg.kmeans_iters; ++it) {
         SPR_TRY(spr::launch_group_sort(labels, perm, off, h->counts, h->bases, h->km_done, P, n, G, s));
         h->launches += 2;  // histogram, scan and scatter kernels
         SPR_TRY(spr::launch_km_update(X, perm, off, h->kmC, h->km_done, P, n, G, DP, s));
-        SPR_TRY(spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, h->km_done, P, n, G, DP, false, s));
+        SPR_TRY(assign(false, h->km_done));
         SPR_TRY(spr::launch_km_check(h->km_changed, h->km_done, P, s));
     }
     SPR_TRY(spr::launch_group_sort(labels, perm, off, h->counts, h->bases, nullptr, P, n, G, s));
@@ -328,6 +343,8 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     h->cfg = *cfg;
     const sparsepr_config& c = h->cfg;
     cudaGetDevice(&h->device);
+    if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess || h->num_sms < 1)
+        h->num_sms = 148;
     h->P = c.B * c.Hkv;
     h->Hp = c.B * c.Hq;
     h->g = c.Hq / c.Hkv;
@@ -367,6 +384,11 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     A_(Odense, Hp * M * d); A_(R, Hp * M * d); A_(Xprobe, Hp * M * d);
     A_(obar, Hp * d); A_(Rbar, Hp * d); A_(A, Hp * d * d); A_(U, Hp * d * r); A_(Bm, Hp * r * d); A_(c0, Hp * r);
     A_(rank, Hp); A_(dev_status, 1);
+    {
+        const size_t G16 = (size_t)((h->Gmax + 15) / 16 * 16), G32 = (size_t)((h->Gmax + 31) / 32 * 32);
+        A_(kmX3, 3 * P * N * 64); A_(kmxx, P * N);
+        A_(kmC3, 3 * P * G16 * 64); A_(kmcc, P * G32);
+    }
 #undef A_
     bool ok = cudaMemset(h->dev_status, 0, sizeof(int)) == cudaSuccess;
     if (h->proj) {

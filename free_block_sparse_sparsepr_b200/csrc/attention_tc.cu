@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_primitives.cuh"
+#include "tmap.h"
 
 namespace spr {
 namespace {
@@ -378,43 +379,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
 }
 
-// ---------------------------------------------------------------- host side: tensor maps
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-// [rows][128] bf16 row-major tensor, boxes of 128 rows x 64 columns, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const bf16* ptr, long long rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kD * sizeof(bf16)};
-    cuuint32_t box[2] = {64, 128};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
+// ---------------------------------------------------------------- host side
 
 template <int MODE>
 cudaError_t launch_tc(const bf16* Q, const bf16* K, const bf16* V, const TcParams& p, int B, int Hq, int Hkv,
                       dim3 grid, cudaStream_t s) {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, Q, (long long)B * Hq * p.N) || !make_map(&mk, K, (long long)B * Hkv * p.N) ||
-        !make_map(&mv, V, (long long)B * Hkv * p.N))
+    if (!make_tmap_bf16_sw128(&mq, Q, (long long)B * Hq * p.N, kD, kBM, 64) ||
+        !make_tmap_bf16_sw128(&mk, K, (long long)B * Hkv * p.N, kD, kBN, 64) ||
+        !make_tmap_bf16_sw128(&mv, V, (long long)B * Hkv * p.N, kD, kBN, 64))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -34,17 +34,21 @@ __global__ void coords_center_kernel(const float* __restrict__ u, bf16* uhi, bf1
     if (i >= N) return;
     const float invg = 1.f / (float)g;
     float v[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) v[t] = 0.f;
+    for (int j = 0; j < g; ++j) {
+        const float* ur = u + (((long long)z * g + j) * N + i) * Gk;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {             // 32 independent loads in flight per head
+            const int gk = lane + 32 * t;
+            if (gk < Gk) v[t] += ur[gk];
+        }
+    }
     float s = 0.f;
 #pragma unroll
     for (int t = 0; t < 32; ++t) {
-        int gk = lane + 32 * t;
-        float a = 0.f;
-        if (gk < Gk) {
-            for (int j = 0; j < g; ++j) a += u[(((long long)z * g + j) * N + i) * Gk + gk];
-            a *= invg;
-        }
-        v[t] = a;
-        s += a;
+        v[t] *= invg;
+        s += v[t];
     }
     const float mean = warp_sum(s) / (float)Gk;
     float ss = 0.f;
@@ -77,14 +81,17 @@ __global__ void coords_center_kernel(const float* __restrict__ u, bf16* uhi, bf1
     }
 }
 
-__global__ void rows_normalize_kernel(float* y, int rows, int DP) {
-    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+// One warp per row: y / ||y|| (zero rows stay zero), DP <= 64.
+__global__ void rows_normalize_kernel(float* y, long long rows, int DP) {
+    const long long i = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
     if (i >= rows) return;
     float* r = y + i * DP;
-    float ss = 0.f;
-    for (int k = 0; k < DP; ++k) ss = fmaf(r[k], r[k], ss);
-    const float nrm = sqrtf(ss);
-    for (int k = 0; k < DP; ++k) r[k] = nrm > 0.f ? r[k] / nrm : 0.f;
+    const float a = lane < DP ? r[lane] : 0.f;
+    const float b = lane + 32 < DP ? r[lane + 32] : 0.f;
+    const float nrm = sqrtf(warp_sum(fmaf(a, a, b * b)));
+    if (lane < DP) r[lane] = nrm > 0.f ? a / nrm : 0.f;
+    if (lane + 32 < DP) r[lane + 32] = nrm > 0.f ? b / nrm : 0.f;
 }
 
 __global__ void make_projection_kernel(bf16* projT, int Gk, int Gkp, int rQ, int DPy,
@@ -198,7 +205,7 @@ cudaError_t launch_coords_center(const float* u, bf16* uhi, bf16* ulo, float* y,
 }
 
 cudaError_t launch_rows_normalize(float* y, int rows, int DP, cudaStream_t s) {
-    rows_normalize_kernel<<<(rows + 255) / 256, 256, 0, s>>>(y, rows, DP);
+    rows_normalize_kernel<<<(unsigned)(((long long)rows + 7) / 8), 256, 0, s>>>(y, rows, DP);
     return cudaGetLastError();
 }
 

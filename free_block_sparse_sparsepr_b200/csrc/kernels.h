@@ -41,6 +41,14 @@ cudaError_t launch_group_sort(const int32_t* labels, int32_t* perm, int32_t* off
 cudaError_t launch_group_mean_bf16(const bf16* Y, const int32_t* perm, const int32_t* off,
                                    float* cent, bf16* chi, bf16* clo, int P, int n, int G, int d,
                                    cudaStream_t s);
+// Tensor-core assignment (G <= 256): rows and centroids split into three bf16 parts
+// (X3: [3][P][n][64], C3: [3][P][G16][64]).
+bool km_tc_supported(int G);
+cudaError_t launch_km_split_rows(const float* X, bf16* X3, float* xx, int P, int n, int DP, cudaStream_t s);
+cudaError_t launch_km_split_cent(const float* C, bf16* C3, float* cc, int P, int G, int DP, cudaStream_t s);
+cudaError_t launch_km_assign_tc(const bf16* X3, const float* xx, const bf16* C3, const float* cc, int32_t* labels,
+                                float* dist, int* changed, const int* done, int* status, int P, int n, int G,
+                                int DP, bool first, int num_sms, cudaStream_t s);
 // Split fp32 group means into bf16 hi/lo (used when the partition is handed in).
 cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long count, cudaStream_t s);
 
