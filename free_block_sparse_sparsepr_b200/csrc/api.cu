@@ -18,7 +18,7 @@ namespace {
 
 constexpr int kMaxGroups = 1024;
 constexpr int kProbeSplits = 32;
-constexpr int kSortChunk = 256;
+constexpr int kSortChunk = 2048;   // rows per counting-sort chunk (matches the sort kernels)
 constexpr unsigned kSupportedFlags =
     SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_STAGE_TIMING;
 

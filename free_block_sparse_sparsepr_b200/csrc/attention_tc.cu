@@ -4,12 +4,15 @@
 //
 // One CTA per 128-row query tile, six warps:
 //   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r; it reads its row
-//              of S from TMEM, keeps the running max / sum, writes P (bf16) into shared
-//              memory in the 128-byte-swizzled K-major layout, rescales its O row in TMEM
-//              when the max grows by more than 2^8, and finally normalises and stores O;
+//              of S from TMEM, keeps the running max / sum, writes P (bf16) into one of two
+//              shared-memory buffers in the 128-byte-swizzled K-major layout, rescales its O
+//              row in TMEM when the max grows by more than 2^8, and finally normalises and
+//              stores O;
 //   warp 4     TMA producer: Q once, then K and V tiles of 128 keys into a 2-stage ring;
 //   warp 5     TMEM allocation and the MMA issue (one elected thread): S = Q K^T into one of
 //              two TMEM buffers, O += P V into a third, completion signalled by tcgen05.commit.
+// With two P buffers the tensor core runs S(j+1) and PV(j) while the softmax warps work on
+// tile j+1; they wait for PV(j) only when their O row needs rescaling.
 // Key tiles are cut from merged runs of consecutive kept key groups; keys past a run's end
 // (the next group's, or zero fill past the tensor) are masked to -inf.
 #include <cuda.h>
@@ -39,10 +42,11 @@ constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + 2 * kRegion;
 constexpr int kOffV = kOffK + kStages * 2 * kRegion;
 constexpr int kOffP = kOffV + kStages * 2 * kRegion;
-constexpr int kOffBar = kOffP + 2 * kRegion;
-// barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full, o_done, mma_done
+constexpr int kOffBar = kOffP + 2 * 2 * kRegion;          // two P buffers
+// barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], mma_done
+// (s/p/o barriers indexed by tile parity so no waiter can fall two phases behind)
 constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kStages, kBarE = kBarV + kStages, kBarS = kBarE + kStages,
-              kBarP = kBarS + 2, kBarO = kBarP + 1, kBarMma = kBarO + 1, kNumBars = kBarMma + 1;
+              kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2, kNumBars = kBarMma + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;          // tmem base (u32), abort flag (int)
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;          // + slack to align the base to 1024
 
@@ -149,10 +153,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             tc::mbar_init(bar(kBarV + s), 1);
             tc::mbar_init(bar(kBarE + s), 1);
         }
-        tc::mbar_init(bar(kBarS), 1);
-        tc::mbar_init(bar(kBarS + 1), 1);
-        tc::mbar_init(bar(kBarP), 128);
-        tc::mbar_init(bar(kBarO), 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(bar(kBarS + b), 1);
+            tc::mbar_init(bar(kBarP + b), 128);
+            tc::mbar_init(bar(kBarO + b), 1);
+        }
         tc::mbar_init(bar(kBarMma), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
@@ -234,20 +239,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             bool nhave = it.next(start, lim);
             if (nhave && !issue_S(j + 1)) { ok = false; break; }
             const int s = j % kStages;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarP), j & 1, abort_flag))) { ok = false; break; }
+            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarP + (j & 1)), (j >> 1) & 1, abort_flag))) { ok = false; break; }
             if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kStages) & 1, abort_flag))) { ok = false; break; }
             tc::fence_after_sync();
             if (lane == 0) {
                 const uint32_t vb = sV + s * 2 * kRegion;
 #pragma unroll
                 for (int k = 0; k < kBN / 16; ++k) {
-                    const uint32_t pa = sP + (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
+                    const uint32_t pa = sP + (uint32_t)((j & 1) * 2 * kRegion + (k >> 2) * kRegion + (k & 3) * 32);
                     const uint32_t vbk = vb + (uint32_t)(k * 2048);
                     tc::mma_f16_ss(tO, tc::smem_desc_sw128(pa, 16, 1024), tc::smem_desc_sw128(vbk, kRegion, 1024), idO,
                                    (j > 0 || k > 0) ? 1u : 0u);
                 }
                 tc::commit(bar(kBarE + s));
-                tc::commit(bar(kBarO));
+                tc::commit(bar(kBarO + (j & 1)));
             }
             __syncwarp();
             have = nhave;
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         int start, lim, j = 0;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        unsigned char* prow = sbase + kOffP + r * 128;
+        const float c_log2 = p.scale_log2;
         while (it.next(start, lim)) {
             // every TMEM access below is warp-collective: decisions are made warp-uniform
             const bool got_s = tc::mbar_wait(bar(kBarS + (j & 1)), (j >> 1) & 1, abort_flag);
@@ -280,40 +285,52 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             tc::tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 4; ++c) tc::regs_after_wait(sv[c]);
+            // row max of the raw logits; keys past the run's end are set to -inf
             float mx = -INFINITY;
+            if (lim == kBN) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float v = (32 * c + i) < lim ? __uint_as_float(sv[c][i]) * p.scale_log2 : -INFINITY;
-                    sv[c][i] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
-                }
+                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (32 * c + i >= lim) sv[c][i] = __float_as_uint(-INFINITY);
+                        mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+                    }
             }
-            const float m_new = fmaxf(m_run, mx);
+            const float m_new = fmaxf(m_run, mx * c_log2);
             const bool rescale = m_new > m_run + kRescaleLog2;
-            if (j > 0) {
-                const bool got_o = tc::mbar_wait(bar(kBarO), (j - 1) & 1, abort_flag);
+            if (j > 0 && __any_sync(kFull, rescale)) {
+                // O holds PV(0..j-1): wait for PV(j-1), then scale the rows whose max moved
+                const bool got_o = tc::mbar_wait(bar(kBarO + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag);
                 if (!__all_sync(kFull, got_o)) { ok = false; break; }
                 tc::fence_after_sync();
-                if (__any_sync(kFull, rescale)) {
-                    const float f = rescale ? exp2f(m_run - m_new) : 1.f;
+                const float f = rescale ? exp2f(m_run - m_new) : 1.f;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t ov[32];
-                        tc::tmem_ld32(tO + lane_off + 32 * c, ov);
-                        tc::tmem_wait_ld();
-                        tc::regs_after_wait(ov);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tc::tmem_ld32(tO + lane_off + 32 * c, ov);
+                    tc::tmem_wait_ld();
+                    tc::regs_after_wait(ov);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-                        tc::tmem_st32(tO + lane_off + 32 * c, ov);
-                    }
-                    tc::tmem_wait_st();
-                    l_run *= f;
+                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+                    tc::tmem_st32(tO + lane_off + 32 * c, ov);
                 }
+                tc::tmem_wait_st();
+                if (rescale) l_run *= f;
             }
             if (rescale) m_run = m_new;
-            // P = 2^(s - m_run) as bf16, 16-byte chunks into the swizzled K-major P tile
+            // P buffer j&1 was last read by PV(j-2)
+            if (j >= 2) {
+                const bool got_b = tc::mbar_wait(bar(kBarO + (j & 1)), ((j - 2) >> 1) & 1, abort_flag);
+                if (!__all_sync(kFull, got_b)) { ok = false; break; }
+            }
+            // P = 2^(s*c - m_run) as bf16, 16-byte chunks into the swizzled K-major P tile
+            unsigned char* prow = sbase + kOffP + (j & 1) * 2 * kRegion + r * 128;
+            const float neg_m = -m_run;
             float sum = 0.f;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
@@ -321,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(__uint_as_float(sv[c >> 2][(c & 3) * 8 + 2 * e]) - m_run);
-                    const float p1 = exp2f(__uint_as_float(sv[c >> 2][(c & 3) * 8 + 2 * e + 1]) - m_run);
+                    const float p0 = exp2f(fmaf(__uint_as_float(sv[c >> 2][(c & 3) * 8 + 2 * e]), c_log2, neg_m));
+                    const float p1 = exp2f(fmaf(__uint_as_float(sv[c >> 2][(c & 3) * 8 + 2 * e + 1]), c_log2, neg_m));
                     sum += p0 + p1;
                     __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<uint32_t*>(&b2);
@@ -332,12 +349,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             l_run += sum;
             tc::fence_proxy_async_smem();
             tc::fence_before_sync();
-            tc::mbar_arrive(bar(kBarP));
+            tc::mbar_arrive(bar(kBarP + (j & 1)));
             ++j;
         }
         // epilogue: O / l, bf16 row store, lse
         bool got_last = false;
-        if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO), (j - 1) & 1, abort_flag);
+        if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag);
         if (j > 0 && __all_sync(kFull, got_last)) {
             tc::fence_after_sync();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;

@@ -26,22 +26,40 @@ __global__ void gather_samples_kernel(const bf16* __restrict__ Q, bf16* Qs, int 
 }
 
 // One warp per query row of a KV head: mean of the g heads' logits, centred over the groups.
+// VEC (Gk % 8 == 0): lane l owns the 8 consecutive columns 256*b + 8*l .. +7 of each block b of
+// 256 columns, read as two float4 and written as one 16-byte bf16 vector per part; otherwise
+// lane l owns the strided columns l + 32*t.
+template <bool VEC>
 __global__ void coords_center_kernel(const float* __restrict__ u, bf16* uhi, bf16* ulo, float* y,
                                      int g, int N, int Gk, int Gkp, int DPy, int proj) {
     const int z = blockIdx.y;
     const int lane = threadIdx.x & 31;
     const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (i >= N) return;
+    auto col = [&](int t) { return VEC ? (t >> 3) * 256 + lane * 8 + (t & 7) : lane + 32 * t; };
     const float invg = 1.f / (float)g;
     float v[32];
 #pragma unroll
     for (int t = 0; t < 32; ++t) v[t] = 0.f;
     for (int j = 0; j < g; ++j) {
         const float* ur = u + (((long long)z * g + j) * N + i) * Gk;
+        if (VEC) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {             // 32 independent loads in flight per head
-            const int gk = lane + 32 * t;
-            if (gk < Gk) v[t] += ur[gk];
+            for (int b = 0; b < 4; ++b) {
+                const int c0 = b * 256 + lane * 8;
+                if (c0 < Gk) {
+                    const float4 a0 = *reinterpret_cast<const float4*>(ur + c0);
+                    const float4 a1 = *reinterpret_cast<const float4*>(ur + c0 + 4);
+                    v[8 * b + 0] += a0.x; v[8 * b + 1] += a0.y; v[8 * b + 2] += a0.z; v[8 * b + 3] += a0.w;
+                    v[8 * b + 4] += a1.x; v[8 * b + 5] += a1.y; v[8 * b + 6] += a1.z; v[8 * b + 7] += a1.w;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {             // 32 independent loads in flight per head
+                const int gk = col(t);
+                if (gk < Gk) v[t] += ur[gk];
+            }
         }
     }
     float s = 0.f;
@@ -54,20 +72,41 @@ __global__ void coords_center_kernel(const float* __restrict__ u, bf16* uhi, bf1
     float ss = 0.f;
 #pragma unroll
     for (int t = 0; t < 32; ++t) {
-        int gk = lane + 32 * t;
+        const int gk = col(t);
         v[t] = gk < Gk ? v[t] - mean : 0.f;
         ss = fmaf(v[t], v[t], ss);
     }
     if (proj) {
         bf16* hr = uhi + ((long long)z * N + i) * Gkp;
         bf16* lr = ulo + ((long long)z * N + i) * Gkp;
+        if (VEC) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            int gk = lane + 32 * t;
-            if (gk < Gkp) {
-                bf16 hh = __float2bfloat16_rn(v[t]);
-                hr[gk] = hh;
-                lr[gk] = __float2bfloat16_rn(v[t] - __bfloat162float(hh));
+            for (int b = 0; b < 4; ++b) {
+                const int c0 = b * 256 + lane * 8;
+                if (c0 < Gkp) {
+                    uint32_t wh[4], wl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = v[8 * b + 2 * e], c = v[8 * b + 2 * e + 1];
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(a, c);
+                        const float2 hf = __bfloat1622float2(h2);
+                        __nv_bfloat162 l2 = __floats2bfloat162_rn(a - hf.x, c - hf.y);
+                        wh[e] = *reinterpret_cast<uint32_t*>(&h2);
+                        wl[e] = *reinterpret_cast<uint32_t*>(&l2);
+                    }
+                    *reinterpret_cast<uint4*>(hr + c0) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                    *reinterpret_cast<uint4*>(lr + c0) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int gk = col(t);
+                if (gk < Gkp) {
+                    bf16 hh = __float2bfloat16_rn(v[t]);
+                    hr[gk] = hh;
+                    lr[gk] = __float2bfloat16_rn(v[t] - __bfloat162float(hh));
+                }
             }
         }
     } else {
@@ -75,7 +114,7 @@ __global__ void coords_center_kernel(const float* __restrict__ u, bf16* uhi, bf1
         float* yr = y + ((long long)z * N + i) * DPy;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-            int gk = lane + 32 * t;
+            const int gk = col(t);
             if (gk < DPy) yr[gk] = (gk < Gk && nrm > 0.f) ? v[t] / nrm : 0.f;
         }
     }
@@ -200,7 +239,10 @@ cudaError_t launch_gather_samples(const bf16* Q, bf16* Qs, int B, int Hq, int Hk
 cudaError_t launch_coords_center(const float* u, bf16* uhi, bf16* ulo, float* y, int P, int g,
                                  int N, int Gk, int Gkp, int DPy, bool proj, cudaStream_t s) {
     dim3 grid((N + 7) / 8, P);
-    coords_center_kernel<<<grid, 256, 0, s>>>(u, uhi, ulo, y, g, N, Gk, Gkp, DPy, proj ? 1 : 0);
+    if (Gk % 8 == 0 && Gkp % 8 == 0)
+        coords_center_kernel<true><<<grid, 256, 0, s>>>(u, uhi, ulo, y, g, N, Gk, Gkp, DPy, proj ? 1 : 0);
+    else
+        coords_center_kernel<false><<<grid, 256, 0, s>>>(u, uhi, ulo, y, g, N, Gk, Gkp, DPy, proj ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -22,61 +22,50 @@ __global__ void probe_residual_kernel(const float* __restrict__ Od, const bf16* 
     R[o] = Od[o] - os;
 }
 
-__device__ __forceinline__ float block_sum(float v, float* red) {
-    v = warp_sum(v);
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    __syncthreads();
-    if (lane == 0) red[w] = v;
-    __syncthreads();
-    float t = 0.f;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
-        red[32] = t;
-    }
-    __syncthreads();
-    return red[32];
-}
-
-// Per query head x:
+// Per query head x (one CTA of 512 threads):
 //   xbar, Rbar   w-weighted means of the probes' sparse outputs X and residuals R
 //   A            argmin sum_m w_m ||(R_m - Rbar) - A (X_m - xbar)||^2 + lambda ||A||_F^2, via the
 //                M x M system: A = Ys^T (Xs Xs^T + lambda I)^-1 Xs, Xs/Ys rows scaled by sqrt(w_m)
-//   U            top-r eigenvectors of the Gram matrix of [sqrt(w_m) R_m] mapped to output
-//                space (= top-r left singular vectors), cyclic Jacobi in fp32
+//                (Cholesky of the M x M matrix)
+//   U            top-r left singular vectors of the d x M matrix W = [sqrt(w_m) R_m]: one-sided
+//                (Hestenes) Jacobi rotates column pairs of W until they are mutually orthogonal;
+//                the columns are then sigma_m u_m, sorted by norm (ties -> lower index)
 //   Bm = U^T A, c0 = U^T Rbar - Bm xbar  so that the correction is U (c0 + Bm o).
-constexpr int kFitThreads = 256;
+constexpr int kFitThreads = 512;
+constexpr int kFitWarps = kFitThreads / 32;
 __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     const float* __restrict__ Rg, const float* __restrict__ Xg, const float* __restrict__ wts,
     float lambda, float* obar, float* Rbar, float* A, float* U, float* Bm, float* c0,
     int32_t* rank_out, int g, int d, int M, int r, int* status) {
     const int x = blockIdx.x, z = x / g, tid = threadIdx.x, nt = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5;
     const int Mp = (M + 1) & ~1;
+    const int ld = d + 1;            // padded row stride: column-wise walks hit distinct banks
     extern __shared__ float sm[];
-    float* X = sm;                 // [M][d]
-    float* Y = X + M * d;          // [M][d]
-    float* Km = Y + M * d;         // [M][M]
-    float* Gr = Km + M * M;        // [M][M]
-    float* Vv = Gr + M * M;        // [M][M]
-    float* Us = Vv + M * M;        // [d][r]
-    float* w = Us + d * r;         // [M]
-    float* sw = w + M;             // [M]
-    float* xb = sw + M;            // [d]
-    float* yb = xb + d;            // [d]
-    float* rc = yb + d;            // [Mp/2]
-    float* rs = rc + Mp / 2;       // [Mp/2]
-    float* eig = rs + Mp / 2;      // [M]
-    float* red = eig + M;          // [33]
-    int* pp = reinterpret_cast<int*>(red + 33);   // [Mp/2]
-    int* pq = pp + Mp / 2;                        // [Mp/2]
-    int* sel = pq + Mp / 2;                       // [r]
+    float* X = sm;                   // [M][ld]   probes' sparse outputs, then Xs, then Z
+    float* Y = X + M * ld;           // [M][ld]   residuals, then Ys
+    float* Wc = Y + M * ld;          // [M][ld]   sqrt(w_m) R_m (rows = columns of W)
+    float* Km = Wc + M * ld;         // [M][M]
+    float* Us = Km + M * M;          // [d][r]
+    float* w = Us + d * r;           // [M]
+    float* sw = w + M;               // [M]
+    float* xb = sw + M;              // [d]
+    float* yb = xb + d;              // [d]
+    float* nrm = yb + d;             // [M]
+    int* sel = reinterpret_cast<int*>(nrm + M);   // [r]
     __shared__ float sW;
-    __shared__ int s_rank, s_stop;
+    __shared__ int s_rank, s_rot;
 
     const float* Rx = Rg + (long long)x * M * d;
     const float* Xx = Xg + (long long)x * M * d;
-    for (int t = tid; t < M * d; t += nt) { X[t] = Xx[t]; Y[t] = Rx[t]; }
     for (int t = tid; t < M; t += nt) { w[t] = wts[(long long)z * M + t]; sw[t] = sqrtf(wts[(long long)z * M + t]); }
     __syncthreads();
+    for (int t = tid; t < M * d; t += nt) {
+        const int m = t / d, c = t % d;
+        X[m * ld + c] = Xx[t];
+        Y[m * ld + c] = Rx[t];
+        Wc[m * ld + c] = sw[m] * Rx[t];
+    }
     if (tid == 0) {
         float W = 0.f;
         for (int m = 0; m < M; ++m) W += w[m];
@@ -86,38 +75,40 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     const float W = sW;
     for (int c = tid; c < d; c += nt) {
         float sx = 0.f, sy = 0.f;
-        for (int m = 0; m < M; ++m) { sx = fmaf(w[m], X[m * d + c], sx); sy = fmaf(w[m], Y[m * d + c], sy); }
+        for (int m = 0; m < M; ++m) { sx = fmaf(w[m], X[m * ld + c], sx); sy = fmaf(w[m], Y[m * ld + c], sy); }
         xb[c] = sx / W;
         yb[c] = sy / W;
-    }
-    // Gram matrix of the weighted, uncentred residuals.
-    for (int t = tid; t < M * M; t += nt) {
-        const int i = t / M, j = t % M;
-        float acc = 0.f;
-        for (int c = 0; c < d; ++c) acc = fmaf(Y[i * d + c], Y[j * d + c], acc);
-        Gr[t] = sw[i] * sw[j] * acc;
     }
     __syncthreads();
     for (int t = tid; t < M * d; t += nt) {
         const int m = t / d, c = t % d;
-        X[t] = sw[m] * (X[t] - xb[c]);
-        Y[t] = sw[m] * (Y[t] - yb[c]);
+        X[m * ld + c] = sw[m] * (X[m * ld + c] - xb[c]);
+        Y[m * ld + c] = sw[m] * (Y[m * ld + c] - yb[c]);
     }
     __syncthreads();
-    for (int t = tid; t < M * M; t += nt) {
-        const int i = t / M, j = t % M;
+    // Km = Xs Xs^T + lambda I: one warp per entry, lanes over the d columns
+    for (int e = warp; e < M * M; e += kFitWarps) {
+        const int i = e / M, j = e % M;
+        if (j > i) continue;
         float acc = 0.f;
-        for (int c = 0; c < d; ++c) acc = fmaf(X[i * d + c], X[j * d + c], acc);
-        Km[t] = acc + (i == j ? lambda : 0.f);
+        for (int c = lane; c < d; c += 32) acc = fmaf(X[i * ld + c], X[j * ld + c], acc);
+        acc = warp_sum(acc);
+        if (lane == 0) {
+            Km[i * M + j] = acc + (i == j ? lambda : 0.f);
+            Km[j * M + i] = acc + (i == j ? lambda : 0.f);
+        }
     }
     __syncthreads();
-    // Cholesky Km = L L^T (lower triangle, in place).
+    // Cholesky Km = L L^T (lower triangle, in place)
     for (int j = 0; j < M; ++j) {
-        if (tid == 0) {
-            float s = Km[j * M + j];
-            for (int k = 0; k < j; ++k) s -= Km[j * M + k] * Km[j * M + k];
-            if (!(s > 0.f)) { set_status(status, kDevBounds); s = 1e-30f; }
-            Km[j * M + j] = sqrtf(s);
+        if (warp == 0) {
+            float s = 0.f;
+            for (int k = lane; k < j; k += 32) s = fmaf(Km[j * M + k], Km[j * M + k], s);
+            s = Km[j * M + j] - warp_sum(s);
+            if (lane == 0) {
+                if (!(s > 0.f)) { set_status(status, kDevBounds); s = 1e-30f; }
+                Km[j * M + j] = sqrtf(s);
+            }
         }
         __syncthreads();
         for (int i = j + 1 + tid; i < M; i += nt) {
@@ -127,17 +118,17 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
         }
         __syncthreads();
     }
-    // Z = Km^-1 Xs, column by column, in place in X.
+    // Z = Km^-1 Xs, column by column, in place in X
     for (int c = tid; c < d; c += nt) {
         for (int m = 0; m < M; ++m) {
-            float s = X[m * d + c];
-            for (int k = 0; k < m; ++k) s -= Km[m * M + k] * X[k * d + c];
-            X[m * d + c] = s / Km[m * M + m];
+            float s = X[m * ld + c];
+            for (int k = 0; k < m; ++k) s -= Km[m * M + k] * X[k * ld + c];
+            X[m * ld + c] = s / Km[m * M + m];
         }
         for (int m = M - 1; m >= 0; --m) {
-            float s = X[m * d + c];
-            for (int k = m + 1; k < M; ++k) s -= Km[k * M + m] * X[k * d + c];
-            X[m * d + c] = s / Km[m * M + m];
+            float s = X[m * ld + c];
+            for (int k = m + 1; k < M; ++k) s -= Km[k * M + m] * X[k * ld + c];
+            X[m * ld + c] = s / Km[m * M + m];
         }
     }
     __syncthreads();
@@ -145,77 +136,63 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     for (int t = tid; t < d * d; t += nt) {
         const int c = t / d, c2 = t % d;
         float acc = 0.f;
-        for (int m = 0; m < M; ++m) acc = fmaf(Y[m * d + c], X[m * d + c2], acc);
+        for (int m = 0; m < M; ++m) acc = fmaf(Y[m * ld + c], X[m * ld + c2], acc);
         Ax[t] = acc;
     }
-    // Cyclic Jacobi on Gr with round-robin disjoint pairs; V accumulates the rotations.
-    for (int t = tid; t < M * M; t += nt) Vv[t] = (t / M == t % M) ? 1.f : 0.f;
-    __syncthreads();
-    for (int sweep = 0; sweep < 15; ++sweep) {
-        float off = 0.f, tot = 0.f;
-        for (int t = tid; t < M * M; t += nt) {
-            const float v = Gr[t] * Gr[t];
-            tot += v;
-            if (t / M != t % M) off += v;
-        }
-        off = block_sum(off, red);
-        tot = block_sum(tot, red);
-        if (tid == 0) s_stop = (off <= 1e-12f * tot) ? 1 : 0;
+    // One-sided Jacobi on the columns of W (round-robin disjoint pairs, one warp per pair)
+    for (int sweep = 0; sweep < 12; ++sweep) {
+        if (tid == 0) s_rot = 0;
         __syncthreads();
-        if (s_stop) break;
         for (int k = 0; k < Mp - 1; ++k) {
-            for (int i = tid; i < Mp / 2; i += nt) {
+            for (int i = warp; i < Mp / 2; i += kFitWarps) {
                 const int a1 = (i == 0) ? 0 : ((i - 1 + k) % (Mp - 1)) + 1;
                 const int b1 = ((Mp - 2 - i + k) % (Mp - 1)) + 1;
-                const int p = min(a1, b1), q = max(a1, b1);
-                float c = 1.f, s = 0.f;
-                if (q < M) {
-                    const float apq = Gr[p * M + q];
-                    if (apq != 0.f) {
-                        const float theta = (Gr[q * M + q] - Gr[p * M + p]) / (2.f * apq);
-                        const float tt = (theta >= 0.f ? 1.f : -1.f) / (fabsf(theta) + sqrtf(theta * theta + 1.f));
-                        c = 1.f / sqrtf(tt * tt + 1.f);
-                        s = tt * c;
-                    }
+                const int pc = min(a1, b1), qc = max(a1, b1);
+                if (qc >= M) continue;
+                float al = 0.f, be = 0.f, ga = 0.f;
+                for (int c = lane; c < d; c += 32) {
+                    const float u1 = Wc[pc * ld + c], u2 = Wc[qc * ld + c];
+                    al = fmaf(u1, u1, al);
+                    be = fmaf(u2, u2, be);
+                    ga = fmaf(u1, u2, ga);
                 }
-                pp[i] = p; pq[i] = q; rc[i] = c; rs[i] = s;
-            }
-            __syncthreads();
-            for (int t = tid; t < (Mp / 2) * M; t += nt) {
-                const int i = t / M, col = t % M, p = pp[i], q = pq[i];
-                if (q >= M) continue;
-                const float c = rc[i], s = rs[i];
-                const float gp = Gr[p * M + col], gq = Gr[q * M + col];
-                Gr[p * M + col] = c * gp - s * gq;
-                Gr[q * M + col] = s * gp + c * gq;
-            }
-            __syncthreads();
-            for (int t = tid; t < (Mp / 2) * M; t += nt) {
-                const int i = t / M, row = t % M, p = pp[i], q = pq[i];
-                if (q >= M) continue;
-                const float c = rc[i], s = rs[i];
-                const float gp = Gr[row * M + p], gq = Gr[row * M + q];
-                Gr[row * M + p] = c * gp - s * gq;
-                Gr[row * M + q] = s * gp + c * gq;
-                const float vp = Vv[row * M + p], vq = Vv[row * M + q];
-                Vv[row * M + p] = c * vp - s * vq;
-                Vv[row * M + q] = s * vp + c * vq;
+                al = warp_sum(al);
+                be = warp_sum(be);
+                ga = warp_sum(ga);
+                if (fabsf(ga) > 1e-7f * sqrtf(al * be) && ga != 0.f) {
+                    const float zeta = (be - al) / (2.f * ga);
+                    const float tt = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(zeta * zeta + 1.f));
+                    const float cs = 1.f / sqrtf(tt * tt + 1.f), sn = tt * cs;
+                    for (int c = lane; c < d; c += 32) {
+                        const float u1 = Wc[pc * ld + c], u2 = Wc[qc * ld + c];
+                        Wc[pc * ld + c] = cs * u1 - sn * u2;
+                        Wc[qc * ld + c] = sn * u1 + cs * u2;
+                    }
+                    if (lane == 0) s_rot = 1;
+                }
             }
             __syncthreads();
         }
+        const int rotated = s_rot;   // read by every thread before thread 0 resets it
+        __syncthreads();
+        if (!rotated) break;
     }
-    // Top-r eigenpairs (descending; ties -> lower index) and the numerical rank.
-    for (int t = tid; t < M; t += nt) eig[t] = fmaxf(Gr[t * M + t], 0.f);
+    // column norms = singular values; top r (descending, ties -> lower index) and the rank
+    for (int m = warp; m < M; m += kFitWarps) {
+        float s = 0.f;
+        for (int c = lane; c < d; c += 32) s = fmaf(Wc[m * ld + c], Wc[m * ld + c], s);
+        s = warp_sum(s);
+        if (lane == 0) nrm[m] = sqrtf(s);
+    }
     __syncthreads();
-    if (tid < 32) {
-        const int lane = tid;
+    if (warp == 0) {
         for (int k = 0; k < r; ++k) {
             float best = -1.f;
             int bi = M;
             for (int m = lane; m < M; m += 32) {
                 bool used = false;
                 for (int j = 0; j < k; ++j) used |= (sel[j] == m);
-                if (!used && (eig[m] > best || (eig[m] == best && m < bi))) { best = eig[m]; bi = m; }
+                if (!used && (nrm[m] > best || (nrm[m] == best && m < bi))) { best = nrm[m]; bi = m; }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -228,12 +205,10 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
         }
         if (lane == 0) {
             const float tol = (float)(M > d ? M : d) * FLT_EPSILON;
-            const float e0 = eig[sel[0]];
+            const float s0 = nrm[sel[0]];
             int rk = 0;
-            for (int k = 0; k < r && k < M; ++k) {
-                const float e = eig[sel[k]];
-                if (e > 0.f && e > e0 * tol * tol) ++rk;
-            }
+            for (int k = 0; k < r && k < M; ++k)
+                if (nrm[sel[k]] > 0.f && nrm[sel[k]] > s0 * tol) ++rk;
             s_rank = rk;
         }
     }
@@ -241,13 +216,7 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     const int rank = s_rank;
     for (int t = tid; t < d * r; t += nt) {
         const int c = t / r, k = t % r;
-        float val = 0.f;
-        if (k < rank) {
-            const int e = sel[k];
-            float acc = 0.f;
-            for (int m = 0; m < M; ++m) acc = fmaf(sw[m] * Rx[m * d + c], Vv[m * M + e], acc);
-            val = acc / sqrtf(eig[e]);
-        }
+        const float val = k < rank ? Wc[sel[k] * ld + c] / nrm[sel[k]] : 0.f;
         Us[t] = val;
         U[(long long)x * d * r + t] = val;
     }
@@ -260,13 +229,15 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
         Bx[t] = acc;
     }
     __syncthreads();
-    for (int k = tid; k < r; k += nt) {
+    for (int k = warp; k < r; k += kFitWarps) {
         float a1 = 0.f, a2 = 0.f;
-        for (int c = 0; c < d; ++c) {
+        for (int c = lane; c < d; c += 32) {
             a1 = fmaf(Us[c * r + k], yb[c], a1);
             a2 = fmaf(Bx[(long long)k * d + c], xb[c], a2);
         }
-        c0[(long long)x * r + k] = a1 - a2;
+        a1 = warp_sum(a1);
+        a2 = warp_sum(a2);
+        if (lane == 0) c0[(long long)x * r + k] = a1 - a2;
     }
     for (int c = tid; c < d; c += nt) {
         obar[(long long)x * d + c] = xb[c];
@@ -364,10 +335,9 @@ __global__ void probe_override_kernel(const float* __restrict__ Od, const int32_
 }  // namespace
 
 size_t fit_smem_bytes(int d, int M, int r) {
-    const int Mp = (M + 1) & ~1;
-    size_t floats = (size_t)2 * M * d + 3 * (size_t)M * M + (size_t)d * r + 2 * M + 2 * d + Mp + M + 33;
-    size_t ints = (size_t)Mp + r;
-    return floats * 4 + ints * 4;
+    const size_t ld = (size_t)d + 1;
+    size_t floats = 3 * (size_t)M * ld + (size_t)M * M + (size_t)d * r + 2 * (size_t)M + 2 * (size_t)d + (size_t)M;
+    return floats * 4 + (size_t)r * 4;
 }
 
 cudaError_t launch_probe_residual(const float* Odense, const bf16* Osp, const int32_t* probe_pos,

@@ -10,7 +10,8 @@
 namespace spr {
 namespace {
 
-constexpr int kSortChunk = 256;     // rows per counting-sort chunk (one CTA, one row per thread)
+constexpr int kSortSub = 256;       // rows per sub-chunk (one row per thread)
+constexpr int kSortChunk = 2048;    // rows per counting-sort chunk (one CTA, 8 sub-chunks in order)
 constexpr int kAssignRows = 128;    // rows per assignment CTA (one row per thread)
 constexpr int kAssignCent = 128;    // centroids staged in shared memory per pass
 
@@ -127,8 +128,10 @@ __global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int* counts
     extern __shared__ int sh[];
     for (int t = threadIdx.x; t < G; t += blockDim.x) sh[t] = 0;
     __syncthreads();
-    const int i = ch * kSortChunk + threadIdx.x;
-    if (i < n) atomicAdd(&sh[labels[(long long)z * n + i]], 1);
+    for (int k = 0; k < kSortChunk / kSortSub; ++k) {
+        const int i = ch * kSortChunk + k * kSortSub + threadIdx.x;
+        if (i < n) atomicAdd(&sh[labels[(long long)z * n + i]], 1);
+    }
     __syncthreads();
     for (int t = threadIdx.x; t < G; t += blockDim.x) counts[((long long)z * nch + ch) * G + t] = sh[t];
 }
@@ -163,28 +166,39 @@ __global__ void sort_scan_kernel(const int* __restrict__ counts, int* bases, int
     }
 }
 
-// Stable scatter: position = off[g] + rows of g in earlier chunks + earlier warps + earlier lanes.
+// Stable scatter: position = off[g] + rows of g in earlier chunks + earlier sub-chunks of this
+// chunk + earlier warps of this sub-chunk + earlier lanes of this warp.
 __global__ void sort_scatter_kernel(const int32_t* __restrict__ labels, const int* __restrict__ bases,
                                     const int32_t* __restrict__ off, int32_t* perm, const int* done,
                                     int n, int G, int nch) {
     const int z = blockIdx.y, ch = blockIdx.x;
     if (done && done[z]) return;
-    extern __shared__ int wc[];  // [8][G]
-    for (int t = threadIdx.x; t < 8 * G; t += blockDim.x) wc[t] = 0;
+    extern __shared__ int wc[];  // [8][G] per-warp counts, then [G] running counts
+    int* run = wc + 8 * G;
+    for (int t = threadIdx.x; t < 9 * G; t += blockDim.x) wc[t] = 0;
     __syncthreads();
-    const int i = ch * kSortChunk + threadIdx.x;
-    const bool valid = i < n;
-    const int lab = valid ? labels[(long long)z * n + i] : -1;
-    const unsigned m = __match_any_sync(kFull, lab);
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int rank = __popc(m & ((1u << lane) - 1u));
-    if (valid && rank == 0) wc[w * G + lab] = __popc(m);
-    __syncthreads();
-    if (valid) {
-        int pre = 0;
-        for (int w2 = 0; w2 < w; ++w2) pre += wc[w2 * G + lab];
-        int pos = off[(long long)z * (G + 1) + lab] + bases[((long long)z * nch + ch) * G + lab] + pre + rank;
-        perm[(long long)z * n + pos] = i;
+    for (int k = 0; k < kSortChunk / kSortSub; ++k) {
+        const int i = ch * kSortChunk + k * kSortSub + threadIdx.x;
+        const bool valid = i < n;
+        const int lab = valid ? labels[(long long)z * n + i] : -1;
+        const unsigned m = __match_any_sync(kFull, lab);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        if (valid && rank == 0) wc[w * G + lab] = __popc(m);
+        __syncthreads();
+        if (valid) {
+            int pre = run[lab];
+            for (int w2 = 0; w2 < w; ++w2) pre += wc[w2 * G + lab];
+            const int pos = off[(long long)z * (G + 1) + lab] + bases[((long long)z * nch + ch) * G + lab] + pre + rank;
+            perm[(long long)z * n + pos] = i;
+        }
+        __syncthreads();
+        for (int g = threadIdx.x; g < G; g += blockDim.x) {
+            int add = 0;
+            for (int w2 = 0; w2 < 8; ++w2) { add += wc[w2 * G + g]; wc[w2 * G + g] = 0; }
+            run[g] += add;
+        }
+        __syncthreads();
     }
 }
 
@@ -263,13 +277,13 @@ cudaError_t launch_group_sort(const int32_t* labels, int32_t* perm, int32_t* off
                               int* bases, const int* done, int P, int n, int G, cudaStream_t s) {
     const int nch = (n + kSortChunk - 1) / kSortChunk;
     dim3 grid(nch, P);
-    sort_hist_kernel<<<grid, kSortChunk, G * sizeof(int), s>>>(labels, counts, done, n, G, nch);
+    sort_hist_kernel<<<grid, kSortSub, G * sizeof(int), s>>>(labels, counts, done, n, G, nch);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     sort_scan_kernel<<<P, 1024, G * sizeof(int), s>>>(counts, bases, off, done, G, nch);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    sort_scatter_kernel<<<grid, kSortChunk, 8 * G * sizeof(int), s>>>(labels, bases, off, perm, done, n, G, nch);
+    sort_scatter_kernel<<<grid, kSortSub, 9 * G * sizeof(int), s>>>(labels, bases, off, perm, done, n, G, nch);
     return cudaGetLastError();
 }
 
