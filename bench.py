@@ -333,9 +333,10 @@ def run_ours(args):
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         d0.record(stream)
         h.dense_attn(q, k, v, Od)
+        h.dense_attn(q, k, v, Od)
         d1.record(stream)
         torch.cuda.synchronize()
-        dms = reduce_max(d0.elapsed_time(d1), dev)
+        dms = reduce_max(d0.elapsed_time(d1) / 2.0, dev)
         dense = {"ms_per_call": dms, "tflops": flops / (dms * 1e-3) / 1e12, "speedup_vs_dense": dms / ms_max,
                  "frac_of_peak": flops / (dms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
 

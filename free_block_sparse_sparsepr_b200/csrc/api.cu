@@ -46,7 +46,8 @@ struct sparsepr_handle_s {
     float *u = nullptr, *ulse = nullptr;
     // route
     float* scores = nullptr;
-    int32_t *rowptr = nullptr, *kg = nullptr, *tile_off = nullptr;
+    int32_t *rowptr = nullptr, *kg = nullptr, *tile_off = nullptr, *ktile_cnt = nullptr, *ktile_off = nullptr;
+    int2* ktile_list = nullptr;
     int64_t* pairs = nullptr;
     // permuted tensors and sparse output
     bf16 *Qp = nullptr, *Kp = nullptr, *Vp = nullptr, *Osp = nullptr;
@@ -278,9 +279,12 @@ sparsepr_status attn_impl(sparsepr_handle h, const bf16* Qp, const bf16* Kp, con
                           cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
     if (spr::attn_tc_supported(c.d)) {
-        SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, 128, s));
-        SPR_TRY(spr::launch_attn_sparse_tc(Qp, Kp, Vp, p->qoff, p->koff, h->tile_off, r->rowptr, r->kg, Osp, lse,
-                                           c.B, c.Hq, c.Hkv, c.N, c.Gq, c.Gk, h->dev_status, s));
+        SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, spr::attn_tc_rows_per_cta(), s));
+        SPR_TRY(spr::launch_key_tiles(r->rowptr, r->kg, p->koff, h->ktile_cnt, h->ktile_off, h->ktile_list, h->P, c.N,
+                                      c.Gq, c.Gk, s));
+        h->launches += 2;  // count, scan and write kernels
+        SPR_TRY(spr::launch_attn_sparse_tc(Qp, Kp, Vp, p->qoff, h->tile_off, h->ktile_list, h->ktile_off, Osp, lse,
+                                           c.B, c.Hq, c.Hkv, c.N, c.Gq, h->dev_status, s));
         return SPARSEPR_OK;
     }
     SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, 64, s));
@@ -379,6 +383,8 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     }
     A_(scores, P * Gq * Gk); A_(rowptr, P * (Gq + 1)); A_(kg, P * Gq * Gk); A_(tile_off, P * (Gq + 1));
     A_(pairs, P);
+    A_(ktile_cnt, P * Gq); A_(ktile_off, P * (Gq + 1));
+    A_(ktile_list, P * (size_t)spr::key_tiles_capacity(c.N, c.Gq, c.Gk));
     A_(Qp, Hp * N * d); A_(Kp, P * N * d); A_(Vp, P * N * d); A_(Osp, Hp * N * d); A_(lse, Hp * N);
     A_(Opart, Hp * kProbeSplits * M * d); A_(mpart, Hp * kProbeSplits * M); A_(lpart, Hp * kProbeSplits * M);
     A_(Odense, Hp * M * d); A_(R, Hp * M * d); A_(Xprobe, Hp * M * d);

@@ -2,17 +2,20 @@
 // block-sparse pass over each query group's kept key groups, renormalised over
 // those keys only, and the dense baseline (one key range [0, N)).
 //
-// One CTA per 128-row query tile, six warps:
-//   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r; it reads its row
-//              of S from TMEM, keeps the running max / sum, writes P (bf16) into one of two
-//              shared-memory buffers in the 128-byte-swizzled K-major layout, rescales its O
-//              row in TMEM when the max grows by more than 2^8, and finally normalises and
-//              stores O;
-//   warp 4     TMA producer: Q once, then K and V tiles of 128 keys into a 2-stage ring;
-//   warp 5     TMEM allocation and the MMA issue (one elected thread): S = Q K^T into one of
-//              two TMEM buffers, O += P V into a third, completion signalled by tcgen05.commit.
-// With two P buffers the tensor core runs S(j+1) and PV(j) while the softmax warps work on
-// tile j+1; they wait for PV(j) only when their O row needs rescaling.
+// One CTA per pair of 128-row query tiles (t = 0, 1) of the same query group; both tiles
+// stream the same 128-key K/V tiles. Ten warps:
+//   warps 0-3 / 4-7  softmax + epilogue of tile 0 / tile 1: thread r owns query row r =
+//              TMEM lane r. Per key tile it reads its row of S_t from TMEM into registers,
+//              forms 2^(s c - m) against the running max, writes P_t as bf16 pairs into the first 64 columns of S_t's
+//              own TMEM buffer, rescales its O_t row when the max grows by more than 2^8, and
+//              finally normalises and stores O_t;
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles into a 2-stage ring;
+//   warp 9     TMEM allocation and the MMA issue (one thread): S_t = Q_t K^T (A and B from
+//              shared memory), O_t += P_t V (A from TMEM), completions via tcgen05.commit.
+// The tensor core alternates between the tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)), so one
+// softmax warpgroup works while the other's MMAs run. S_t(j+1) overwrites the columns P_t(j)
+// occupied only after PV_t(j) in issue order; its completion also tells softmax t that
+// PV_t(j) is done, so O_t may be rescaled and P_t(j+1) written.
 // Key tiles are cut from merged runs of consecutive kept key groups; keys past a run's end
 // (the next group's, or zero fill past the tensor) are masked to -inf.
 #include <cuda.h>
@@ -28,23 +31,21 @@
 namespace spr {
 namespace {
 
-constexpr int kBM = 128;            // query rows per CTA
+constexpr int kBM = 128;            // rows per query tile (two tiles per CTA)
 constexpr int kBN = 128;            // keys per tile
 constexpr int kD = 128;             // head dimension
 constexpr int kStages = 2;          // K/V ring depth
 constexpr int kRegion = 16384;      // one [128 rows][64 bf16] 128B-swizzled region
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512; // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512; // S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512)
 constexpr float kRescaleLog2 = 8.f; // lazy rescale threshold (P <= 2^8)
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + 2 * kRegion;
+constexpr int kOffQ = 0;                                   // tile t at + t * 2 * kRegion
+constexpr int kOffK = kOffQ + 2 * 2 * kRegion;
 constexpr int kOffV = kOffK + kStages * 2 * kRegion;
-constexpr int kOffP = kOffV + kStages * 2 * kRegion;
-constexpr int kOffBar = kOffP + 2 * 2 * kRegion;          // two P buffers
-// barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], mma_done
-// (s/p/o barriers indexed by tile parity so no waiter can fall two phases behind)
+constexpr int kOffBar = kOffV + kStages * 2 * kRegion;
+// barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_last[2], mma_done
 constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kStages, kBarE = kBarV + kStages, kBarS = kBarE + kStages,
               kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2, kNumBars = kBarMma + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;          // tmem base (u32), abort flag (int)
@@ -56,57 +57,62 @@ struct TcParams {
     bf16* O;
     float* lse;
     const int32_t* qoff;
-    const int32_t* koff;
-    const int32_t* tile_off;
-    const int32_t* rowptr;
-    const int32_t* kg;
+    const int32_t* tile_off;      // [P][Gq+1] CTA (query-tile pair) offsets per query group
+    const int2* klist;            // key tiles (start row, valid keys) of every query group
+    const int32_t* klist_off;     // [P][Gq+1] offsets into klist
     int* status;
-    int N, g, Gq, Gk;
+    int N, g, Gq;
     float scale_log2;
 };
 
-// Sequence of key tiles of one query tile (identical in every warp role).
-struct TileIter {
-    const int32_t* kept;
-    const int32_t* ko;
-    int ri, r1;
-    int lo, hi;     // current merged run
-    int t0;         // next tile start
-    bool dense;
-    __device__ __forceinline__ bool next_run() {
-        while (ri < r1) {
-            const int g0 = kept[ri++];
-            lo = ko[g0];
-            hi = ko[g0 + 1];
-            while (ri < r1 && ko[kept[ri]] == hi) { hi = ko[kept[ri] + 1]; ++ri; }
-            if (hi > lo) { t0 = lo; return true; }
+// Half h (64 columns) of this thread's row of S from TMEM, keys at or past `lim` set to -inf;
+// mx receives the half's raw maximum.
+__device__ __forceinline__ void load_half(uint32_t tS, int h, int lim, uint32_t (&sv)[2][32], float& mx) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tc::tmem_ld32(tS + 64 * h + 32 * c, sv[c]);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tc::regs_after_wait(sv[c]);
+    float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const int c0 = 64 * h + 32 * c;
+        if (c0 + 32 <= lim) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(sv[c][i]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (c0 + i >= lim) sv[c][i] = __float_as_uint(-INFINITY);
+                pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(sv[c][i]));
+            }
         }
-        return false;
     }
-    // Next tile: start row and number of valid keys (<= kBN); false when exhausted.
-    __device__ __forceinline__ bool next(int& start, int& lim) {
-        if (t0 >= hi) {
-            if (dense || !next_run()) return false;
-        }
-        start = t0;
-        lim = min(kBN, hi - t0);
-        t0 += kBN;
-        return true;
-    }
-};
+    mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+}
 
-__device__ __forceinline__ bool make_iter(const TcParams& p, int mode, int z, int a, TileIter& it) {
-    it.dense = mode == kModeDense;
-    if (it.dense) {
-        it.lo = 0; it.hi = p.N; it.t0 = 0; it.ri = it.r1 = 0; it.kept = nullptr; it.ko = nullptr;
-        return true;
+// p = 2^(s c + neg_m) for a half row, packed as bf16 pairs (32 registers), sums into ps.
+__device__ __forceinline__ void exp_half(const uint32_t (&sv)[2][32], float c_log2, float neg_m, uint32_t* pk,
+                                         float* ps) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float p0 = exp2f(fmaf(__uint_as_float(sv[c][2 * e]), c_log2, neg_m));
+            const float p1 = exp2f(fmaf(__uint_as_float(sv[c][2 * e + 1]), c_log2, neg_m));
+            ps[e & 7] += p0 + p1;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            pk[16 * c + e] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+}
+
+// Key tile j of the CTA: start row and number of valid keys (<= kBN).
+__device__ __forceinline__ int2 key_tile(const TcParams& p, int mode, const int2* list, int j) {
+    if (mode == kModeDense) {
+        const int st = j * kBN;
+        return make_int2(st, min(kBN, p.N - st));
     }
-    it.kept = p.kg + (long long)z * p.Gq * p.Gk;
-    it.ko = p.koff + (long long)z * (p.Gk + 1);
-    it.ri = p.rowptr[(long long)z * (p.Gq + 1) + a];
-    it.r1 = p.rowptr[(long long)z * (p.Gq + 1) + a + 1];
-    it.lo = it.hi = it.t0 = 0;
-    return true;
+    return list[j];
 }
 
 template <int MODE>
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t raw = tc::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     unsigned char* sbase = smem_raw + (base - raw);
-    const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV, sP = base + kOffP;
+    const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV;
     const uint32_t bars = base + kOffBar;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffMisc + 4);
@@ -129,23 +135,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // a CTA that timed out earlier in this launch (or call) makes the rest return at once
     if (p.status && *reinterpret_cast<volatile int*>(p.status) == kDevTimeout) return;
 
-    // ---- which query tile
-    int qlo, qn, a = 0;
+    // ---- which query tiles: rows [qlo, qlo + qn0) and [qlo + 128, qlo + 128 + qn1)
+    int qlo, qn0, qn1, a = 0, ntk = 0;
+    const int2* klist = nullptr;
     if (MODE == kModeSparse) {
         const int32_t* toff = p.tile_off + (long long)z * (p.Gq + 1);
-        const int tile = blockIdx.x;
-        if (tile >= toff[p.Gq]) return;
-        a = upper_index(toff, p.Gq, tile);
+        const int pair = blockIdx.x;
+        if (pair >= toff[p.Gq]) return;
+        a = upper_index(toff, p.Gq, pair);
+        const int32_t* lo = p.klist_off + (long long)z * (p.Gq + 1);
+        klist = p.klist + lo[a];
+        ntk = lo[a + 1] - lo[a];
         const int32_t* qo = p.qoff + (long long)z * (p.Gq + 1);
-        qlo = qo[a] + (tile - toff[a]) * kBM;
-        qn = min(kBM, qo[a + 1] - qlo);
+        qlo = qo[a] + (pair - toff[a]) * 2 * kBM;
+        const int rows = qo[a + 1] - qlo;
+        qn0 = min(kBM, rows);
+        qn1 = min(kBM, rows - kBM);
     } else {
-        qlo = blockIdx.x * kBM;
+        qlo = blockIdx.x * 2 * kBM;
         if (qlo >= p.N) return;
-        qn = min(kBM, p.N - qlo);
+        qn0 = min(kBM, p.N - qlo);
+        qn1 = min(kBM, p.N - qlo - kBM);
+        ntk = (p.N + kBN - 1) / kBN;
     }
+    const bool two = qn1 > 0;
 
-    // ---- set-up: barriers (thread 0), TMEM (warp 5)
+    // ---- set-up: barriers (thread 0), TMEM (warp 9)
     if (threadIdx.x == 0) {
         tc::mbar_init(bar(kBarQ), 1);
         for (int s = 0; s < kStages; ++s) {
@@ -153,16 +168,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             tc::mbar_init(bar(kBarV + s), 1);
             tc::mbar_init(bar(kBarE + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            tc::mbar_init(bar(kBarS + b), 1);
-            tc::mbar_init(bar(kBarP + b), 128);
-            tc::mbar_init(bar(kBarO + b), 1);
+        for (int t = 0; t < 2; ++t) {
+            tc::mbar_init(bar(kBarS + t), 1);
+            tc::mbar_init(bar(kBarP + t), 128);
+            tc::mbar_init(bar(kBarO + t), 1);
         }
         tc::mbar_init(bar(kBarMma), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tc::tmem_alloc(tc::smem_addr(tmem_slot), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -170,22 +185,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem, tO = tmem + 256;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ================= TMA producer
         if (lane == 0) {
             const int qrow = x * p.N + qlo;
-            tc::mbar_arrive_expect_tx(bar(kBarQ), 2 * kRegion);
+            tc::mbar_arrive_expect_tx(bar(kBarQ), (two ? 4 : 2) * kRegion);
             tc::tma_load_2d(sQ, &tmQ, bar(kBarQ), 0, qrow);
             tc::tma_load_2d(sQ + kRegion, &tmQ, bar(kBarQ), 64, qrow);
-            TileIter it;
-            make_iter(p, MODE, z, a, it);
-            int start, lim, j = 0;
-            while (it.next(start, lim)) {
+            if (two) {
+                tc::tma_load_2d(sQ + 2 * kRegion, &tmQ, bar(kBarQ), 0, qrow + kBM);
+                tc::tma_load_2d(sQ + 3 * kRegion, &tmQ, bar(kBarQ), 64, qrow + kBM);
+            }
+            int j = 0;
+            for (; j < ntk; ++j) {
                 const int s = j % kStages;
                 if (j >= kStages && !tc::mbar_wait(bar(kBarE + s), ((j / kStages) - 1) & 1, abort_flag)) break;
-                const int krow = z * p.N + start;
+                const int krow = z * p.N + key_tile(p, MODE, klist, j).x;
                 const uint32_t dk = sK + s * 2 * kRegion, dv = sV + s * 2 * kRegion;
                 tc::mbar_arrive_expect_tx(bar(kBarK + s), 2 * kRegion);
                 tc::tma_load_2d(dk, &tmK, bar(kBarK + s), 0, krow);
@@ -193,67 +209,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tc::mbar_arrive_expect_tx(bar(kBarV + s), 2 * kRegion);
                 tc::tma_load_2d(dv, &tmV, bar(kBarV + s), 0, krow);
                 tc::tma_load_2d(dv + kRegion, &tmV, bar(kBarV + s), 64, krow);
-                ++j;
             }
             // every issued load must land before the CTA can exit
+            int never = 0;
             for (int t = (j > kStages ? j - kStages : 0); t < j; ++t) {
                 const int s = t % kStages;
                 const uint32_t par = (t / kStages) & 1;
-                int dummy = 0;
-                volatile int* never = &dummy;
-                tc::mbar_wait(bar(kBarK + s), par, never);
-                tc::mbar_wait(bar(kBarV + s), par, never);
+                tc::mbar_wait(bar(kBarK + s), par, &never);
+                tc::mbar_wait(bar(kBarV + s), par, &never);
             }
-            tc::mbar_wait(bar(kBarQ), 0, abort_flag);
+            tc::mbar_wait(bar(kBarQ), 0, &never);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ================= MMA issuer
         const uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0);
         const uint32_t idO = tc::idesc_bf16_f32(kBM, kD, 1);
-        TileIter it;
-        make_iter(p, MODE, z, a, it);
-        int start, lim;
-        bool have = it.next(start, lim);
+        const int ntiles = two ? 2 : 1;
+        bool have = ntk > 0;
         bool ok = __all_sync(kFull, tc::mbar_wait(bar(kBarQ), 0, abort_flag));
-        auto issue_S = [&](int j) -> bool {
-            const int s = j % kStages;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarK + s), (j / kStages) & 1, abort_flag))) return false;
-            tc::fence_after_sync();
-            if (lane == 0) {
-                const uint32_t dS = tS0 + (uint32_t)((j & 1) * 128);
-                const uint32_t kb = sK + s * 2 * kRegion;
+        auto issue_S = [&](int t, int j) {
+            const uint32_t kb = sK + (j % kStages) * 2 * kRegion;
+            const uint32_t qb = sQ + t * 2 * kRegion;
 #pragma unroll
-                for (int k = 0; k < kD / 16; ++k) {
-                    const uint32_t off = (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
-                    tc::mma_f16_ss(dS, tc::smem_desc_sw128(sQ + off, 16, 1024), tc::smem_desc_sw128(kb + off, 16, 1024),
-                                   idS, k > 0 ? 1u : 0u);
-                }
-                tc::commit(bar(kBarS + (j & 1)));
+            for (int k = 0; k < kD / 16; ++k) {
+                const uint32_t off = (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
+                tc::mma_f16_ss(tmem + (uint32_t)(t * 128), tc::smem_desc_sw128(qb + off, 16, 1024),
+                               tc::smem_desc_sw128(kb + off, 16, 1024), idS, k > 0 ? 1u : 0u);
             }
-            __syncwarp();
-            return true;
+            tc::commit(bar(kBarS + t));
         };
         int j = 0;
-        if (ok && have) ok = issue_S(0);
-        while (ok && have) {
-            bool nhave = it.next(start, lim);
-            if (nhave && !issue_S(j + 1)) { ok = false; break; }
-            const int s = j % kStages;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarP + (j & 1)), (j >> 1) & 1, abort_flag))) { ok = false; break; }
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kStages) & 1, abort_flag))) { ok = false; break; }
-            tc::fence_after_sync();
-            if (lane == 0) {
-                const uint32_t vb = sV + s * 2 * kRegion;
-#pragma unroll
-                for (int k = 0; k < kBN / 16; ++k) {
-                    const uint32_t pa = sP + (uint32_t)((j & 1) * 2 * kRegion + (k >> 2) * kRegion + (k & 3) * 32);
-                    const uint32_t vbk = vb + (uint32_t)(k * 2048);
-                    tc::mma_f16_ss(tO, tc::smem_desc_sw128(pa, 16, 1024), tc::smem_desc_sw128(vbk, kRegion, 1024), idO,
-                                   (j > 0 || k > 0) ? 1u : 0u);
-                }
-                tc::commit(bar(kBarE + s));
-                tc::commit(bar(kBarO + (j & 1)));
+        if (ok && have) {
+            ok = __all_sync(kFull, tc::mbar_wait(bar(kBarK), 0, abort_flag));
+            if (ok) {
+                tc::fence_after_sync();
+                if (lane == 0)
+                    for (int t = 0; t < ntiles; ++t) issue_S(t, 0);
+                __syncwarp();
             }
+        }
+        while (ok && have) {
+            const bool nhave = j + 1 < ntk;
+            const int s = j % kStages;
+            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kStages) & 1, abort_flag))) break;
+            if (nhave && !__all_sync(kFull, tc::mbar_wait(bar(kBarK + ((j + 1) % kStages)), ((j + 1) / kStages) & 1,
+                                                         abort_flag)))
+                break;
+            for (int t = 0; t < ntiles && ok; ++t) {
+                if (!__all_sync(kFull, tc::mbar_wait(bar(kBarP + t), j & 1, abort_flag))) { ok = false; break; }
+                tc::fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t vb = sV + s * 2 * kRegion;
+                    const uint32_t pt = tmem + (uint32_t)(t * 128);       // P_t packed in S_t's columns
+#pragma unroll
+                    for (int k = 0; k < kBN / 16; ++k)
+                        tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
+                                       tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
+                                       (j > 0 || k > 0) ? 1u : 0u);
+                    if (nhave) issue_S(t, j + 1);
+                    else tc::commit(bar(kBarO + t));
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) tc::commit(bar(kBarE + s));
             __syncwarp();
             have = nhave;
             ++j;
@@ -261,139 +280,219 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // all issued MMAs complete before TMEM can be released
         if (lane == 0) tc::commit(bar(kBarMma));
         __syncwarp();
-        int dummy = 0;
-        tc::mbar_wait(bar(kBarMma), 0, &dummy);
+        int never = 0;
+        tc::mbar_wait(bar(kBarMma), 0, &never);
     } else {
-        // ================= softmax warps 0-3: thread r <-> query row r <-> TMEM lane r
-        const int r = threadIdx.x;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        TileIter it;
-        make_iter(p, MODE, z, a, it);
-        int start, lim, j = 0;
-        float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
-        const float c_log2 = p.scale_log2;
-        while (it.next(start, lim)) {
-            // every TMEM access below is warp-collective: decisions are made warp-uniform
-            const bool got_s = tc::mbar_wait(bar(kBarS + (j & 1)), (j >> 1) & 1, abort_flag);
-            if (!__all_sync(kFull, got_s)) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint32_t tS = tS0 + (uint32_t)((j & 1) * 128) + lane_off;
-            uint32_t sv[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS + 32 * c, sv[c]);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tc::regs_after_wait(sv[c]);
-            // row max of the raw logits; keys past the run's end are set to -inf
-            float mx = -INFINITY;
-            if (lim == kBN) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (32 * c + i >= lim) sv[c][i] = __float_as_uint(-INFINITY);
-                        mx = fmaxf(mx, __uint_as_float(sv[c][i]));
-                    }
-            }
-            const float m_new = fmaxf(m_run, mx * c_log2);
-            const bool rescale = m_new > m_run + kRescaleLog2;
-            if (j > 0 && __any_sync(kFull, rescale)) {
-                // O holds PV(0..j-1): wait for PV(j-1), then scale the rows whose max moved
-                const bool got_o = tc::mbar_wait(bar(kBarO + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag);
-                if (!__all_sync(kFull, got_o)) { ok = false; break; }
+        // ================= softmax warpgroup t: thread r <-> row r of tile t <-> TMEM lane r
+        const int t = warp >> 2;
+        const int r = threadIdx.x & 127;
+        const int qn = t == 0 ? qn0 : qn1;
+        if (qn > 0) {
+            const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+            const uint32_t tS = tmem + (uint32_t)(t * 128) + lane_off;
+            const uint32_t tO = tmem + 256 + (uint32_t)(t * 128) + lane_off;
+            const float c_log2 = p.scale_log2;
+            int j = 0;
+            float m_run = -INFINITY, l_run = 0.f;
+            bool ok = true;
+            int lim_next = ntk > 0 ? key_tile(p, MODE, klist, 0).y : 0;
+            for (; j < ntk; ++j) {
+                const int lim = lim_next;
+                if (j + 1 < ntk) lim_next = key_tile(p, MODE, klist, j + 1).y;   // prefetch
+                // every TMEM access below is warp-collective: decisions are made warp-uniform
+                const bool got_s = tc::mbar_wait(bar(kBarS + t), j & 1, abort_flag);
+                if (!__all_sync(kFull, got_s)) { ok = false; break; }
                 tc::fence_after_sync();
-                const float f = rescale ? exp2f(m_run - m_new) : 1.f;
+                // Half h of the row (64 columns) at a time. P of the first half is formed
+                // against the running max before the second half is seen and kept packed in
+                // registers; only when some row of the warp has a logit more than 2^8 above its
+                // running max (rare after the first tile) is the tile redone from S, which stays
+                // in TMEM until P is written.
+                const float thr = (m_run + kRescaleLog2) / c_log2;      // raw-logit threshold
+                uint32_t pk0[32];                                       // P of columns 0..63
+                float ps[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+                bool slow = false;
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+                {
+                    uint32_t sv[2][32];
+                    load_half(tS, 0, lim, sv, mx0);
+                    slow = __any_sync(kFull, mx0 > thr);
+                    if (!slow) exp_half(sv, c_log2, -m_run, pk0, ps);
+                }
+                {
+                    uint32_t sv[2][32];
+                    load_half(tS, 1, lim, sv, mx1);
+                    slow = slow || __any_sync(kFull, mx1 > thr);
+                    if (!slow) {
+                        uint32_t pk1[32];
+                        if (lim > 64) exp_half(sv, c_log2, -m_run, pk1, ps);
+                        else
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) pk1[e] = 0u;    // all keys of this half masked
+                        tc::tmem_st16(tS, pk0);
+                        tc::tmem_st16(tS + 16, pk0 + 16);
+                        tc::tmem_st16(tS + 32, pk1);
+                        tc::tmem_st16(tS + 48, pk1 + 16);
+                    }
+                }
+                if (slow) {
+                    // some row's max moved by more than 2^8: new per-row max, rescale O and l
+                    const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * c_log2);
+                    const bool rescale = m_new > m_run + kRescaleLog2;
+                    if (j > 0 && __any_sync(kFull, rescale)) {
+                        // S_t(j) complete => PV_t(j-1) complete: O_t may be rescaled now
+                        const float f = rescale ? exp2f(m_run - m_new) : 1.f;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t ov[32];
+                            tc::tmem_ld32(tO + 32 * c, ov);
+                            tc::tmem_wait_ld();
+                            tc::regs_after_wait(ov);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+                            tc::tmem_st32(tO + 32 * c, ov);
+                        }
+                        if (rescale) l_run *= f;
+                    }
+                    if (rescale) m_run = m_new;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+                    uint32_t pk1[32];
+                    {
+                        uint32_t sv[2][32];
+                        float dummy;
+                        load_half(tS, 0, lim, sv, dummy);
+                        exp_half(sv, c_log2, -m_run, pk0, ps);
+                    }
+                    if (lim > 64) {
+                        uint32_t sv[2][32];
+                        float dummy;
+                        load_half(tS, 1, lim, sv, dummy);
+                        exp_half(sv, c_log2, -m_run, pk1, ps);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pk1[e] = 0u;
+                    }
+                    tc::tmem_st16(tS, pk0);
+                    tc::tmem_st16(tS + 16, pk0 + 16);
+                    tc::tmem_st16(tS + 32, pk1);
+                    tc::tmem_st16(tS + 48, pk1 + 16);
+                }
+                l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                tc::mbar_arrive(bar(kBarP + t));
+            }
+            // epilogue: O / l, bf16 row store, lse
+            bool got_last = false;
+            if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO + t), 0, abort_flag);
+            if (j > 0 && __all_sync(kFull, got_last)) {
+                tc::fence_after_sync();
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                bf16* orow = p.O + ((long long)x * p.N + qlo + t * kBM + r) * kD;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t ov[32];
-                    tc::tmem_ld32(tO + lane_off + 32 * c, ov);
+                    tc::tmem_ld32(tO + 32 * c, ov);
                     tc::tmem_wait_ld();
                     tc::regs_after_wait(ov);
+                    if (r < qn) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-                    tc::tmem_st32(tO + lane_off + 32 * c, ov);
-                }
-                tc::tmem_wait_st();
-                if (rescale) l_run *= f;
-            }
-            if (rescale) m_run = m_new;
-            // P buffer j&1 was last read by PV(j-2)
-            if (j >= 2) {
-                const bool got_b = tc::mbar_wait(bar(kBarO + (j & 1)), ((j - 2) >> 1) & 1, abort_flag);
-                if (!__all_sync(kFull, got_b)) { ok = false; break; }
-            }
-            // P = 2^(s*c - m_run) as bf16, 16-byte chunks into the swizzled K-major P tile
-            unsigned char* prow = sbase + kOffP + (j & 1) * 2 * kRegion + r * 128;
-            const float neg_m = -m_run;
-            float sum = 0.f;
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t w[4];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int h = c >> 3, cc = c & 7;
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(fmaf(__uint_as_float(sv[c >> 2][(c & 3) * 8 + 2 * e]), c_log2, neg_m));
-                    const float p1 = exp2f(fmaf(__uint_as_float(sv[c >> 2][(c & 3) * 8 + 2 * e + 1]), c_log2, neg_m));
-                    sum += p0 + p1;
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<uint32_t*>(&b2);
-                }
-                *reinterpret_cast<uint4*>(prow + h * kRegion + ((cc ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            l_run += sum;
-            tc::fence_proxy_async_smem();
-            tc::fence_before_sync();
-            tc::mbar_arrive(bar(kBarP + (j & 1)));
-            ++j;
-        }
-        // epilogue: O / l, bf16 row store, lse
-        bool got_last = false;
-        if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag);
-        if (j > 0 && __all_sync(kFull, got_last)) {
-            tc::fence_after_sync();
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            bf16* orow = p.O + ((long long)x * p.N + qlo + r) * kD;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t ov[32];
-                tc::tmem_ld32(tO + lane_off + 32 * c, ov);
-                tc::tmem_wait_ld();
-                tc::regs_after_wait(ov);
-                if (r < qn) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q + 2 * e]) * inv,
-                                                                      __uint_as_float(ov[8 * q + 2 * e + 1]) * inv);
-                            w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(ov[8 * q + 2 * e]) * inv,
+                                                                          __uint_as_float(ov[8 * q + 2 * e + 1]) * inv);
+                                w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
                         }
-                        *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
+                if (r < qn && p.lse)
+                    p.lse[(long long)x * p.N + qlo + t * kBM + r] = (m_run + log2f(l_run)) * kLn2;
+            } else if (j == 0 && r < qn) {
+                bf16* orow = p.O + ((long long)x * p.N + qlo + t * kBM + r) * kD;
+                for (int c = 0; c < kD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                if (p.lse) p.lse[(long long)x * p.N + qlo + t * kBM + r] = -INFINITY;
             }
-            if (r < qn && p.lse) p.lse[(long long)x * p.N + qlo + r] = (m_run + log2f(l_run)) * kLn2;
-        } else if (j == 0 && r < qn) {
-            bf16* orow = p.O + ((long long)x * p.N + qlo + r) * kD;
-            for (int c = 0; c < kD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-            if (p.lse) p.lse[(long long)x * p.N + qlo + r] = -INFINITY;
         }
     }
 
     tc::fence_before_sync();
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kDevTimeout);
-    if (warp == 5) {
+    if (warp == 9) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// ---------------------------------------------------------------- key-tile lists
+// One warp per (KV head z, query group a): walk the kept key groups of route row a in
+// ascending order, merge groups whose key ranges touch (empty groups pass through), and
+// cut every merged run [lo, hi) into 128-key tiles. WRITE == false counts the tiles,
+// WRITE == true stores them at list + off[z][a].
+template <bool WRITE>
+__global__ void key_tiles_kernel(const int32_t* __restrict__ rowptr, const int32_t* __restrict__ kg,
+                                 const int32_t* __restrict__ koff, int32_t* cnt, const int32_t* __restrict__ off,
+                                 int2* list, int P, int Gq, int Gk) {
+    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= P * Gq) return;
+    const int z = wid / Gq, a = wid % Gq;
+    const int32_t* rp = rowptr + (long long)z * (Gq + 1);
+    const int32_t* kept = kg + (long long)z * Gq * Gk;
+    const int32_t* ko = koff + (long long)z * (Gk + 1);
+    const int r0 = rp[a], r1 = rp[a + 1];
+    int2* out = WRITE ? list + off[(long long)z * (Gq + 1) + a] : nullptr;
+    int ntiles = 0;
+    int cur_lo = 0, cur_hi = 0;
+    bool in_run = false;
+    auto emit = [&](int lo, int hi) {
+        if (hi <= lo) return;
+        const int nt = (hi - lo + kBN - 1) / kBN;
+        if (WRITE)
+            for (int t = lane; t < nt; t += 32) out[ntiles + t] = make_int2(lo + t * kBN, min(kBN, hi - lo - t * kBN));
+        ntiles += nt;
+    };
+    for (int c0 = r0; c0 < r1; c0 += 32) {
+        const int n = min(32, r1 - c0);
+        int glo = 0, ghi = 0;
+        if (lane < n) {
+            const int g = kept[c0 + lane];
+            glo = ko[g];
+            ghi = ko[g + 1];
+        }
+        for (int i = 0; i < n; ++i) {
+            const int lo = __shfl_sync(kFull, glo, i), hi = __shfl_sync(kFull, ghi, i);
+            if (in_run && lo == cur_hi) {
+                cur_hi = hi;
+            } else {
+                if (in_run) emit(cur_lo, cur_hi);
+                cur_lo = lo;
+                cur_hi = hi;
+                in_run = true;
+            }
+        }
+    }
+    if (in_run) emit(cur_lo, cur_hi);
+    if (!WRITE && lane == 0) cnt[(long long)z * Gq + a] = ntiles;
+}
+
+// off[z][a] = z * cap + sum_{a' < a} cnt[z][a']; one thread per KV head.
+__global__ void key_tiles_scan_kernel(const int32_t* __restrict__ cnt, int32_t* off, int P, int Gq, int cap) {
+    const int z = blockIdx.x * blockDim.x + threadIdx.x;
+    if (z >= P) return;
+    int s = z * cap;
+    for (int a = 0; a < Gq; ++a) {
+        off[(long long)z * (Gq + 1) + a] = s;
+        s += cnt[(long long)z * Gq + a];
+    }
+    off[(long long)z * (Gq + 1) + Gq] = s;
 }
 
 // ---------------------------------------------------------------- host side
@@ -428,21 +527,38 @@ TcParams params(bf16* O, float* lse, int N, int g, int* status) {
 
 bool attn_tc_supported(int d) { return d == kD; }
 
+int attn_tc_rows_per_cta() { return 2 * kBM; }
+
+long long key_tiles_capacity(int N, int Gq, int Gk) { return (long long)Gq * ((N + kBN - 1) / kBN + Gk); }
+
+cudaError_t launch_key_tiles(const int32_t* rowptr, const int32_t* kg, const int32_t* koff, int32_t* cnt,
+                             int32_t* off, int2* list, int P, int N, int Gq, int Gk, cudaStream_t s) {
+    const long long warps = (long long)P * Gq;
+    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
+    key_tiles_kernel<false><<<blocks, 256, 0, s>>>(rowptr, kg, koff, cnt, nullptr, nullptr, P, Gq, Gk);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    key_tiles_scan_kernel<<<(P + 127) / 128, 128, 0, s>>>(cnt, off, P, Gq, (int)key_tiles_capacity(N, Gq, Gk));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    key_tiles_kernel<true><<<blocks, 256, 0, s>>>(rowptr, kg, koff, cnt, off, list, P, Gq, Gk);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp, const int32_t* qoff,
-                                  const int32_t* koff, const int32_t* tile_off, const int32_t* rowptr,
-                                  const int32_t* kg, bf16* O, float* lse, int B, int Hq, int Hkv, int N, int Gq,
-                                  int Gk, int* status, cudaStream_t s) {
+                                  const int32_t* tile_off, const int2* klist, const int32_t* klist_off, bf16* O,
+                                  float* lse, int B, int Hq, int Hkv, int N, int Gq, int* status, cudaStream_t s) {
     TcParams p = params(O, lse, N, Hq / Hkv, status);
-    p.qoff = qoff; p.koff = koff; p.tile_off = tile_off; p.rowptr = rowptr; p.kg = kg;
-    p.Gq = Gq; p.Gk = Gk;
-    dim3 grid((N + kBM - 1) / kBM + Gq, B * Hq);
+    p.qoff = qoff; p.tile_off = tile_off; p.klist = klist; p.klist_off = klist_off;
+    p.Gq = Gq;
+    dim3 grid((N + 2 * kBM - 1) / (2 * kBM) + Gq, B * Hq);
     return launch_tc<kModeSparse>(Qp, Kp, Vp, p, B, Hq, Hkv, grid, s);
 }
 
 cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
                                  int Hkv, int N, int* status, cudaStream_t s) {
     TcParams p = params(O, lse, N, Hq / Hkv, status);
-    dim3 grid((N + kBM - 1) / kBM, B * Hq);
+    dim3 grid((N + 2 * kBM - 1) / (2 * kBM), B * Hq);
     return launch_tc<kModeDense>(Q, K, V, p, B, Hq, Hkv, grid, s);
 }
 

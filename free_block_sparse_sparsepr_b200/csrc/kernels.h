@@ -101,12 +101,17 @@ cudaError_t launch_attn_sparse(const bf16* Qp, const bf16* Kp, const bf16* Vp,
 // Dense attention of every query over all keys.
 cudaError_t launch_attn_dense(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse,
                               int B, int Hq, int Hkv, int N, int d, cudaStream_t s);
-// tcgen05/TMEM versions (head dimension 128): 128-row query tiles, 128-key tiles.
+// tcgen05/TMEM versions (head dimension 128): two 128-row query tiles per CTA, 128-key tiles.
 bool attn_tc_supported(int d);
+int attn_tc_rows_per_cta();
+// Key tiles (start row, valid keys) of every query group's merged kept runs: cnt [P][Gq]
+// scratch, off [P][Gq+1] absolute offsets, list of key_tiles_capacity(N, Gq, Gk) * P entries.
+long long key_tiles_capacity(int N, int Gq, int Gk);
+cudaError_t launch_key_tiles(const int32_t* rowptr, const int32_t* kg, const int32_t* koff, int32_t* cnt,
+                             int32_t* off, int2* list, int P, int N, int Gq, int Gk, cudaStream_t s);
 cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp, const int32_t* qoff,
-                                  const int32_t* koff, const int32_t* tile_off, const int32_t* rowptr,
-                                  const int32_t* kg, bf16* O, float* lse, int B, int Hq, int Hkv, int N, int Gq,
-                                  int Gk, int* status, cudaStream_t s);
+                                  const int32_t* tile_off, const int2* klist, const int32_t* klist_off, bf16* O,
+                                  float* lse, int B, int Hq, int Hkv, int N, int Gq, int* status, cudaStream_t s);
 cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
                                  int Hkv, int N, int* status, cudaStream_t s);
 // Dense attention of gathered probe rows, split over ns key chunks, then combined.
