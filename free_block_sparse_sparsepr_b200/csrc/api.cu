@@ -171,9 +171,16 @@ sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t
     return SPARSEPR_OK;
 }
 
-// u[x] = Q[x] . kcent[z]^T / sqrt(d) with kcent split into bf16 hi + lo.
-sparsepr_status query_logits(sparsepr_handle h, const bf16* Q, const bf16* chi, const bf16* clo, cudaStream_t s) {
+// u[x] = Q[x] . kcent[z]^T / sqrt(d) with kcent split into bf16 hi + lo, and the routing normaliser
+// ulse[x][i] = log sum_g |K_g| exp(u[x][i][g]) (fused into the tensor-core kernel's epilogue).
+sparsepr_status query_logits(sparsepr_handle h, const bf16* Q, const bf16* chi, const bf16* clo,
+                             const int32_t* koff, cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
+    if (spr::logits_tc_supported(c.d, c.Gk)) {
+        SPR_TRY(spr::launch_logits_tc(Q, chi, clo, koff, h->u, h->ulse, h->dev_status, c.B, c.Hq, c.Hkv, c.N, c.Gk,
+                                      h->num_sms, s));
+        return SPARSEPR_OK;
+    }
     spr::GemmArgs a;
     memset(&a, 0, sizeof(a));
     a.A1 = Q; a.A2 = nullptr; a.sA = (long long)c.N * c.d; a.lda = c.d;
@@ -182,6 +189,7 @@ sparsepr_status query_logits(sparsepr_handle h, const bf16* Q, const bf16* chi, 
     a.M = c.N; a.N = c.Gk; a.K = c.d; a.batch = h->Hp;
     a.alpha = (float)(1.0 / sqrt((double)c.d));
     SPR_TRY(spr::launch_gemm_bf16(a, s));
+    SPR_TRY(spr::launch_row_lse(h->u, koff, h->ulse, h->Hp, h->g, c.N, c.Gk, s));
     return SPARSEPR_OK;
 }
 
@@ -203,7 +211,7 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     if (st) return st;
     SPR_TRY(spr::launch_group_mean_bf16(K, h->kperm, h->koff, h->kcent, h->chi, h->clo, P, N, c.Gk, d, s));
     // (2b) query coordinates and query groups
-    st = query_logits(h, Q, h->chi, h->clo, s);
+    st = query_logits(h, Q, h->chi, h->clo, h->koff, s);
     if (st) return st;
     SPR_TRY(spr::launch_coords_center(h->u, h->uhi, h->ulo, h->ycoord, P, h->g, N, c.Gk, h->Gkp, h->DPy, h->proj, s));
     if (h->proj) {
@@ -254,10 +262,9 @@ sparsepr_status route_impl(sparsepr_handle h, const bf16* Q, const sparsepr_part
     const sparsepr_config& c = h->cfg;
     if (!logits_ready) {
         SPR_TRY(spr::launch_split_bf16(p->kcent, h->chi, h->clo, (long long)h->P * c.Gk * c.d, s));
-        sparsepr_status st = query_logits(h, Q, h->chi, h->clo, s);
+        sparsepr_status st = query_logits(h, Q, h->chi, h->clo, p->koff, s);
         if (st) return st;
     }
-    SPR_TRY(spr::launch_row_lse(h->u, p->koff, h->ulse, h->Hp, h->g, c.N, c.Gk, s));
     SPR_TRY(spr::launch_cell_scores(h->u, h->ulse, p->qperm, p->qoff, p->koff, h->scores, h->P, h->g, c.N,
                                     c.Gq, c.Gk, s));
     SPR_TRY(spr::launch_route_select(h->scores, p->qoff, p->koff, h->rowptr, h->kg, h->pairs, h->P, c.Gq, c.Gk,

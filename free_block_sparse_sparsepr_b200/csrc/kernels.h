@@ -44,6 +44,10 @@ cudaError_t launch_group_mean_bf16(const bf16* Y, const int32_t* perm, const int
 // Tensor-core assignment (G <= 256): rows and centroids split into three bf16 parts
 // (X3: [3][P][n][64], C3: [3][P][G16][64]).
 bool km_tc_supported(int G);
+bool logits_tc_supported(int d, int Gk);
+cudaError_t launch_logits_tc(const bf16* Q, const bf16* chi, const bf16* clo, const int32_t* koff, float* u,
+                             float* lse, int* status, int B, int Hq, int Hkv, int N, int Gk, int num_sms,
+                             cudaStream_t s);
 cudaError_t launch_km_split_rows(const float* X, bf16* X3, float* xx, int P, int n, int DP, cudaStream_t s);
 cudaError_t launch_km_split_cent(const float* C, bf16* C3, float* cc, int P, int G, int DP, cudaStream_t s);
 cudaError_t launch_km_assign_tc(const bf16* X3, const float* xx, const bf16* C3, const float* cc, int32_t* labels,

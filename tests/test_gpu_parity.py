@@ -26,6 +26,10 @@ CASES = {
     # ragged d=64: N=777, more query groups than key groups
     "ragged_d64_n777": Workload("ragged_d64_n777", B=1, Hq=3, Hkv=3, T=3, Hg=7, Wg=37, d=64, Gk=20, Gq=24,
                                 block=64, rho=0.35, M=32, r=12),
+    # ragged N=1500 with Gk=40 (a ragged column chunk) and GQA, d=128: the logits kernel's tiled
+    # stores must clip each head's last row tile at N and its last column chunk at Gk
+    "ragged_gqa_n1500_g40": Workload("ragged_gqa_n1500_g40", B=1, Hq=4, Hkv=2, T=5, Hg=15, Wg=20, d=128, Gk=40,
+                                     Gq=24, block=128, rho=0.3, M=48, r=16, locality=1.0, noise=0.3),
     # Gk > rQ: the query coordinates go through the +-1 projection
     "proj_n4096": Workload("proj_n4096", B=1, Hq=2, Hkv=2, T=4, Hg=32, Wg=32, d=128, Gk=96, Gq=80, block=128,
                            rho=0.25, locality=1.2),
