@@ -67,8 +67,10 @@ struct sparsepr_handle_s {
     bool user_events = false;
     bool timing = false, timed_call = false;
     // tensor-core k-means operands
-    bf16 *kmX3 = nullptr, *kmC3 = nullptr;
+    bf16 *kmX2 = nullptr, *kmC2 = nullptr;
     float *kmxx = nullptr, *kmcc = nullptr;
+    int4* kmfix = nullptr;
+    int* kmfix_count = nullptr;
     int launches = 0;
     int device = 0;
     int num_sms = 148;
@@ -142,21 +144,26 @@ long long budget_pairs(const sparsepr_config& c, int M) {
 }
 
 // Lloyd k-means on X [P][n][DP] into G groups, then the stable group-major order. With
-// G <= 256 the assignment runs on tensor cores (bf16 hi/lo split operands).
+// G <= 256 the assignment runs on tensor cores (bf16 split operands, near ties settled in fp64)
+// and the radial distances come from one exact pass after the last assignment.
 sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t* labels, float* dist,
                        int32_t* perm, int32_t* off, cudaStream_t s) {
     const int P = h->P, n = h->cfg.N;
     const bool tc = spr::km_tc_supported(G);
     auto assign = [&](bool first, const int* done) -> cudaError_t {
         if (!tc) return spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, done, P, n, G, DP, first, s);
-        cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC3, h->kmcc, P, G, DP, s);
+        cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC2, h->kmcc, h->kmfix_count, P, G, DP, s);
         if (e != cudaSuccess) return e;
         ++h->launches;
-        return spr::launch_km_assign_tc(h->kmX3, h->kmxx, h->kmC3, h->kmcc, labels, dist, h->km_changed, done,
-                                        h->dev_status, P, n, G, DP, first, h->num_sms, s);
+        e = spr::launch_km_assign_tc(X, h->kmX2, h->kmxx, h->kmC, h->kmC2, h->kmcc, labels, h->km_changed, done,
+                                     h->kmfix, h->kmfix_count, h->dev_status, P, n, G, DP, first, h->num_sms, s);
+        if (e != cudaSuccess) return e;
+        ++h->launches;
+        return spr::launch_km_fixup(h->kmfix, h->kmfix_count, X, h->kmC, labels, h->km_changed, n, G, DP,
+                                    h->num_sms, s);
     };
     SPR_TRY(spr::launch_km_reset(h->km_changed, h->km_done, P, s));
-    if (tc) SPR_TRY(spr::launch_km_split_rows(X, h->kmX3, h->kmxx, P, n, DP, s));
+    if (tc) SPR_TRY(spr::launch_km_split_rows(X, h->kmX2, h->kmxx, P, n, DP, s));
     SPR_TRY(spr::launch_km_seed(X, h->kmC, P, n, G, DP, s));
     SPR_TRY(assign(true, nullptr));
     for (int it = 0; it < h->cfg.kmeans_iters; ++it) {
@@ -166,6 +173,7 @@ sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t
         SPR_TRY(assign(false, h->km_done));
         SPR_TRY(spr::launch_km_check(h->km_changed, h->km_done, P, s));
     }
+    if (tc) SPR_TRY(spr::launch_km_dist(X, h->kmC, labels, dist, P, n, G, DP, s));
     SPR_TRY(spr::launch_group_sort(labels, perm, off, h->counts, h->bases, nullptr, P, n, G, s));
     h->launches += 2;
     return SPARSEPR_OK;
@@ -399,8 +407,9 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     A_(rank, Hp); A_(dev_status, 1);
     {
         const size_t G16 = (size_t)((h->Gmax + 15) / 16 * 16), G32 = (size_t)((h->Gmax + 31) / 32 * 32);
-        A_(kmX3, 3 * P * N * 64); A_(kmxx, P * N);
-        A_(kmC3, 3 * P * G16 * 64); A_(kmcc, P * G32);
+        A_(kmX2, 2 * P * N * 64); A_(kmxx, P * N);
+        A_(kmC2, 2 * P * G16 * 64); A_(kmcc, P * G32);
+        A_(kmfix, 3 * P * N); A_(kmfix_count, 1);
     }
 #undef A_
     bool ok = cudaMemset(h->dev_status, 0, sizeof(int)) == cudaSuccess;

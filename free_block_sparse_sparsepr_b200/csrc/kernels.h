@@ -41,18 +41,28 @@ cudaError_t launch_group_sort(const int32_t* labels, int32_t* perm, int32_t* off
 cudaError_t launch_group_mean_bf16(const bf16* Y, const int32_t* perm, const int32_t* off,
                                    float* cent, bf16* chi, bf16* clo, int P, int n, int G, int d,
                                    cudaStream_t s);
-// Tensor-core assignment (G <= 256): rows and centroids split into three bf16 parts
-// (X3: [3][P][n][64], C3: [3][P][G16][64]).
+// Tensor-core assignment (G <= 256): rows and centroids split into two bf16 parts
+// (X2: [2][P][n][DP] compact, C2: [2][P][G16][64]); near ties are settled exactly in fp64 from
+// the fp32 rows X and centroids C, so labels are the argmin of the fp32 distances.
 bool km_tc_supported(int G);
+cudaError_t launch_km_split_rows(const float* X, bf16* X2, float* xx, int P, int n, int DP, cudaStream_t s);
+cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int* fix_count, int P, int G, int DP,
+                                 cudaStream_t s);
+// fix: room for P*n flagged rows (3 int4 each); fix_count is cleared by launch_km_split_cent.
+cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx, const float* C, const bf16* C2,
+                                const float* cc, int32_t* labels, int* changed, const int* done, int4* fix,
+                                int* fix_count, int* status, int P, int n, int G, int DP, bool first, int num_sms,
+                                cudaStream_t s);
+// Exact fp64 resolution of the rows the assignment flagged (labels and moved counts corrected).
+cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, int32_t* labels,
+                            int* changed, int n, int G, int DP, int num_sms, cudaStream_t s);
+// dist[z][i] = fp32 of the fp64 squared distance of row i to its own centroid.
+cudaError_t launch_km_dist(const float* X, const float* C, const int32_t* labels, float* dist, int P, int n, int G,
+                           int DP, cudaStream_t s);
 bool logits_tc_supported(int d, int Gk);
 cudaError_t launch_logits_tc(const bf16* Q, const bf16* chi, const bf16* clo, const int32_t* koff, float* u,
                              float* lse, int* status, int B, int Hq, int Hkv, int N, int Gk, int num_sms,
                              cudaStream_t s);
-cudaError_t launch_km_split_rows(const float* X, bf16* X3, float* xx, int P, int n, int DP, cudaStream_t s);
-cudaError_t launch_km_split_cent(const float* C, bf16* C3, float* cc, int P, int G, int DP, cudaStream_t s);
-cudaError_t launch_km_assign_tc(const bf16* X3, const float* xx, const bf16* C3, const float* cc, int32_t* labels,
-                                float* dist, int* changed, const int* done, int* status, int P, int n, int G,
-                                int DP, bool first, int num_sms, cudaStream_t s);
 // Split fp32 group means into bf16 hi/lo (used when the partition is handed in).
 cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long count, cudaStream_t s);
 

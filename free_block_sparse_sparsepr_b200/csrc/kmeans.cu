@@ -91,7 +91,9 @@ __global__ void __launch_bounds__(kAssignRows) km_assign_kernel(const float* __r
     if ((threadIdx.x & 31) == 0 && b) atomicAdd(&changed[z], __popc(b));
 }
 
-// New centroid = mean of its members (perm/off order, 4 fixed row slices); empty keeps old.
+// New centroid = mean of its members in fp64 (perm/off order, kUpdSlices fixed row slices summed
+// in a fixed order), stored fp32; an empty group keeps its centroid.
+constexpr int kUpdSlices = 8;
 __global__ void km_update_kernel(const float* __restrict__ X, const int32_t* __restrict__ perm,
                                  const int32_t* __restrict__ off, float* C, const int* done, int n,
                                  int G, int DP) {
@@ -100,14 +102,27 @@ __global__ void km_update_kernel(const float* __restrict__ X, const int32_t* __r
     const int lo = off[(long long)z * (G + 1) + g], hi = off[(long long)z * (G + 1) + g + 1];
     if (hi <= lo) return;
     const int c = threadIdx.x % DP, rs = threadIdx.x / DP;
-    float acc = 0.f;
-    for (int j = lo + rs; j < hi; j += 4)
-        acc += X[((long long)z * n + perm[(long long)z * n + j]) * DP + c];
-    __shared__ float red[4][64];
-    red[rs][c] = acc;
+    const int32_t* pz = perm + (long long)z * n;
+    const float* xz = X + (long long)z * n * DP + c;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    int j = lo + rs;
+    for (; j + 3 * kUpdSlices < hi; j += 4 * kUpdSlices) {
+        const int r0 = __ldg(pz + j), r1 = __ldg(pz + j + kUpdSlices);
+        const int r2 = __ldg(pz + j + 2 * kUpdSlices), r3 = __ldg(pz + j + 3 * kUpdSlices);
+        const float v0 = __ldg(xz + (long long)r0 * DP), v1 = __ldg(xz + (long long)r1 * DP);
+        const float v2 = __ldg(xz + (long long)r2 * DP), v3 = __ldg(xz + (long long)r3 * DP);
+        a0 += (double)v0; a1 += (double)v1; a2 += (double)v2; a3 += (double)v3;
+    }
+    for (; j < hi; j += kUpdSlices) a0 += (double)__ldg(xz + (long long)__ldg(pz + j) * DP);
+    __shared__ double red[kUpdSlices][64];
+    red[rs][c] = (a0 + a1) + (a2 + a3);
     __syncthreads();
-    if (rs == 0)
-        C[((long long)z * G + g) * DP + c] = ((red[0][c] + red[1][c]) + (red[2][c] + red[3][c])) / (float)(hi - lo);
+    if (rs == 0) {
+        double t = 0.0;
+#pragma unroll
+        for (int k = 0; k < kUpdSlices; ++k) t += red[k][c];
+        C[((long long)z * G + g) * DP + c] = (float)(t / (double)(hi - lo));
+    }
 }
 
 __global__ void km_check_kernel(int* changed, int* done, int P) {
@@ -259,7 +274,7 @@ cudaError_t launch_km_assign(const float* X, const float* C, int32_t* labels, fl
 
 cudaError_t launch_km_update(const float* X, const int32_t* perm, const int32_t* off, float* C,
                              const int* done, int P, int n, int G, int DP, cudaStream_t s) {
-    km_update_kernel<<<dim3(G, P), 4 * DP, 0, s>>>(X, perm, off, C, done, n, G, DP);
+    km_update_kernel<<<dim3(G, P), kUpdSlices * DP, 0, s>>>(X, perm, off, C, done, n, G, DP);
     return cudaGetLastError();
 }
 

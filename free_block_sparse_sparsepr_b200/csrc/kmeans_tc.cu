@@ -1,16 +1,19 @@
-// Lloyd assignment step on 5th-generation tensor cores (G <= 256 groups).
+// Lloyd assignment step on 5th-generation tensor cores (G <= 256 groups), certified against
+// the fp32 value of the exact distance.
 //
-// For a tile of 128 rows the dot products with every centroid form one
-// 128 x G x D GEMM. Rows and centroids are split into three bf16 parts
-// (x = x0 + x1 + x2, each part the bf16 rounding of what the previous parts leave,
-// so |x - x0 - x1 - x2| <= 2^-27 |x|) and the product is accumulated in fp32 TMEM
-// from the six terms x_i c_j with i + j <= 2: the dot product to fp32 accuracy
-// (a two-part split, about 1e-5 relative, lets near-tie flips cascade through the
-// Lloyd rounds). One epilogue thread per row then takes
-// argmin_g (||c_g||^2 - 2 x.c_g) (ties -> lowest g) straight from its TMEM lane.
+// For a tile of 128 rows the dot products with every centroid form one 128 x G x D GEMM.
+// Rows and centroids are split into two bf16 parts (x = x0 + x1 + e, |e| <= 2^-16 |x|
+// elementwise) and the three terms x0 c0 + x0 c1 + x1 c0 are accumulated in fp32 TMEM, so
+// each dot product is known to within about 2^-14 ||x|| ||c||. One epilogue thread per row
+// takes the best and second-best of dd_g = ||c_g||^2 - 2 x.c_g straight from its TMEM lane.
+// When the gap between them exceeds a bound on the estimate's error the estimate decides;
+// otherwise (about 1% of rows) the row and its candidates (every group within the bound of
+// the best) go to a list, and a second kernel recomputes those candidates exactly:
+// ||x||^2 - 2 x.c + ||c||^2 in fp64 from the fp32 rows and centroids, rounded to fp32, ties to
+// the lowest group. The labels are therefore those of the fp32 distances themselves.
 //
-// Warps 0-3 epilogue, warp 4 TMA producer (centroids once, row tiles in a 2-stage
-// ring), warp 5 MMA issuer; TMEM holds two 256-column accumulators.
+// Warps 0-7 epilogue (two warpgroups taking alternate tiles, one TMEM buffer each), warp 8
+// TMA producer (centroids once, row tiles in a 3-stage ring), warp 9 MMA issuer.
 #include <float.h>
 #include <math.h>
 #include <string.h>
@@ -24,36 +27,56 @@ namespace spr {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kCols = 64;                 // padded feature width (one 128-byte swizzle row)
+constexpr int kCols = 64;                 // feature width of one 128-byte swizzle row
 constexpr int kMaxG = 256;
-constexpr int kTile = kRows * kCols * 2;  // 16 KB per hi or lo row tile
-constexpr int kThreads = 192;
+constexpr int kMaxDP = 64;
+constexpr int kTile = kRows * kCols * 2;  // 16 KB per part per row tile
+constexpr int kParts = 2;
+constexpr int kStages = 3;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kParts = 3;
 constexpr int kOffC = 0;                                     // part q at kOffC + q * kMaxG * 128
 constexpr int kOffX = kOffC + kParts * kMaxG * 128;          // stage s, part q at + (s * kParts + q) * kTile
-constexpr int kOffCC = kOffX + 2 * kParts * kTile;           // kMaxG floats
+constexpr int kOffCC = kOffX + kStages * kParts * kTile;     // kMaxG floats
 constexpr int kOffBar = kOffCC + kMaxG * 4;
-constexpr int kBarC = 0, kBarXF = 1, kBarXE = 3, kBarDF = 5, kBarDE = 7, kBarMma = 9, kNumBars = 10;
+constexpr int kBarC = 0, kBarXF = 1, kBarXE = kBarXF + kStages, kBarDF = kBarXE + kStages, kBarDE = kBarDF + 2,
+              kBarMma = kBarDE + 2, kNumBars = kBarMma + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// Gap below which a row is recomputed exactly: 4 kKappa ||x|| max_g ||c_g|| covers twice the
+// error of two dot-product estimates (each at most ~3.1 * 2^-16 ||x|| ||c|| from the dropped
+// split terms plus fp32 accumulation); kSlack (||x||^2 + max ||c||^2) covers the fp32
+// rounding of ||c||^2 and of dd.
+constexpr float kKappa = 1.0f / 8192.0f;   // 2^-13
+constexpr float kSlack = 1.0f / 65536.0f;  // 2^-16
 
 struct KmParams {
+    const float* X;        // [P][n][DP] fp32 rows
+    const float* C;        // [P][G][DP] fp32 centroids
     const float* xx;       // [P][n]
     const float* cc;       // [P][G32]  ||c||^2, +inf past G
     int32_t* labels;       // [P][n]
-    float* dist;           // [P][n]
     int* changed;          // [P]
     const int* done;       // [P] or null
     int* status;
-    int n, G16, G32, ksteps, first;
+    int4* fix;             // flagged rows: {row, previous label, estimate, 0}, then 8 candidate mask words
+    int* fix_count;
+    int n, G, G16, G32, DP, ksteps, first;
 };
 
 struct KmMaps {
-    CUtensorMap x[kParts];   // row parts [P*n][64] bf16
+    CUtensorMap x[kParts];   // row parts [P*n][DP] bf16 (columns DP..63 of a box read as zero)
     CUtensorMap c[kParts];   // centroid parts [P*G16][64] bf16
 };
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
 
 __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_constant__ KmMaps maps,
                                                                    const KmParams p) {
@@ -71,20 +94,22 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles = (p.n + kRows - 1) / kRows;
 
-    for (int t = threadIdx.x; t < p.G32; t += kThreads) sCC[t] = p.cc[(long long)z * p.G32 + t];
+    for (int t = threadIdx.x; t < kMaxG; t += kThreads) sCC[t] = t < p.G32 ? p.cc[(long long)z * p.G32 + t] : INFINITY;
     if (threadIdx.x == 0) {
         tc::mbar_init(bar(kBarC), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(bar(kBarXF + s), 1);
             tc::mbar_init(bar(kBarXE + s), 1);
-            tc::mbar_init(bar(kBarDF + s), 1);
-            tc::mbar_init(bar(kBarDE + s), 128);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(bar(kBarDF + b), 1);
+            tc::mbar_init(bar(kBarDE + b), 128);
         }
         tc::mbar_init(bar(kBarMma), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tc::tmem_alloc(tc::smem_addr(tmem_slot), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -93,54 +118,49 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
             tc::mbar_arrive_expect_tx(bar(kBarC), (uint32_t)kParts * (uint32_t)p.G16 * 128u);
             for (int q = 0; q < kParts; ++q)
                 tc::tma_load_2d(base + kOffC + q * kMaxG * 128, &maps.c[q], bar(kBarC), 0, z * p.G16);
             int i = 0;
             for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-                const int s = i & 1;
-                if (i >= 2 && !tc::mbar_wait(bar(kBarXE + s), ((i >> 1) - 1) & 1, abort_flag)) break;
+                const int s = i % kStages, u = i / kStages;
+                if (u >= 1 && !tc::mbar_wait(bar(kBarXE + s), (u - 1) & 1, abort_flag)) break;
                 const uint32_t dx = base + kOffX + s * kParts * kTile;
                 const int row = z * p.n + t * kRows;
                 tc::mbar_arrive_expect_tx(bar(kBarXF + s), kParts * kTile);
                 for (int q = 0; q < kParts; ++q) tc::tma_load_2d(dx + q * kTile, &maps.x[q], bar(kBarXF + s), 0, row);
             }
             int never = 0;
-            for (int k = (i > 2 ? i - 2 : 0); k < i; ++k) tc::mbar_wait(bar(kBarXF + (k & 1)), (k >> 1) & 1, &never);
+            for (int k = (i > kStages ? i - kStages : 0); k < i; ++k)
+                tc::mbar_wait(bar(kBarXF + k % kStages), (k / kStages) & 1, &never);
             tc::mbar_wait(bar(kBarC), 0, &never);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         const uint32_t idesc = tc::idesc_bf16_f32(kRows, p.G16, 0);
         bool ok = __all_sync(kFull, tc::mbar_wait(bar(kBarC), 0, abort_flag));
         int i = 0;
         for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
-            const int s = i & 1;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarXF + s), (i >> 1) & 1, abort_flag))) break;
-            if (i >= 2 && !__all_sync(kFull, tc::mbar_wait(bar(kBarDE + s), ((i >> 1) - 1) & 1, abort_flag))) break;
+            const int s = i % kStages, b = i & 1;
+            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarXF + s), (i / kStages) & 1, abort_flag))) break;
+            if (i >= 2 && !__all_sync(kFull, tc::mbar_wait(bar(kBarDE + b), ((i >> 1) - 1) & 1, abort_flag))) break;
             tc::fence_after_sync();
             if (lane == 0) {
-                const uint32_t d = tmem + (uint32_t)(s * 256);
+                const uint32_t d = tmem + (uint32_t)(b * 256);
                 const uint32_t xb = base + kOffX + s * kParts * kTile;
                 for (int k = 0; k < p.ksteps; ++k) {
                     const uint32_t off = (uint32_t)(k * 32);
-                    uint64_t dx[kParts], dc[kParts];
-#pragma unroll
-                    for (int q = 0; q < kParts; ++q) {
-                        dx[q] = tc::smem_desc_sw128(xb + q * kTile + off, 16, 1024);
-                        dc[q] = tc::smem_desc_sw128(base + kOffC + q * kMaxG * 128 + off, 16, 1024);
-                    }
-                    // terms x_i c_j with i + j <= 2, largest first
-                    tc::mma_f16_ss(d, dx[0], dc[0], idesc, k > 0 ? 1u : 0u);
-                    tc::mma_f16_ss(d, dx[0], dc[1], idesc, 1u);
-                    tc::mma_f16_ss(d, dx[1], dc[0], idesc, 1u);
-                    tc::mma_f16_ss(d, dx[0], dc[2], idesc, 1u);
-                    tc::mma_f16_ss(d, dx[2], dc[0], idesc, 1u);
-                    tc::mma_f16_ss(d, dx[1], dc[1], idesc, 1u);
+                    const uint64_t x0 = tc::smem_desc_sw128(xb + off, 16, 1024);
+                    const uint64_t x1 = tc::smem_desc_sw128(xb + kTile + off, 16, 1024);
+                    const uint64_t c0 = tc::smem_desc_sw128(base + kOffC + off, 16, 1024);
+                    const uint64_t c1 = tc::smem_desc_sw128(base + kOffC + kMaxG * 128 + off, 16, 1024);
+                    tc::mma_f16_ss(d, x0, c0, idesc, k > 0 ? 1u : 0u);
+                    tc::mma_f16_ss(d, x0, c1, idesc, 1u);
+                    tc::mma_f16_ss(d, x1, c0, idesc, 1u);
                 }
                 tc::commit(bar(kBarXE + s));
-                tc::commit(bar(kBarDF + s));
+                tc::commit(bar(kBarDF + b));
             }
             __syncwarp();
         }
@@ -149,62 +169,126 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
         int never = 0;
         tc::mbar_wait(bar(kBarMma), 0, &never);
     } else {
-        const int r = threadIdx.x;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        int i = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-            const int s = i & 1;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarDF + s), (i >> 1) & 1, abort_flag))) break;
+        const int wg = warp >> 2, wr = (warp & 3) * 32;
+        const uint32_t tb = tmem + (uint32_t)(wg * 256) + ((uint32_t)wr << 16);
+        // Columns [G16, G32) are never written by the MMA: make them read as zero (dd = +inf).
+        if (p.G16 < p.G32) {
+            uint32_t zr[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) zr[e] = 0u;
+            tc::tmem_st16(tb + (uint32_t)p.G16, zr);
+            tc::tmem_wait_st();
+        }
+        float cmax2 = 0.f;
+        for (int g = 0; g < p.G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
+        const float cmax = sqrtf(cmax2);
+        for (int i = wg, t = blockIdx.x + wg * gridDim.x; t < tiles; i += 2, t += 2 * gridDim.x) {
+            // The row's ||x||^2 and previous label are fetched before waiting for the tile.
+            const int row = t * kRows + wr + lane;
+            const bool valid = row < p.n;
+            const long long o = (long long)z * p.n + row;
+            const float xxr = valid ? __ldg(p.xx + o) : 0.f;
+            const int prev = (valid && !p.first) ? p.labels[o] : -1;
+            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarDF + wg), (i >> 1) & 1, abort_flag))) break;
             tc::fence_after_sync();
-            const uint32_t d = tmem + (uint32_t)(s * 256) + lane_off;
-            float best = FLT_MAX;
-            int bi = 0;
+            float b1[4], b2[4];
+            int i1[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { b1[j] = INFINITY; b2[j] = INFINITY; i1[j] = 0; }
             for (int c = 0; c < p.G32; c += 32) {
                 uint32_t v[32];
-                tc::tmem_ld32(d + c, v);
+                tc::tmem_ld32(tb + (uint32_t)c, v);
                 tc::tmem_wait_ld();
                 tc::regs_after_wait(v);
+                const float4* cc4 = reinterpret_cast<const float4*>(sCC + c);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float dd = fmaf(-2.f, __uint_as_float(v[e]), sCC[c + e]);
-                    if (dd < best) { best = dd; bi = c + e; }
+                for (int q = 0; q < 8; ++q) {
+                    const float4 cq = cc4[q];
+                    const float ce[4] = {cq.x, cq.y, cq.z, cq.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int e = 4 * q + j;
+                        const float dd = fmaf(-2.f, __uint_as_float(v[e]), ce[j]);
+                        b2[j] = fminf(b2[j], fmaxf(b1[j], dd));
+                        if (dd < b1[j]) { b1[j] = dd; i1[j] = c + e; }
+                    }
                 }
             }
-            tc::fence_before_sync();
-            tc::mbar_arrive(bar(kBarDE + s));
-            const int row = t * kRows + r;
-            int moved = 0;
-            if (row < p.n) {
-                const long long o = (long long)z * p.n + row;
-                if (!p.first && p.labels[o] != bi) moved = 1;
-                p.labels[o] = bi;
-                p.dist[o] = fmaxf(p.xx[o] + best, 0.f);
+            float B1 = b1[0];
+            int I1 = i1[0], jw = 0;
+#pragma unroll
+            for (int j = 1; j < 4; ++j)
+                if (b1[j] < B1 || (b1[j] == B1 && i1[j] < I1)) { B1 = b1[j]; I1 = i1[j]; jw = j; }
+            float B2 = INFINITY;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) B2 = fminf(B2, j == jw ? b2[j] : fminf(b1[j], b2[j]));
+
+            const float T = 4.f * kKappa * sqrtf(xxr) * cmax + kSlack * (xxr + cmax2);
+            const bool flag = valid && !(B2 - B1 > T);
+            if (__any_sync(kFull, flag)) {
+                // Candidates of each flagged row: every group with dd <= B1 + T (a bit per column).
+                const float thr = B1 + T;
+                uint32_t cm[kMaxG / 32];
+#pragma unroll
+                for (int k = 0; k < kMaxG / 32; ++k) {
+                    cm[k] = 0u;
+                    if (32 * k < p.G32) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(tb + (uint32_t)(32 * k), v);
+                        tc::tmem_wait_ld();
+                        tc::regs_after_wait(v);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float dd = fmaf(-2.f, __uint_as_float(v[e]), sCC[32 * k + e]);
+                            if (flag && dd <= thr) cm[k] |= 1u << e;
+                        }
+                    }
+                }
+                tc::fence_before_sync();
+                tc::mbar_arrive(bar(kBarDE + wg));
+                // Hand each flagged row, with its candidates, to the exact pass.
+                const unsigned fl = __ballot_sync(kFull, flag);
+                int slot = 0;
+                if (lane == 0) slot = atomicAdd(p.fix_count, __popc(fl));
+                slot = __shfl_sync(kFull, slot, 0) + __popc(fl & ((1u << lane) - 1u));
+                if (flag) {
+                    int4* ent = p.fix + 3ll * slot;
+                    ent[0] = make_int4((int)o, prev, I1, 0);
+                    ent[1] = make_int4((int)cm[0], (int)cm[1], (int)cm[2], (int)cm[3]);
+                    ent[2] = make_int4((int)cm[4], (int)cm[5], (int)cm[6], (int)cm[7]);
+                }
+            } else {
+                tc::fence_before_sync();
+                tc::mbar_arrive(bar(kBarDE + wg));
             }
-            const unsigned b = __ballot_sync(kFull, moved);
-            if (lane == 0 && b) atomicAdd(&p.changed[z], __popc(b));
+            int moved = 0;
+            if (valid) {
+                if (!p.first && prev != I1) moved = 1;
+                p.labels[o] = I1;
+            }
+            const unsigned bm = __ballot_sync(kFull, moved);
+            if (lane == 0 && bm) atomicAdd(&p.changed[z], __popc(bm));
         }
     }
 
     tc::fence_before_sync();
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kDevTimeout);
-    if (warp == 5) {
+    if (warp == 9) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-// The three bf16 parts of v: each part is the bf16 rounding of what the previous ones leave.
-__device__ __forceinline__ void split3(float v, bf16& a, bf16& b, bf16& c) {
+// The two bf16 parts of v: the bf16 rounding of v and of what it leaves.
+__device__ __forceinline__ void split2(float v, bf16& a, bf16& b) {
     a = __float2bfloat16_rn(v);
-    const float r1 = v - __bfloat162float(a);
-    b = __float2bfloat16_rn(r1);
-    c = __float2bfloat16_rn(r1 - __bfloat162float(b));
+    b = __float2bfloat16_rn(v - __bfloat162float(a));
 }
 
-// X [P][n][DP] fp32 -> three bf16 parts [P][n][64] (zero padded, part q at X3 + q*stride)
-// and ||x||^2; one warp per row.
-__global__ void km_split_rows_kernel(const float* __restrict__ X, bf16* X3, long long stride, float* xx,
+// X [rows][DP] fp32 -> two bf16 parts [rows][DP] (part q at X2 + q*stride) and ||x||^2 in fp32;
+// one warp per row.
+__global__ void km_split_rows_kernel(const float* __restrict__ X, bf16* X2, long long stride, float* xx,
                                      long long rows, int DP) {
     const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -213,23 +297,25 @@ __global__ void km_split_rows_kernel(const float* __restrict__ X, bf16* X3, long
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int c = lane + 32 * h;
-        const float v = c < DP ? X[row * DP + c] : 0.f;
-        ss = fmaf(v, v, ss);
-        bf16 a, b, e;
-        split3(v, a, b, e);
-        X3[row * kCols + c] = a;
-        X3[stride + row * kCols + c] = b;
-        X3[2 * stride + row * kCols + c] = e;
+        if (c < DP) {
+            const float v = X[row * DP + c];
+            ss = fmaf(v, v, ss);
+            bf16 a, b;
+            split2(v, a, b);
+            X2[row * DP + c] = a;
+            X2[stride + row * DP + c] = b;
+        }
     }
     ss = warp_sum(ss);
     if (lane == 0) xx[row] = ss;
 }
 
-// C [P][G][DP] fp32 -> three bf16 parts [P][G16][64] (zero rows past G, part q at C3 + q*stride)
-// and ||c||^2 [P][G32] (+inf past G so padded columns never win).
-__global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C3, long long stride, float* cc, int G,
-                                     int G16, int G32, int DP) {
+// C [P][G][DP] fp32 -> two bf16 parts [P][G16][64] (zero past G and DP, part q at C2 + q*stride)
+// and ||c||^2 [P][G32] (+inf past G so padded columns never win); also clears the flagged-row count.
+__global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long long stride, float* cc, int G,
+                                     int G16, int G32, int DP, int* fix_count) {
     const int z = blockIdx.y;
+    if (fix_count && blockIdx.x == 0 && z == 0 && threadIdx.x == 0) *fix_count = 0;
     const int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (g >= G32) return;
@@ -240,49 +326,123 @@ __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C3, long
         const float v = (g < G && c < DP) ? C[((long long)z * G + g) * DP + c] : 0.f;
         ss = fmaf(v, v, ss);
         if (g < G16) {
-            bf16 a, b, e;
-            split3(v, a, b, e);
+            bf16 a, b;
+            split2(v, a, b);
             const long long o = ((long long)z * G16 + g) * kCols + c;
-            C3[o] = a;
-            C3[stride + o] = b;
-            C3[2 * stride + o] = e;
+            C2[o] = a;
+            C2[stride + o] = b;
         }
     }
     ss = warp_sum(ss);
     if (lane == 0) cc[(long long)z * G32 + g] = g < G ? ss : INFINITY;
 }
 
+// Exact pass over the flagged rows (one warp per row): the fp32 value of the fp64 distance to
+// each candidate, argmin with ties to the lowest group; corrects the label and the count of
+// rows that moved.
+__global__ void km_fixup_kernel(const int4* __restrict__ fix, const int* __restrict__ fix_count,
+                                const float* __restrict__ X, const float* __restrict__ C, int32_t* labels,
+                                int* changed, int n, int G, int DP) {
+    const int lane = threadIdx.x & 31;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int cnt = *fix_count;
+    for (int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < cnt; w += nw) {
+        const int4 h = fix[3ll * w];
+        const int4 m0 = fix[3ll * w + 1], m1 = fix[3ll * w + 2];
+        const uint32_t mk[8] = {(uint32_t)m0.x, (uint32_t)m0.y, (uint32_t)m0.z, (uint32_t)m0.w,
+                                (uint32_t)m1.x, (uint32_t)m1.y, (uint32_t)m1.z, (uint32_t)m1.w};
+        const long long o = h.x;
+        const int z = (int)(o / n);
+        const float* xr = X + o * DP;
+        const double xa = lane < DP ? (double)xr[lane] : 0.0;
+        const double xb = lane + 32 < DP ? (double)xr[lane + 32] : 0.0;
+        const double xxd = warp_sum_d(xa * xa + xb * xb);
+        float best = INFINITY;
+        int bg = h.z;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            uint32_t m = mk[k];
+            while (m) {
+                const int g = 32 * k + __ffs(m) - 1;
+                m &= m - 1;
+                const float* cr = C + ((long long)z * G + g) * DP;
+                const double ca = lane < DP ? (double)cr[lane] : 0.0;
+                const double cb = lane + 32 < DP ? (double)cr[lane + 32] : 0.0;
+                const double xc = warp_sum_d(xa * ca + xb * cb);
+                const double ccd = warp_sum_d(ca * ca + cb * cb);
+                const float dg = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
+                if (dg < best) { best = dg; bg = g; }
+            }
+        }
+        if (lane == 0) {
+            labels[o] = bg;
+            const int prev = h.y;
+            if (prev >= 0) {
+                const int dmoved = (prev != bg ? 1 : 0) - (prev != h.z ? 1 : 0);
+                if (dmoved) atomicAdd(&changed[z], dmoved);
+            }
+        }
+    }
+}
+
+// dist[z][i] = fp32(max(||x||^2 - 2 x.c + ||c||^2, 0)) in fp64 for the row's own centroid;
+// one thread per row.
+__global__ void km_dist_kernel(const float* __restrict__ X, const float* __restrict__ C,
+                               const int32_t* __restrict__ labels, float* dist, int n, int G, int DP) {
+    const int z = blockIdx.y;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const long long o = (long long)z * n + i;
+    const float4* xr = reinterpret_cast<const float4*>(X + o * DP);
+    const float4* cr = reinterpret_cast<const float4*>(C + ((long long)z * G + labels[o]) * DP);
+    double xx = 0.0, xc = 0.0, cc = 0.0;
+    for (int k = 0; k < DP / 4; ++k) {
+        const float4 a = xr[k], b = __ldg(cr + k);
+        xx = fma((double)a.x, (double)a.x, xx); xx = fma((double)a.y, (double)a.y, xx);
+        xx = fma((double)a.z, (double)a.z, xx); xx = fma((double)a.w, (double)a.w, xx);
+        xc = fma((double)a.x, (double)b.x, xc); xc = fma((double)a.y, (double)b.y, xc);
+        xc = fma((double)a.z, (double)b.z, xc); xc = fma((double)a.w, (double)b.w, xc);
+        cc = fma((double)b.x, (double)b.x, cc); cc = fma((double)b.y, (double)b.y, cc);
+        cc = fma((double)b.z, (double)b.z, cc); cc = fma((double)b.w, (double)b.w, cc);
+    }
+    dist[o] = (float)fmax((xx - 2.0 * xc) + cc, 0.0);
+}
+
 }  // namespace
 
 bool km_tc_supported(int G) { return G >= 1 && G <= kMaxG; }
 
-cudaError_t launch_km_split_rows(const float* X, bf16* X3, float* xx, int P, int n, int DP, cudaStream_t s) {
+cudaError_t launch_km_split_rows(const float* X, bf16* X2, float* xx, int P, int n, int DP, cudaStream_t s) {
     const long long rows = (long long)P * n;
-    km_split_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(X, X3, rows * kCols, xx, rows, DP);
+    km_split_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(X, X2, rows * DP, xx, rows, DP);
     return cudaGetLastError();
 }
 
-cudaError_t launch_km_split_cent(const float* C, bf16* C3, float* cc, int P, int G, int DP, cudaStream_t s) {
+cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int* fix_count, int P, int G, int DP,
+                                 cudaStream_t s) {
     const int G16 = (G + 15) / 16 * 16, G32 = (G + 31) / 32 * 32;
-    km_split_cent_kernel<<<dim3((G32 + 7) / 8, P), 256, 0, s>>>(C, C3, (long long)P * G16 * kCols, cc, G, G16, G32,
-                                                                 DP);
+    km_split_cent_kernel<<<dim3((G32 + 7) / 8, P), 256, 0, s>>>(C, C2, (long long)P * G16 * kCols, cc, G, G16, G32,
+                                                                 DP, fix_count);
     return cudaGetLastError();
 }
 
-cudaError_t launch_km_assign_tc(const bf16* X3, const float* xx, const bf16* C3, const float* cc, int32_t* labels,
-                                float* dist, int* changed, const int* done, int* status, int P, int n, int G,
-                                int DP, bool first, int num_sms, cudaStream_t s) {
+cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx, const float* C, const bf16* C2,
+                                const float* cc, int32_t* labels, int* changed, const int* done, int4* fix,
+                                int* fix_count, int* status, int P, int n, int G, int DP, bool first, int num_sms,
+                                cudaStream_t s) {
+    if (DP < 16 || DP > kMaxDP || DP % 16 != 0 || (long long)P * n >= (1ll << 31)) return cudaErrorInvalidValue;
     const int G16 = (G + 15) / 16 * 16, G32 = (G + 31) / 32 * 32;
     KmMaps maps;
     for (int q = 0; q < kParts; ++q) {
-        if (!make_tmap_bf16_sw128(&maps.x[q], X3 + (long long)q * P * n * kCols, (long long)P * n, kCols, kRows, 64) ||
-            !make_tmap_bf16_sw128(&maps.c[q], C3 + (long long)q * P * G16 * kCols, (long long)P * G16, kCols, G16, 64))
+        if (!make_tmap_bf16_sw128(&maps.x[q], X2 + (long long)q * P * n * DP, (long long)P * n, DP, kRows, 64) ||
+            !make_tmap_bf16_sw128(&maps.c[q], C2 + (long long)q * P * G16 * kCols, (long long)P * G16, kCols, G16, 64))
             return cudaErrorInvalidValue;
     }
     KmParams p;
     memset(&p, 0, sizeof(p));
-    p.xx = xx; p.cc = cc; p.labels = labels; p.dist = dist; p.changed = changed; p.done = done; p.status = status;
-    p.n = n; p.G16 = G16; p.G32 = G32; p.ksteps = (DP + 15) / 16; p.first = first ? 1 : 0;
+    p.X = X; p.C = C; p.xx = xx; p.cc = cc; p.labels = labels; p.changed = changed; p.done = done;
+    p.status = status; p.fix = fix; p.fix_count = fix_count;
+    p.n = n; p.G = G; p.G16 = G16; p.G32 = G32; p.DP = DP; p.ksteps = DP / 16; p.first = first ? 1 : 0;
     const int tiles = (n + kRows - 1) / kRows;
     int per = num_sms / P;
     if (per < 1) per = 1;
@@ -290,6 +450,19 @@ cudaError_t launch_km_assign_tc(const bf16* X3, const float* xx, const bf16* C3,
     cudaError_t e = cudaFuncSetAttribute(km_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     km_assign_tc_kernel<<<dim3(per, P), kThreads, kSmemBytes, s>>>(maps, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, int32_t* labels,
+                            int* changed, int n, int G, int DP, int num_sms, cudaStream_t s) {
+    km_fixup_kernel<<<4 * num_sms, 256, 0, s>>>(fix, fix_count, X, C, labels, changed, n, G, DP);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_km_dist(const float* X, const float* C, const int32_t* labels, float* dist, int P, int n, int G,
+                           int DP, cudaStream_t s) {
+    if (DP % 4 != 0) return cudaErrorInvalidValue;
+    km_dist_kernel<<<dim3((n + 255) / 256, P), 256, 0, s>>>(X, C, labels, dist, n, G, DP);
     return cudaGetLastError();
 }
 
