@@ -152,15 +152,15 @@ sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t
     const bool tc = spr::km_tc_supported(G);
     auto assign = [&](bool first, const int* done) -> cudaError_t {
         if (!tc) return spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, done, P, n, G, DP, first, s);
-        cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC2, h->kmcc, h->kmfix_count, P, G, DP, s);
+        cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC2, h->kmcc, P, G, DP, s);
         if (e != cudaSuccess) return e;
         ++h->launches;
         e = spr::launch_km_assign_tc(X, h->kmX2, h->kmxx, h->kmC, h->kmC2, h->kmcc, labels, h->km_changed, done,
                                      h->kmfix, h->kmfix_count, h->dev_status, P, n, G, DP, first, h->num_sms, s);
         if (e != cudaSuccess) return e;
         ++h->launches;
-        return spr::launch_km_fixup(h->kmfix, h->kmfix_count, X, h->kmC, labels, h->km_changed, n, G, DP,
-                                    h->num_sms, s);
+        return spr::launch_km_fixup(h->kmfix, h->kmfix_count, X, h->kmC, h->kmcc, labels, h->km_changed, done, P, n,
+                                    G, DP, h->num_sms, s);
     };
     SPR_TRY(spr::launch_km_reset(h->km_changed, h->km_done, P, s));
     if (tc) SPR_TRY(spr::launch_km_split_rows(X, h->kmX2, h->kmxx, P, n, DP, s));
@@ -409,7 +409,7 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
         const size_t G16 = (size_t)((h->Gmax + 15) / 16 * 16), G32 = (size_t)((h->Gmax + 31) / 32 * 32);
         A_(kmX2, 2 * P * N * 64); A_(kmxx, P * N);
         A_(kmC2, 2 * P * G16 * 64); A_(kmcc, P * G32);
-        A_(kmfix, 3 * P * N); A_(kmfix_count, 1);
+        A_(kmfix, spr::km_fix_slots(P, N, h->num_sms)); A_(kmfix_count, P * h->num_sms);
     }
 #undef A_
     bool ok = cudaMemset(h->dev_status, 0, sizeof(int)) == cudaSuccess;

@@ -46,16 +46,18 @@ cudaError_t launch_group_mean_bf16(const bf16* Y, const int32_t* perm, const int
 // the fp32 rows X and centroids C, so labels are the argmin of the fp32 distances.
 bool km_tc_supported(int G);
 cudaError_t launch_km_split_rows(const float* X, bf16* X2, float* xx, int P, int n, int DP, cudaStream_t s);
-cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int* fix_count, int P, int G, int DP,
-                                 cudaStream_t s);
-// fix: room for P*n flagged rows (3 int4 each); fix_count is cleared by launch_km_split_cent.
+cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int P, int G, int DP, cudaStream_t s);
+// fix: km_fix_slots(P, n, num_sms) int4 slots (each CTA owns a region); fix_count: one int per
+// CTA (P * num_sms at most).
+size_t km_fix_slots(int P, int n, int num_sms);
 cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx, const float* C, const bf16* C2,
                                 const float* cc, int32_t* labels, int* changed, const int* done, int4* fix,
                                 int* fix_count, int* status, int P, int n, int G, int DP, bool first, int num_sms,
                                 cudaStream_t s);
 // Exact fp64 resolution of the rows the assignment flagged (labels and moved counts corrected).
-cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, int32_t* labels,
-                            int* changed, int n, int G, int DP, int num_sms, cudaStream_t s);
+cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, const float* cc,
+                            int32_t* labels, int* changed, const int* done, int P, int n, int G, int DP, int num_sms,
+                            cudaStream_t s);
 // dist[z][i] = fp32 of the fp64 squared distance of row i to its own centroid.
 cudaError_t launch_km_dist(const float* X, const float* C, const int32_t* labels, float* dist, int P, int n, int G,
                            int DP, cudaStream_t s);

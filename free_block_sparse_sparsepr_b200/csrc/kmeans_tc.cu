@@ -7,10 +7,11 @@
 // each dot product is known to within about 2^-14 ||x|| ||c||. One epilogue thread per row
 // takes the best and second-best of dd_g = ||c_g||^2 - 2 x.c_g straight from its TMEM lane.
 // When the gap between them exceeds a bound on the estimate's error the estimate decides;
-// otherwise (about 1% of rows) the row and its candidates (every group within the bound of
-// the best) go to a list, and a second kernel recomputes those candidates exactly:
-// ||x||^2 - 2 x.c + ||c||^2 in fp64 from the fp32 rows and centroids, rounded to fp32, ties to
-// the lowest group. The labels are therefore those of the fp32 distances themselves.
+// otherwise (about 1% of rows) the row goes to a list, and a second kernel settles it exactly:
+// an fp32 pass over all centroids keeps those within a relative 1e-4 of the nearest, and each
+// of those gets ||x||^2 - 2 x.c + ||c||^2 in fp64 from the fp32 rows and centroids, rounded to
+// fp32, ties to the lowest group. The labels are therefore those of the fp32 distances
+// themselves.
 //
 // Warps 0-7 epilogue (two warpgroups taking alternate tiles, one TMEM buffer each), warp 8
 // TMA producer (centroids once, row tiles in a 3-stage ring), warp 9 MMA issuer.
@@ -49,9 +50,11 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 // Gap below which a row is recomputed exactly: 4 kKappa ||x|| max_g ||c_g|| covers twice the
 // error of two dot-product estimates (each at most ~3.1 * 2^-16 ||x|| ||c|| from the dropped
 // split terms plus fp32 accumulation); kSlack (||x||^2 + max ||c||^2) covers the fp32
-// rounding of ||c||^2 and of dd.
+// rounding of ||c||^2 and of dd, and the low bits that the keys below give up to the column index.
 constexpr float kKappa = 1.0f / 8192.0f;   // 2^-13
-constexpr float kSlack = 1.0f / 65536.0f;  // 2^-16
+constexpr float kSlack = 1.0f / 32768.0f;  // 2^-15 (also covers the 5 index bits packed into keys)
+// ||c||^2 of padding columns: finite (so packed keys never form a NaN) and far above any distance.
+constexpr float kFar = 1.0e37f;
 
 struct KmParams {
     const float* X;        // [P][n][DP] fp32 rows
@@ -62,15 +65,22 @@ struct KmParams {
     int* changed;          // [P]
     const int* done;       // [P] or null
     int* status;
-    int4* fix;             // flagged rows: {row, previous label, estimate, 0}, then 8 candidate mask words
-    int* fix_count;
-    int n, G, G16, G32, DP, ksteps, first;
+    int4* fix;             // flagged rows {row, previous label, estimate, 0}; fix_cap slots per CTA
+    int* fix_count;        // [P * gridDim.x] rows each CTA flagged
+    int n, G, G16, G32, DP, ksteps, first, fix_cap;
 };
 
 struct KmMaps {
     CUtensorMap x[kParts];   // row parts [P*n][DP] bf16 (columns DP..63 of a box read as zero)
     CUtensorMap c[kParts];   // centroid parts [P*G16][64] bf16
 };
+
+// Three-input fp32 minimum.
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
@@ -90,12 +100,17 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
     float* sCC = reinterpret_cast<float*>(sbase + kOffCC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffMisc + 4);
+    int* sFix = reinterpret_cast<int*>(sbase + kOffMisc + 8);
+    // This CTA's region of the flagged-row list: one slot per row it can own.
+    const int cta = z * gridDim.x + blockIdx.x;
+    int4* fix = p.fix + (long long)cta * p.fix_cap;
     auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles = (p.n + kRows - 1) / kRows;
 
-    for (int t = threadIdx.x; t < kMaxG; t += kThreads) sCC[t] = t < p.G32 ? p.cc[(long long)z * p.G32 + t] : INFINITY;
+    for (int t = threadIdx.x; t < kMaxG; t += kThreads) sCC[t] = t < p.G32 ? p.cc[(long long)z * p.G32 + t] : kFar;
     if (threadIdx.x == 0) {
+        *sFix = 0;
         tc::mbar_init(bar(kBarC), 1);
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(bar(kBarXF + s), 1);
@@ -189,77 +204,83 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
             const long long o = (long long)z * p.n + row;
             const float xxr = valid ? __ldg(p.xx + o) : 0.f;
             const int prev = (valid && !p.first) ? p.labels[o] : -1;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarDF + wg), (i >> 1) & 1, abort_flag))) break;
-            tc::fence_after_sync();
+            // Keys: dd with its low 5 bits replaced by the column within the 32-column chunk,
+            // so one min also carries the argmin; four chains (column mod 4) for ILP, and the
+            // chunk that last lowered each chain's minimum.
             float b1[4], b2[4];
-            int i1[4];
+            int bc[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) { b1[j] = INFINITY; b2[j] = INFINITY; i1[j] = 0; }
-            for (int c = 0; c < p.G32; c += 32) {
-                uint32_t v[32];
-                tc::tmem_ld32(tb + (uint32_t)c, v);
-                tc::tmem_wait_ld();
-                tc::regs_after_wait(v);
+            for (int j = 0; j < 4; ++j) { b1[j] = INFINITY; b2[j] = INFINITY; bc[j] = 0; }
+            auto scan = [&](const uint32_t* v, int c) {
+                float old[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) old[j] = b1[j];
                 const float4* cc4 = reinterpret_cast<const float4*>(sCC + c);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 cq = cc4[q];
-                    const float ce[4] = {cq.x, cq.y, cq.z, cq.w};
+                for (int q = 0; q < 8; q += 2) {
+                    const float4 ca = cc4[q], cb = cc4[q + 1];
+                    const float ce[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const int e = 4 * q + j;
-                        const float dd = fmaf(-2.f, __uint_as_float(v[e]), ce[j]);
-                        b2[j] = fminf(b2[j], fmaxf(b1[j], dd));
-                        if (dd < b1[j]) { b1[j] = dd; i1[j] = c + e; }
+                        // Columns e and e + 4 of chain j: the two smallest of {b1, b2, k1, k2}.
+                        const uint32_t e = (uint32_t)(4 * q + j);
+                        const float d1 = fmaf(-2.f, __uint_as_float(v[e]), ce[j]);
+                        const float d2 = fmaf(-2.f, __uint_as_float(v[e + 4]), ce[j + 4]);
+                        const float k1 = __uint_as_float((__float_as_uint(d1) & ~31u) | e);
+                        const float k2 = __uint_as_float((__float_as_uint(d2) & ~31u) | (e + 4));
+                        const float lo = fminf(k1, k2), hi = fmaxf(k1, k2);
+                        b2[j] = fmin3(b2[j], fmaxf(b1[j], lo), hi);
+                        b1[j] = fminf(b1[j], lo);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) bc[j] = b1[j] != old[j] ? c : bc[j];
+            };
+            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarDF + wg), (i >> 1) & 1, abort_flag))) break;
+            tc::fence_after_sync();
+            {
+                uint32_t va[32], vb[32];
+                tc::tmem_ld32(tb, va);
+                tc::tmem_wait_ld();
+                tc::regs_after_wait(va);
+                for (int c = 0; c < p.G32; c += 64) {
+                    const bool hb = c + 32 < p.G32, ha = c + 64 < p.G32;
+                    if (hb) tc::tmem_ld32(tb + (uint32_t)(c + 32), vb);
+                    scan(va, c);
+                    if (hb) {
+                        tc::tmem_wait_ld();
+                        tc::regs_after_wait(vb);
+                        if (ha) tc::tmem_ld32(tb + (uint32_t)(c + 64), va);
+                        scan(vb, c + 32);
+                        if (ha) {
+                            tc::tmem_wait_ld();
+                            tc::regs_after_wait(va);
+                        }
                     }
                 }
             }
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(kBarDE + wg));
+            int jw = 0;
             float B1 = b1[0];
-            int I1 = i1[0], jw = 0;
+            int I1 = bc[0];
 #pragma unroll
             for (int j = 1; j < 4; ++j)
-                if (b1[j] < B1 || (b1[j] == B1 && i1[j] < I1)) { B1 = b1[j]; I1 = i1[j]; jw = j; }
+                if (b1[j] < B1) { B1 = b1[j]; I1 = bc[j]; jw = j; }
+            I1 += (int)(__float_as_uint(B1) & 31u);
             float B2 = INFINITY;
 #pragma unroll
             for (int j = 0; j < 4; ++j) B2 = fminf(B2, j == jw ? b2[j] : fminf(b1[j], b2[j]));
 
             const float T = 4.f * kKappa * sqrtf(xxr) * cmax + kSlack * (xxr + cmax2);
             const bool flag = valid && !(B2 - B1 > T);
-            if (__any_sync(kFull, flag)) {
-                // Candidates of each flagged row: every group with dd <= B1 + T (a bit per column).
-                const float thr = B1 + T;
-                uint32_t cm[kMaxG / 32];
-#pragma unroll
-                for (int k = 0; k < kMaxG / 32; ++k) {
-                    cm[k] = 0u;
-                    if (32 * k < p.G32) {
-                        uint32_t v[32];
-                        tc::tmem_ld32(tb + (uint32_t)(32 * k), v);
-                        tc::tmem_wait_ld();
-                        tc::regs_after_wait(v);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float dd = fmaf(-2.f, __uint_as_float(v[e]), sCC[32 * k + e]);
-                            if (flag && dd <= thr) cm[k] |= 1u << e;
-                        }
-                    }
-                }
-                tc::fence_before_sync();
-                tc::mbar_arrive(bar(kBarDE + wg));
-                // Hand each flagged row, with its candidates, to the exact pass.
-                const unsigned fl = __ballot_sync(kFull, flag);
+            // Hand each flagged row to the exact pass.
+            const unsigned fl = __ballot_sync(kFull, flag);
+            if (fl) {
                 int slot = 0;
-                if (lane == 0) slot = atomicAdd(p.fix_count, __popc(fl));
+                if (lane == 0) slot = atomicAdd(sFix, __popc(fl));
                 slot = __shfl_sync(kFull, slot, 0) + __popc(fl & ((1u << lane) - 1u));
-                if (flag) {
-                    int4* ent = p.fix + 3ll * slot;
-                    ent[0] = make_int4((int)o, prev, I1, 0);
-                    ent[1] = make_int4((int)cm[0], (int)cm[1], (int)cm[2], (int)cm[3]);
-                    ent[2] = make_int4((int)cm[4], (int)cm[5], (int)cm[6], (int)cm[7]);
-                }
-            } else {
-                tc::fence_before_sync();
-                tc::mbar_arrive(bar(kBarDE + wg));
+                if (flag) fix[slot] = make_int4((int)o, prev, I1, 0);
             }
             int moved = 0;
             if (valid) {
@@ -273,7 +294,10 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
 
     tc::fence_before_sync();
     __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kDevTimeout);
+    if (threadIdx.x == 0) {
+        if (*abort_flag) set_status(p.status, kDevTimeout);
+        p.fix_count[cta] = *sFix;
+    }
     if (warp == 9) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
@@ -311,11 +335,10 @@ __global__ void km_split_rows_kernel(const float* __restrict__ X, bf16* X2, long
 }
 
 // C [P][G][DP] fp32 -> two bf16 parts [P][G16][64] (zero past G and DP, part q at C2 + q*stride)
-// and ||c||^2 [P][G32] (+inf past G so padded columns never win); also clears the flagged-row count.
+// and ||c||^2 [P][G32] (kFar past G so padded columns never win).
 __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long long stride, float* cc, int G,
-                                     int G16, int G32, int DP, int* fix_count) {
+                                     int G16, int G32, int DP) {
     const int z = blockIdx.y;
-    if (fix_count && blockIdx.x == 0 && z == 0 && threadIdx.x == 0) *fix_count = 0;
     const int g = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (g >= G32) return;
@@ -334,44 +357,85 @@ __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long
         }
     }
     ss = warp_sum(ss);
-    if (lane == 0) cc[(long long)z * G32 + g] = g < G ? ss : INFINITY;
+    if (lane == 0) cc[(long long)z * G32 + g] = g < G ? ss : kFar;
 }
 
-// Exact pass over the flagged rows (one warp per row): the fp32 value of the fp64 distance to
-// each candidate, argmin with ties to the lowest group; corrects the label and the count of
-// rows that moved.
-__global__ void km_fixup_kernel(const int4* __restrict__ fix, const int* __restrict__ fix_count,
-                                const float* __restrict__ X, const float* __restrict__ C, int32_t* labels,
-                                int* changed, int n, int G, int DP) {
-    const int lane = threadIdx.x & 31;
-    const int nw = (gridDim.x * blockDim.x) >> 5;
-    const int cnt = *fix_count;
-    for (int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < cnt; w += nw) {
-        const int4 h = fix[3ll * w];
-        const int4 m0 = fix[3ll * w + 1], m1 = fix[3ll * w + 2];
-        const uint32_t mk[8] = {(uint32_t)m0.x, (uint32_t)m0.y, (uint32_t)m0.z, (uint32_t)m0.w,
-                                (uint32_t)m1.x, (uint32_t)m1.y, (uint32_t)m1.z, (uint32_t)m1.w};
+// Exact pass over the flagged rows: one block per assignment CTA (its centroids staged in shared
+// memory k-major), one warp per row, the row in registers. Candidates are the groups whose fp32
+// ||x||^2 - 2 x.c + ||c||^2 (error below 2^-19 (||x||^2 + ||c||^2)) is within 1e-4 (d + ||x||^2
+// + max ||c||^2) of the smallest; each gets the fp32 value of its fp64 distance, argmin with ties
+// to the lowest group. Corrects the label and the count of rows that moved.
+constexpr int kFixThreads = 512;
+template <int DP>
+__global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __restrict__ fix,
+                                                               const int* __restrict__ fix_count,
+                                                               const float* __restrict__ X,
+                                                               const float* __restrict__ C,
+                                                               const float* __restrict__ cc, int32_t* labels,
+                                                               int* changed, const int* done, int n, int G, int G32,
+                                                               int fix_cap) {
+    const int z = blockIdx.y;
+    if (done && done[z]) return;
+    const int cta = z * gridDim.x + blockIdx.x;
+    const int cnt = fix_count[cta];
+    if (cnt == 0) return;
+    extern __shared__ float fsm[];
+    float* sC = fsm;                          // [DP][kMaxG], k-major
+    float* sCC = fsm + DP * kMaxG;            // [kMaxG]
+    for (int t = threadIdx.x; t < G * DP; t += blockDim.x) sC[(t % DP) * kMaxG + t / DP] = C[(long long)z * G * DP + t];
+    for (int t = threadIdx.x; t < kMaxG; t += blockDim.x) sCC[t] = t < G ? cc[(long long)z * G32 + t] : 0.f;
+    __syncthreads();
+    float cmax2 = 0.f;
+    for (int g = 0; g < G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
+    const int4* reg = fix + (long long)cta * fix_cap;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int w = warp; w < cnt; w += kFixThreads / 32) {
+        const int4 h = reg[w];
         const long long o = h.x;
-        const int z = (int)(o / n);
         const float* xr = X + o * DP;
+        float x[DP];
+#pragma unroll
+        for (int k = 0; k < DP; k += 4) {
+            const float4 q = __ldg(reinterpret_cast<const float4*>(xr + k));
+            x[k] = q.x; x[k + 1] = q.y; x[k + 2] = q.z; x[k + 3] = q.w;
+        }
+        float xx = 0.f;
+#pragma unroll
+        for (int k = 0; k < DP; ++k) xx = fmaf(x[k], x[k], xx);
+        float dg[kMaxG / 32];
+        float dmin = INFINITY;
+#pragma unroll
+        for (int j = 0; j < kMaxG / 32; ++j) {
+            const int g = lane + 32 * j;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < DP; k += 2) {
+                a0 = fmaf(x[k], sC[k * kMaxG + g], a0);
+                a1 = fmaf(x[k + 1], sC[(k + 1) * kMaxG + g], a1);
+            }
+            const float d = g < G ? fmaf(-2.f, a0 + a1, xx + sCC[g]) : INFINITY;
+            dg[j] = d;
+            dmin = fminf(dmin, d);
+        }
+        dmin = warp_min(dmin);
+        const float thr = dmin + 1e-4f * (fabsf(dmin) + xx + cmax2);
         const double xa = lane < DP ? (double)xr[lane] : 0.0;
         const double xb = lane + 32 < DP ? (double)xr[lane + 32] : 0.0;
         const double xxd = warp_sum_d(xa * xa + xb * xb);
         float best = INFINITY;
         int bg = h.z;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            uint32_t m = mk[k];
+        for (int j = 0; j < kMaxG / 32; ++j) {
+            uint32_t m = __ballot_sync(kFull, dg[j] <= thr);
             while (m) {
-                const int g = 32 * k + __ffs(m) - 1;
+                const int g = 32 * j + __ffs(m) - 1;
                 m &= m - 1;
-                const float* cr = C + ((long long)z * G + g) * DP;
-                const double ca = lane < DP ? (double)cr[lane] : 0.0;
-                const double cb = lane + 32 < DP ? (double)cr[lane + 32] : 0.0;
+                const double ca = lane < DP ? (double)sC[lane * kMaxG + g] : 0.0;
+                const double cb = lane + 32 < DP ? (double)sC[(lane + 32) * kMaxG + g] : 0.0;
                 const double xc = warp_sum_d(xa * ca + xb * cb);
                 const double ccd = warp_sum_d(ca * ca + cb * cb);
-                const float dg = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
-                if (dg < best) { best = dg; bg = g; }
+                const float d = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
+                if (d < best) { best = d; bg = g; }
             }
         }
         if (lane == 0) {
@@ -412,17 +476,26 @@ __global__ void km_dist_kernel(const float* __restrict__ X, const float* __restr
 
 bool km_tc_supported(int G) { return G >= 1 && G <= kMaxG; }
 
+// Grid of the assignment: per CTAs for each of the P problems, each owning at most cap rows.
+void km_grid(int P, int n, int num_sms, int* per, int* cap) {
+    const int tiles = (n + kRows - 1) / kRows;
+    int q = num_sms / P;
+    if (q < 1) q = 1;
+    if (q > tiles) q = tiles;
+    *per = q;
+    *cap = (tiles + q - 1) / q * kRows;
+}
+
 cudaError_t launch_km_split_rows(const float* X, bf16* X2, float* xx, int P, int n, int DP, cudaStream_t s) {
     const long long rows = (long long)P * n;
     km_split_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(X, X2, rows * DP, xx, rows, DP);
     return cudaGetLastError();
 }
 
-cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int* fix_count, int P, int G, int DP,
-                                 cudaStream_t s) {
+cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int P, int G, int DP, cudaStream_t s) {
     const int G16 = (G + 15) / 16 * 16, G32 = (G + 31) / 32 * 32;
     km_split_cent_kernel<<<dim3((G32 + 7) / 8, P), 256, 0, s>>>(C, C2, (long long)P * G16 * kCols, cc, G, G16, G32,
-                                                                 DP, fix_count);
+                                                                 DP);
     return cudaGetLastError();
 }
 
@@ -443,20 +516,47 @@ cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx,
     p.X = X; p.C = C; p.xx = xx; p.cc = cc; p.labels = labels; p.changed = changed; p.done = done;
     p.status = status; p.fix = fix; p.fix_count = fix_count;
     p.n = n; p.G = G; p.G16 = G16; p.G32 = G32; p.DP = DP; p.ksteps = DP / 16; p.first = first ? 1 : 0;
-    const int tiles = (n + kRows - 1) / kRows;
-    int per = num_sms / P;
-    if (per < 1) per = 1;
-    if (per > tiles) per = tiles;
+    int per, cap;
+    km_grid(P, n, num_sms, &per, &cap);
+    p.fix_cap = cap;
     cudaError_t e = cudaFuncSetAttribute(km_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     km_assign_tc_kernel<<<dim3(per, P), kThreads, kSmemBytes, s>>>(maps, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, int32_t* labels,
-                            int* changed, int n, int G, int DP, int num_sms, cudaStream_t s) {
-    km_fixup_kernel<<<4 * num_sms, 256, 0, s>>>(fix, fix_count, X, C, labels, changed, n, G, DP);
+cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, const float* cc,
+                            int32_t* labels, int* changed, const int* done, int P, int n, int G, int DP, int num_sms,
+                            cudaStream_t s) {
+    int per, cap;
+    km_grid(P, n, num_sms, &per, &cap);
+    const int G32 = (G + 31) / 32 * 32;
+    const size_t smem = ((size_t)DP * kMaxG + kMaxG) * sizeof(float);
+    const dim3 grid(per, P);
+#define SPR_FIXUP(DPV)                                                                                               \
+    case DPV: {                                                                                                      \
+        cudaError_t e = cudaFuncSetAttribute(km_fixup_kernel<DPV>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
+                                             (int)smem);                                                             \
+        if (e != cudaSuccess) return e;                                                                              \
+        km_fixup_kernel<DPV><<<grid, kFixThreads, smem, s>>>(fix, fix_count, X, C, cc, labels, changed, done, n, G,  \
+                                                            G32, cap);                                               \
+        break;                                                                                                       \
+    }
+    switch (DP) {
+        SPR_FIXUP(16)
+        SPR_FIXUP(32)
+        SPR_FIXUP(48)
+        SPR_FIXUP(64)
+        default: return cudaErrorInvalidValue;
+    }
+#undef SPR_FIXUP
     return cudaGetLastError();
+}
+
+size_t km_fix_slots(int P, int n, int num_sms) {
+    int per, cap;
+    km_grid(P, n, num_sms, &per, &cap);
+    return (size_t)P * per * cap;
 }
 
 cudaError_t launch_km_dist(const float* X, const float* C, const int32_t* labels, float* dist, int P, int n, int G,
