@@ -45,9 +45,12 @@ constexpr int kOffQ = 0;                                   // tile t at + t * 2 
 constexpr int kOffK = kOffQ + 2 * 2 * kRegion;
 constexpr int kOffV = kOffK + kStages * 2 * kRegion;
 constexpr int kOffBar = kOffV + kStages * 2 * kRegion;
-// barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_last[2], mma_done
-constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kStages, kBarE = kBarV + kStages, kBarS = kBarE + kStages,
-              kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2, kNumBars = kBarMma + 1;
+// barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_last[2],
+// mma_done. K and V stages are released separately: a K tile as soon as the last S MMA that
+// reads it completes, a V tile after the last PV MMA, so the next K load starts a step early.
+constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kStages, kBarEK = kBarV + kStages, kBarEV = kBarEK + kStages,
+              kBarS = kBarEV + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2,
+              kNumBars = kBarMma + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;          // tmem base (u32), abort flag (int)
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;          // + slack to align the base to 1024
 
@@ -65,6 +68,13 @@ struct TcParams {
     float scale_log2;
 };
 
+// Three-input fp32 maximum.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Half h (64 columns) of this thread's row of S from TMEM, keys at or past `lim` set to -inf;
 // mx receives the half's raw maximum.
 __device__ __forceinline__ void load_half(uint32_t tS, int h, int lim, uint32_t (&sv)[2][32], float& mx) {
@@ -77,30 +87,58 @@ __device__ __forceinline__ void load_half(uint32_t tS, int h, int lim, uint32_t 
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         const int c0 = 64 * h + 32 * c;
-        if (c0 + 32 <= lim) {
+        if (c0 + 32 > lim) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(sv[c][i]));
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 32; ++i)
                 if (c0 + i >= lim) sv[c][i] = __float_as_uint(-INFINITY);
-                pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(sv[c][i]));
-            }
         }
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            pm[(i >> 1) & 3] = fmax3(pm[(i >> 1) & 3], __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
     }
-    mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+    mx = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
 }
 
-// p = 2^(s c + neg_m) for a half row, packed as bf16 pairs (32 registers), sums into ps.
+// 2^x on the special-function unit (flushes results below 2^-126 to zero).
+__device__ __forceinline__ float ex2_sfu(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Pairs of fp32 in one 64-bit register, for the packed f32x2 arithmetic of sm_100.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// p = 2^(s c + neg_m) for a half row, packed as bf16 pairs (32 registers); pair sums into ps
+// (four packed accumulators).
 __device__ __forceinline__ void exp_half(const uint32_t (&sv)[2][32], float c_log2, float neg_m, uint32_t* pk,
-                                         float* ps) {
+                                         uint64_t* ps) {
+    const uint64_t cc = pk2(c_log2, c_log2), nm = pk2(neg_m, neg_m);
 #pragma unroll
     for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const float p0 = exp2f(fmaf(__uint_as_float(sv[c][2 * e]), c_log2, neg_m));
-            const float p1 = exp2f(fmaf(__uint_as_float(sv[c][2 * e + 1]), c_log2, neg_m));
-            ps[e & 7] += p0 + p1;
+            float x0, x1;
+            up2(fma2(pk2(__uint_as_float(sv[c][2 * e]), __uint_as_float(sv[c][2 * e + 1])), cc, nm), x0, x1);
+            const float p0 = ex2_sfu(x0), p1 = ex2_sfu(x1);
+            ps[e & 3] = add2(ps[e & 3], pk2(p0, p1));
             __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
             pk[16 * c + e] = *reinterpret_cast<uint32_t*>(&b2);
         }
@@ -166,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(bar(kBarK + s), 1);
             tc::mbar_init(bar(kBarV + s), 1);
-            tc::mbar_init(bar(kBarE + s), 1);
+            tc::mbar_init(bar(kBarEK + s), 1);
+            tc::mbar_init(bar(kBarEV + s), 1);
         }
         for (int t = 0; t < 2; ++t) {
             tc::mbar_init(bar(kBarS + t), 1);
@@ -197,27 +236,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tc::tma_load_2d(sQ + 2 * kRegion, &tmQ, bar(kBarQ), 0, qrow + kBM);
                 tc::tma_load_2d(sQ + 3 * kRegion, &tmQ, bar(kBarQ), 64, qrow + kBM);
             }
-            int j = 0;
-            for (; j < ntk; ++j) {
-                const int s = j % kStages;
-                if (j >= kStages && !tc::mbar_wait(bar(kBarE + s), ((j / kStages) - 1) & 1, abort_flag)) break;
-                const int krow = z * p.N + key_tile(p, MODE, klist, j).x;
-                const uint32_t dk = sK + s * 2 * kRegion, dv = sV + s * 2 * kRegion;
-                tc::mbar_arrive_expect_tx(bar(kBarK + s), 2 * kRegion);
-                tc::tma_load_2d(dk, &tmK, bar(kBarK + s), 0, krow);
-                tc::tma_load_2d(dk + kRegion, &tmK, bar(kBarK + s), 64, krow);
-                tc::mbar_arrive_expect_tx(bar(kBarV + s), 2 * kRegion);
-                tc::tma_load_2d(dv, &tmV, bar(kBarV + s), 0, krow);
-                tc::tma_load_2d(dv + kRegion, &tmV, bar(kBarV + s), 64, krow);
+            // K runs one tile ahead of V: K(0), then K(j+1) before V(j).
+            auto load = [&](int m, bool isv) -> bool {
+                const int s = m % kStages;
+                if (m >= kStages && !tc::mbar_wait(bar((isv ? kBarEV : kBarEK) + s), ((m / kStages) - 1) & 1, abort_flag))
+                    return false;
+                const int krow = z * p.N + key_tile(p, MODE, klist, m).x;
+                const uint32_t d = (isv ? sV : sK) + s * 2 * kRegion;
+                const uint32_t b = bar((isv ? kBarV : kBarK) + s);
+                tc::mbar_arrive_expect_tx(b, 2 * kRegion);
+                tc::tma_load_2d(d, isv ? &tmV : &tmK, b, 0, krow);
+                tc::tma_load_2d(d + kRegion, isv ? &tmV : &tmK, b, 64, krow);
+                return true;
+            };
+            int nk = 0, nv = 0;   // K and V tiles issued
+            if (ntk > 0 && load(0, false)) nk = 1;
+            for (int j = 0; nk > j && j < ntk; ++j) {
+                if (j + 1 < ntk) {
+                    if (!load(j + 1, false)) break;
+                    nk = j + 2;
+                }
+                if (!load(j, true)) break;
+                nv = j + 1;
             }
             // every issued load must land before the CTA can exit
             int never = 0;
-            for (int t = (j > kStages ? j - kStages : 0); t < j; ++t) {
-                const int s = t % kStages;
-                const uint32_t par = (t / kStages) & 1;
-                tc::mbar_wait(bar(kBarK + s), par, &never);
-                tc::mbar_wait(bar(kBarV + s), par, &never);
-            }
+            for (int m = (nk > kStages ? nk - kStages : 0); m < nk; ++m)
+                tc::mbar_wait(bar(kBarK + m % kStages), (m / kStages) & 1, &never);
+            for (int m = (nv > kStages ? nv - kStages : 0); m < nv; ++m)
+                tc::mbar_wait(bar(kBarV + m % kStages), (m / kStages) & 1, &never);
             tc::mbar_wait(bar(kBarQ), 0, &never);
         }
     } else if (warp == 9) {
@@ -243,8 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ok = __all_sync(kFull, tc::mbar_wait(bar(kBarK), 0, abort_flag));
             if (ok) {
                 tc::fence_after_sync();
-                if (lane == 0)
+                if (lane == 0) {
                     for (int t = 0; t < ntiles; ++t) issue_S(t, 0);
+                    tc::commit(bar(kBarEK));
+                }
                 __syncwarp();
             }
         }
@@ -266,14 +315,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
                                        tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
                                        (j > 0 || k > 0) ? 1u : 0u);
-                    if (nhave) issue_S(t, j + 1);
-                    else tc::commit(bar(kBarO + t));
+                    const bool last = t + 1 == ntiles;
+                    if (last) tc::commit(bar(kBarEV + s));                  // V(j) read by every PV
+                    if (nhave) {
+                        issue_S(t, j + 1);
+                        if (last) tc::commit(bar(kBarEK + (j + 1) % kStages));   // K(j+1) read by every S
+                    } else {
+                        tc::commit(bar(kBarO + t));
+                    }
                 }
                 __syncwarp();
             }
             if (!ok) break;
-            if (lane == 0) tc::commit(bar(kBarE + s));
-            __syncwarp();
             have = nhave;
             ++j;
         }
@@ -310,9 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // in TMEM until P is written.
                 const float thr = (m_run + kRescaleLog2) / c_log2;      // raw-logit threshold
                 uint32_t pk0[32];                                       // P of columns 0..63
-                float ps[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+                uint64_t ps[4] = {0ull, 0ull, 0ull, 0ull};              // packed pair sums
                 bool slow = false;
                 float mx0 = -INFINITY, mx1 = -INFINITY;
                 {
@@ -358,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                     if (rescale) m_run = m_new;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+                    for (int e = 0; e < 4; ++e) ps[e] = 0ull;
                     uint32_t pk1[32];
                     {
                         uint32_t sv[2][32];
@@ -380,7 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tc::tmem_st16(tS + 32, pk1);
                     tc::tmem_st16(tS + 48, pk1 + 16);
                 }
-                l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                {
+                    float a0, a1, b0, b1;
+                    up2(add2(ps[0], ps[1]), a0, a1);
+                    up2(add2(ps[2], ps[3]), b0, b1);
+                    l_run += (a0 + a1) + (b0 + b1);
+                }
                 tc::tmem_wait_st();
                 tc::fence_before_sync();
                 tc::mbar_arrive(bar(kBarP + t));
