@@ -19,6 +19,7 @@ FLAG_HARD_DROP_ONLY = 1 << 0
 FLAG_RIDGE_ONLY = 1 << 1
 FLAG_RBAR_UNPROJECTED = 1 << 2
 FLAG_UNIFORM_WEIGHTS = 1 << 3
+FLAG_TOPMASS = 1 << 4
 FLAG_STAGE_TIMING = 1 << 8
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace allocation failed",
@@ -37,7 +38,7 @@ class Config(ctypes.Structure):
 
 class Partition(ctypes.Structure):
     _fields_ = [(n, _p) for n in ("kgroup", "qgroup", "kperm", "koff", "qperm", "qoff", "kcent", "radial",
-                                  "probe", "probe_pos", "weights", "features")]
+                                  "probe", "probe_pos", "weights", "features", "topmass")]
 
 
 class Route(ctypes.Structure):
@@ -299,6 +300,8 @@ class SparsePR:
         if part.features:
             DP = (c.rK + 15) // 16 * 16
             v["features"] = device_view(part.features, (P, N, DP), torch.float32)
+        if part.topmass:
+            v["topmass"] = device_view(part.topmass, (P, c.rK), torch.float32)
         if M:
             v["probe"] = device_view(part.probe, (P, M), torch.int32)
             v["probe_pos"] = device_view(part.probe_pos, (P, M), torch.int32)
@@ -350,5 +353,5 @@ def route_from_tensors(t: dict) -> Route:
 
 __all__ = ["SparsePR", "SparsePRError", "Config", "Partition", "Route", "Fit", "Stats", "load_library",
            "header_functions", "partition_from_tensors", "route_from_tensors", "device_view", "LIB_PATH",
-           "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS",
+           "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS", "FLAG_TOPMASS",
            "FLAG_STAGE_TIMING"]

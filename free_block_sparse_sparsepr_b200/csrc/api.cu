@@ -20,7 +20,7 @@ constexpr int kMaxGroups = 1024;
 constexpr int kProbeSplits = 32;
 constexpr int kSortChunk = 2048;   // rows per counting-sort chunk (matches the sort kernels)
 constexpr unsigned kSupportedFlags =
-    SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_STAGE_TIMING;
+    SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING;
 
 inline int pad16(int v) { return (v + 15) / 16 * 16; }
 inline int pad64(int v) { return (v + 63) / 64 * 64; }
@@ -39,6 +39,7 @@ struct sparsepr_handle_s {
     // partition
     int32_t *kgroup = nullptr, *qgroup = nullptr, *kperm = nullptr, *koff = nullptr, *qperm = nullptr,
             *qoff = nullptr, *probe = nullptr, *probe_pos = nullptr, *probe_seq = nullptr;
+    float* topmass = nullptr;
     float *kcent = nullptr, *radial = nullptr, *weights = nullptr, *features = nullptr, *ycoord = nullptr,
           *kdist = nullptr, *kmC = nullptr;
     int *counts = nullptr, *bases = nullptr, *km_changed = nullptr, *km_done = nullptr;
@@ -214,6 +215,7 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     a.M = N; a.N = h->DPk; a.K = d; a.batch = P;
     a.alpha = (float)(1.0 / sqrt((double)d));
     SPR_TRY(spr::launch_gemm_bf16(a, s));
+    if (c.flags & SPARSEPR_FLAG_TOPMASS) SPR_TRY(spr::launch_topmass(h->features, h->topmass, P, N, h->DPk, c.rK, s));
     // (2a) key groups and their means in the original key space
     sparsepr_status st = kmeans(h, h->features, h->DPk, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s);
     if (st) return st;
@@ -248,6 +250,7 @@ void fill_partition(sparsepr_handle h, sparsepr_partition_t* p) {
     p->kgroup = h->kgroup; p->qgroup = h->qgroup; p->kperm = h->kperm; p->koff = h->koff;
     p->qperm = h->qperm; p->qoff = h->qoff; p->kcent = h->kcent; p->radial = h->radial;
     p->probe = h->probe; p->probe_pos = h->probe_pos; p->weights = h->weights; p->features = h->features;
+    p->topmass = (h->cfg.flags & SPARSEPR_FLAG_TOPMASS) ? h->topmass : nullptr;
 }
 
 void fill_route(sparsepr_handle h, sparsepr_route_t* r) {
@@ -388,7 +391,7 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     } while (0)
     A_(kgroup, P * N); A_(qgroup, P * N); A_(kperm, P * N); A_(koff, P * (Gk + 1));
     A_(qperm, P * N); A_(qoff, P * (Gq + 1)); A_(probe, P * M); A_(probe_pos, P * M); A_(probe_seq, P * M);
-    A_(kcent, P * Gk * d); A_(radial, P * N); A_(weights, P * M); A_(features, P * N * h->DPk);
+    A_(kcent, P * Gk * d); A_(radial, P * N); A_(weights, P * M); A_(features, P * N * h->DPk); A_(topmass, P * c.rK);
     A_(ycoord, P * N * h->DPy); A_(kdist, P * N); A_(kmC, P * h->Gmax * 64);
     A_(counts, P * h->nch * h->Gmax); A_(bases, P * h->nch * h->Gmax); A_(km_changed, P); A_(km_done, P);
     A_(Qs, P * h->DPk * d); A_(chi, P * Gk * d); A_(clo, P * Gk * d);

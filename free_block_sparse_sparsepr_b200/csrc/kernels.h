@@ -68,6 +68,10 @@ cudaError_t launch_logits_tc(const bf16* Q, const bf16* chi, const bf16* clo, co
 // Split fp32 group means into bf16 hi/lo (used when the partition is handed in).
 cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long count, cudaStream_t s);
 
+// Support diagnostic: out[z][s] = (smallest k whose k largest exp(F[.][s] - max) hold 90% of the
+// row's softmax mass) / N, for s < S; F [P][N][DP] fp32 (DP a multiple of 8, S <= DP).
+cudaError_t launch_topmass(const float* F, float* out, int P, int N, int DP, int S, cudaStream_t s);
+
 // ---------------------------------------------------------------- responses and coordinates
 // Qs[z][s][:] = Q[b][h*g + s%g][floor((s+1/2)N/S)][:] for s < S, zero rows up to DP.
 cudaError_t launch_gather_samples(const bf16* Q, bf16* Qs, int B, int Hq, int Hkv, int N, int d,

@@ -1,0 +1,266 @@
+// Support diagnostic of the sampled query rows ([support]): for each sampled row s, the
+// fraction of keys that carries 90% of its softmax mass, i.e. the smallest k such that the k
+// largest p_j = exp(z_sj - max_j z_sj) sum to at least 0.9 sum_j p_j, divided by N. The
+// responses z_sj are the key features F[j][s] written by the response GEMM.
+//
+// One CTA per (KV head, 8 sampled rows); every pass streams the head's F rows once (8
+// contiguous floats per row). Pass 1: per-row maximum. Pass 2: total mass, and mass and count
+// per bin of delta = max - z (256 bins of 1/8 nat; the last one open-ended). The bin where the
+// cumulative mass from the top crosses 90% is then narrowed (256 sub-bins per level) until it
+// holds at most kCap keys; those are sorted exactly (bitonic, in shared memory) and walked in
+// order to the crossing.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spr {
+namespace {
+
+constexpr int kCols = 8;
+constexpr int kThreads = 512;
+constexpr int kBins = 256;
+constexpr int kCap = 4096;
+constexpr int kMaxLevels = 4;
+constexpr float kMass = 0.9f;
+
+struct Smem {
+    float hmass[kCols][kBins];
+    int hcnt[kCols][kBins];
+    float red[kThreads / 32][kCols];
+    float mx[kCols], total[kCols], lo[kCols], width[kCols], mass0[kCols];
+    int count0[kCols], settled[kCols], nval[kCols], result[kCols];
+    unsigned open[kCols];                // 1 if the current range has no upper end (level 0's last bin)
+    float vals[kCols][kCap];
+};
+
+__device__ __forceinline__ void load_row(const float* Fz, long long j, int DP, int c0, float (&v)[kCols]) {
+    const float4* p = reinterpret_cast<const float4*>(Fz + j * DP + c0);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__global__ void __launch_bounds__(kThreads) topmass_kernel(const float* __restrict__ F, float* out, int N, int DP,
+                                                           int S) {
+    extern __shared__ unsigned char sm_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>(sm_raw);
+    const int z = blockIdx.y, c0 = blockIdx.x * kCols;
+    const int ncol = min(kCols, S - c0);
+    const float* Fz = F + (long long)z * N * DP;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- pass 1: maxima
+    float v[kCols], acc[kCols];
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) acc[c] = -INFINITY;
+    for (long long j = tid; j < N; j += kThreads) {
+        load_row(Fz, j, DP, c0, v);
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) acc[c] = fmaxf(acc[c], v[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) {
+        const float r = warp_max(acc[c]);
+        if (lane == 0) sm.red[warp][c] = r;
+    }
+    __syncthreads();
+    if (tid < kCols) {
+        float r = -INFINITY;
+        for (int w = 0; w < kThreads / 32; ++w) r = fmaxf(r, sm.red[w][tid]);
+        sm.mx[tid] = r;
+        sm.lo[tid] = 0.f;
+        sm.width[tid] = 0.125f;
+        sm.open[tid] = 1u;
+        sm.mass0[tid] = 0.f;
+        sm.count0[tid] = 0;
+        sm.settled[tid] = tid < ncol ? 0 : 1;
+    }
+    __syncthreads();
+    float m[kCols];
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) m[c] = sm.mx[c];
+
+    // ---- histogram levels: level 0 also yields the total mass
+    for (int level = 0; level < kMaxLevels; ++level) {
+        for (int t = tid; t < kCols * kBins; t += kThreads) {
+            (&sm.hmass[0][0])[t] = 0.f;
+            (&sm.hcnt[0][0])[t] = 0;
+        }
+        __syncthreads();
+        float lo[kCols], inv_w[kCols];
+        bool act[kCols], open[kCols];
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) {
+            lo[c] = sm.lo[c];
+            inv_w[c] = 1.f / sm.width[c];
+            act[c] = !sm.settled[c];
+            open[c] = sm.open[c] != 0u;
+            acc[c] = 0.f;
+        }
+        for (long long j = tid; j < N; j += kThreads) {
+            load_row(Fz, j, DP, c0, v);
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) {
+                if (!act[c]) continue;
+                const float d = m[c] - v[c];
+                const float p = expf(v[c] - m[c]);
+                if (level == 0) acc[c] += p;
+                const float b = (d - lo[c]) * inv_w[c];
+                if (b >= 0.f && (b < (float)kBins || open[c])) {
+                    const int bi = min(kBins - 1, (int)b);
+                    atomicAdd(&sm.hmass[c][bi], p);
+                    atomicAdd(&sm.hcnt[c][bi], 1);
+                }
+            }
+        }
+        if (level == 0) {
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) {
+                const float r = warp_sum(acc[c]);
+                if (lane == 0) sm.red[warp][c] = r;
+            }
+        }
+        __syncthreads();
+        // one warp per column: find the bin where the cumulative mass crosses the target
+        if (warp < kCols && !sm.settled[warp]) {
+            const int c = warp;
+            if (level == 0 && lane == 0) {
+                float r = 0.f;
+                for (int w = 0; w < kThreads / 32; ++w) r += sm.red[w][c];
+                sm.total[c] = r;
+            }
+            __syncwarp();
+            const float target = kMass * sm.total[c];
+            float base = sm.mass0[c];
+            int cbase = sm.count0[c];
+            int hit = -1;
+            for (int b0 = 0; b0 < kBins && hit < 0; b0 += 32) {
+                const float bm = sm.hmass[c][b0 + lane];
+                const int bc = sm.hcnt[c][b0 + lane];
+                float inc = bm;
+                int cinc = bc;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float tv = __shfl_up_sync(kFull, inc, o);
+                    const int tc = __shfl_up_sync(kFull, cinc, o);
+                    if (lane >= o) { inc += tv; cinc += tc; }
+                }
+                const unsigned crossed = __ballot_sync(kFull, base + inc >= target);
+                if (crossed) {
+                    const int l = __ffs(crossed) - 1;
+                    hit = b0 + l;
+                    const float before = __shfl_sync(kFull, inc - bm, l);
+                    const int cbefore = __shfl_sync(kFull, cinc - bc, l);
+                    base += before;
+                    cbase += cbefore;
+                } else {
+                    base += __shfl_sync(kFull, inc, 31);
+                    cbase += __shfl_sync(kFull, cinc, 31);
+                }
+            }
+            if (lane == 0) {
+                if (hit < 0) {
+                    // rounding left the target unreached: every key counts
+                    sm.result[c] = N;
+                    sm.settled[c] = 2;
+                } else {
+                    sm.mass0[c] = base;
+                    sm.count0[c] = cbase;
+                    const bool last_open = sm.open[c] && hit == kBins - 1;
+                    sm.lo[c] = sm.lo[c] + (float)hit * sm.width[c];
+                    sm.open[c] = last_open ? 1u : 0u;
+                    if (!last_open) sm.width[c] = sm.width[c] / (float)kBins;
+                    sm.nval[c] = sm.hcnt[c][hit];
+                    if (sm.hcnt[c][hit] <= kCap || level + 1 == kMaxLevels) sm.settled[c] = 3;  // gather next
+                }
+            }
+        }
+        __syncthreads();
+        bool more = false;
+        for (int c = 0; c < kCols; ++c) more |= sm.settled[c] == 0;
+        if (!more) break;
+    }
+
+    // ---- gather the crossing bin's keys and settle each column exactly
+    if (tid < kCols) sm.nval[tid] = 0;
+    __syncthreads();
+    {
+        float lo[kCols], hi[kCols];
+        bool act[kCols];
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) {
+            act[c] = sm.settled[c] == 3;
+            lo[c] = sm.lo[c];
+            // the open range of level 0's last bin has no upper end; a narrowed bin is
+            // [lo, lo + width * kBins) in the units it was found with
+            hi[c] = sm.open[c] ? INFINITY : sm.lo[c] + sm.width[c] * (float)kBins;
+        }
+        for (long long j = tid; j < N; j += kThreads) {
+            load_row(Fz, j, DP, c0, v);
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) {
+                if (!act[c]) continue;
+                const float d = m[c] - v[c];
+                if (d >= lo[c] && d < hi[c]) {
+                    const int at = atomicAdd(&sm.nval[c], 1);
+                    if (at < kCap) sm.vals[c][at] = d;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int c = 0; c < kCols; ++c) {
+        if (sm.settled[c] != 3) continue;
+        const int n = min(sm.nval[c], kCap);
+        int len = 1;
+        while (len < n) len <<= 1;
+        for (int t = n + tid; t < len; t += kThreads) sm.vals[c][t] = INFINITY;
+        __syncthreads();
+        // bitonic sort, ascending delta (descending p)
+        for (int k = 2; k <= len; k <<= 1)
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                for (int t = tid; t < len; t += kThreads) {
+                    const int u = t ^ jj;
+                    if (u > t) {
+                        const float a = sm.vals[c][t], b = sm.vals[c][u];
+                        const bool up = (t & k) == 0;
+                        if ((a > b) == up) { sm.vals[c][t] = b; sm.vals[c][u] = a; }
+                    }
+                }
+                __syncthreads();
+            }
+        if (warp == 0) {
+            const float target = kMass * sm.total[c];
+            float base = sm.mass0[c];
+            int idx = -1;
+            for (int b0 = 0; b0 < n && idx < 0; b0 += 32) {
+                const int t = b0 + lane;
+                float inc = t < n ? expf(-sm.vals[c][t]) : 0.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float tv = __shfl_up_sync(kFull, inc, o);
+                    if (lane >= o) inc += tv;
+                }
+                const unsigned crossed = __ballot_sync(kFull, t < n && base + inc >= target);
+                if (crossed) idx = b0 + __ffs(crossed) - 1;
+                else base += __shfl_sync(kFull, inc, 31);
+            }
+            if (lane == 0) sm.result[c] = sm.count0[c] + (idx >= 0 ? idx + 1 : n);
+        }
+        __syncthreads();
+    }
+    if (tid < ncol) out[(long long)z * S + c0 + tid] = (float)min(sm.result[tid], N) / (float)N;
+}
+
+}  // namespace
+
+cudaError_t launch_topmass(const float* F, float* out, int P, int N, int DP, int S, cudaStream_t s) {
+    if (DP % kCols != 0 || S > DP) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(Smem);
+    cudaError_t e = cudaFuncSetAttribute(topmass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topmass_kernel<<<dim3((S + kCols - 1) / kCols, P), kThreads, smem, s>>>(F, out, N, DP, S);
+    return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -59,6 +59,7 @@ typedef enum sparsepr_status {
 #define SPARSEPR_FLAG_RIDGE_ONLY        (1u << 1)  /* ridge correction without subspace projection */
 #define SPARSEPR_FLAG_RBAR_UNPROJECTED  (1u << 2)  /* project only A(o - obar), add Rbar unprojected */
 #define SPARSEPR_FLAG_UNIFORM_WEIGHTS   (1u << 3)  /* probe weights 1 instead of group coverage */
+#define SPARSEPR_FLAG_TOPMASS           (1u << 4)  /* sparsepr_partition also writes the support diagnostic */
 #define SPARSEPR_FLAG_STAGE_TIMING      (1u << 8)  /* record per-stage CUDA events (sparsepr_get_stats) */
 
 /*
@@ -108,8 +109,12 @@ typedef struct sparsepr_handle_s* sparsepr_handle;
  *   probe_pos [P][M]     position of each probe row in qperm
  *   weights [P][M]       fp32 group-coverage weight of each probe (mean 1)
  *   features [P][N][rK]  fp32 key response features (written by sparsepr_partition; unused as input)
+ *   topmass [P][rK]      fp32 support diagnostic [support paragraph]: for sampled query row s, the
+ *                        fraction of keys whose largest softmax weights first reach 90% of the row's
+ *                        mass (written by sparsepr_partition with SPARSEPR_FLAG_TOPMASS, else NULL;
+ *                        unused as input)
  * When the struct is handed IN, only kgroup/qgroup are ignored; every other
- * field except `features` must be set.
+ * field except `features` and `topmass` must be set.
  */
 typedef struct sparsepr_partition_t {
     int32_t* kgroup;
@@ -124,6 +129,7 @@ typedef struct sparsepr_partition_t {
     int32_t* probe_pos;
     float* weights;
     float* features;
+    float* topmass;
 } sparsepr_partition_t;
 
 /*

@@ -283,3 +283,25 @@ def test_hard_drop_only_flag():
         torch.cuda.synchronize()
         st = h.stats()
         assert abs(st["rho_exec"] - st["route_density"]) < 1e-12
+
+
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000", "ragged_gqa_n1500_g40"])
+def test_support_diagnostic_matches_oracle(name):
+    """The 90%-mass support fraction of every sampled row ([support]) against the oracle's
+    full-sort definition applied to the same response row (the GPU's fp32 features): the key
+    count agrees to 2 keys (fp32 mass sums may move the crossing across near-equal weights);
+    against the oracle's own fp64 responses to 1e-3 of N."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    with spr.SparsePR.from_workload(w, flags=spr.FLAG_TOPMASS) as h:
+        part = h.partition(q, k)
+        torch.cuda.synchronize()
+        pv = {n: t.cpu().numpy() for n, t in h.partition_views(part).items()}
+    assert "topmass" in pv
+    for z in range(w.B * w.Hkv):
+        F = pv["features"][z][:, : w.rK].astype(np.float64)
+        k_gpu = np.rint(pv["topmass"][z] * w.N).astype(np.int64)
+        k_ref = np.array([round(oracle.top_mass_fraction(F[:, s]) * w.N) for s in range(w.rK)])
+        assert np.abs(k_gpu - k_ref).max() <= 2, (k_gpu, k_ref)
+        zo = res["partitions"][(z // w.Hkv, z % w.Hkv)].z
+        k_o = np.array([round(oracle.top_mass_fraction(zo[s]) * w.N) for s in range(w.rK)])
+        assert np.abs(k_gpu - k_o).max() <= max(2, 1e-3 * w.N), (k_gpu, k_o)
