@@ -91,37 +91,55 @@ __global__ void __launch_bounds__(kAssignRows) km_assign_kernel(const float* __r
     if ((threadIdx.x & 31) == 0 && b) atomicAdd(&changed[z], __popc(b));
 }
 
-// New centroid = mean of its members in fp64 (perm/off order, kUpdSlices fixed row slices summed
-// in a fixed order), stored fp32; an empty group keeps its centroid.
-constexpr int kUpdSlices = 8;
-__global__ void km_update_kernel(const float* __restrict__ X, const int32_t* __restrict__ perm,
-                                 const int32_t* __restrict__ off, float* C, const int* done, int n,
-                                 int G, int DP) {
+// New centroid = mean of its members in fp64, stored fp32; an empty group keeps its centroid.
+// One block per group: thread t reads feature quad t % (DP/4) (a float4) of the rows at
+// positions lo + slice, lo + slice + nslices, ... of the group (perm order), four rows in flight;
+// the slices are then summed in a fixed order, so the result does not depend on scheduling.
+constexpr int kUpdThreads = 256;
+template <int DP>
+__global__ void __launch_bounds__(kUpdThreads) km_update_kernel(const float* __restrict__ X,
+                                                                const int32_t* __restrict__ perm,
+                                                                const int32_t* __restrict__ off, float* C,
+                                                                const int* done, int n, int G) {
+    constexpr int kQ = DP / 4;                       // float4 quads per row
+    constexpr int kSl = kUpdThreads / kQ;            // row slices
     const int z = blockIdx.y, g = blockIdx.x;
     if (done && done[z]) return;
     const int lo = off[(long long)z * (G + 1) + g], hi = off[(long long)z * (G + 1) + g + 1];
     if (hi <= lo) return;
-    const int c = threadIdx.x % DP, rs = threadIdx.x / DP;
-    const int32_t* pz = perm + (long long)z * n;
-    const float* xz = X + (long long)z * n * DP + c;
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-    int j = lo + rs;
-    for (; j + 3 * kUpdSlices < hi; j += 4 * kUpdSlices) {
-        const int r0 = __ldg(pz + j), r1 = __ldg(pz + j + kUpdSlices);
-        const int r2 = __ldg(pz + j + 2 * kUpdSlices), r3 = __ldg(pz + j + 3 * kUpdSlices);
-        const float v0 = __ldg(xz + (long long)r0 * DP), v1 = __ldg(xz + (long long)r1 * DP);
-        const float v2 = __ldg(xz + (long long)r2 * DP), v3 = __ldg(xz + (long long)r3 * DP);
-        a0 += (double)v0; a1 += (double)v1; a2 += (double)v2; a3 += (double)v3;
-    }
-    for (; j < hi; j += kUpdSlices) a0 += (double)__ldg(xz + (long long)__ldg(pz + j) * DP);
-    __shared__ double red[kUpdSlices][64];
-    red[rs][c] = (a0 + a1) + (a2 + a3);
-    __syncthreads();
-    if (rs == 0) {
-        double t = 0.0;
+    const int q = threadIdx.x % kQ, rs = threadIdx.x / kQ;
+    __shared__ double red[kSl][DP];
+    if (rs < kSl) {
+        const int32_t* pz = perm + (long long)z * n;
+        const float4* xz = reinterpret_cast<const float4*>(X + (long long)z * n * DP) + q;
+        double a[4][4] = {};
+        int j = lo + rs;
+        for (; j + 3 * kSl < hi; j += 4 * kSl) {
+            int r[4];
 #pragma unroll
-        for (int k = 0; k < kUpdSlices; ++k) t += red[k][c];
-        C[((long long)z * G + g) * DP + c] = (float)(t / (double)(hi - lo));
+            for (int u = 0; u < 4; ++u) r[u] = __ldg(pz + j + u * kSl);
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = __ldg(xz + (long long)r[u] * kQ);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                a[u][0] += (double)v[u].x; a[u][1] += (double)v[u].y;
+                a[u][2] += (double)v[u].z; a[u][3] += (double)v[u].w;
+            }
+        }
+        for (; j < hi; j += kSl) {
+            const float4 v = __ldg(xz + (long long)__ldg(pz + j) * kQ);
+            a[0][0] += (double)v.x; a[0][1] += (double)v.y; a[0][2] += (double)v.z; a[0][3] += (double)v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) red[rs][4 * q + e] = (a[0][e] + a[1][e]) + (a[2][e] + a[3][e]);
+    }
+    __syncthreads();
+    if (threadIdx.x < DP) {
+        double t = 0.0;
+#pragma unroll 4
+        for (int k = 0; k < kSl; ++k) t += red[k][threadIdx.x];
+        C[((long long)z * G + g) * DP + threadIdx.x] = (float)(t / (double)(hi - lo));
     }
 }
 
@@ -274,7 +292,14 @@ cudaError_t launch_km_assign(const float* X, const float* C, int32_t* labels, fl
 
 cudaError_t launch_km_update(const float* X, const int32_t* perm, const int32_t* off, float* C,
                              const int* done, int P, int n, int G, int DP, cudaStream_t s) {
-    km_update_kernel<<<dim3(G, P), kUpdSlices * DP, 0, s>>>(X, perm, off, C, done, n, G, DP);
+    const dim3 grid(G, P);
+    switch (DP) {
+        case 16: km_update_kernel<16><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
+        case 32: km_update_kernel<32><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
+        case 48: km_update_kernel<48><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
+        case 64: km_update_kernel<64><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
+        default: return cudaErrorInvalidValue;
+    }
     return cudaGetLastError();
 }
 

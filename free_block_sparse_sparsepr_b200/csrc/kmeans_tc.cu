@@ -360,12 +360,13 @@ __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long
     if (lane == 0) cc[(long long)z * G32 + g] = g < G ? ss : kFar;
 }
 
-// Exact pass over the flagged rows: one block per assignment CTA (its centroids staged in shared
-// memory k-major), one warp per row, the row in registers. Candidates are the groups whose fp32
+// Exact pass over the flagged rows: kFixSplit blocks per assignment CTA (each with the
+// centroids staged in shared memory k-major), one warp per row, the row in registers. Candidates are the groups whose fp32
 // ||x||^2 - 2 x.c + ||c||^2 (error below 2^-19 (||x||^2 + ||c||^2)) is within 1e-4 (d + ||x||^2
 // + max ||c||^2) of the smallest; each gets the fp32 value of its fp64 distance, argmin with ties
 // to the lowest group. Corrects the label and the count of rows that moved.
 constexpr int kFixThreads = 512;
+constexpr int kFixSplit = 4;   // blocks per assignment CTA's region
 template <int DP>
 __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __restrict__ fix,
                                                                const int* __restrict__ fix_count,
@@ -389,7 +390,8 @@ __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __res
     for (int g = 0; g < G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
     const int4* reg = fix + (long long)cta * fix_cap;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int w = warp; w < cnt; w += kFixThreads / 32) {
+    // blockIdx.z of gridDim.z blocks share the region, each warp taking every (warps * blocks)th row
+    for (int w = blockIdx.z * (kFixThreads / 32) + warp; w < cnt; w += gridDim.z * (kFixThreads / 32)) {
         const int4 h = reg[w];
         const long long o = h.x;
         const float* xr = X + o * DP;
@@ -532,7 +534,7 @@ cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* 
     km_grid(P, n, num_sms, &per, &cap);
     const int G32 = (G + 31) / 32 * 32;
     const size_t smem = ((size_t)DP * kMaxG + kMaxG) * sizeof(float);
-    const dim3 grid(per, P);
+    const dim3 grid(per, P, kFixSplit);
 #define SPR_FIXUP(DPV)                                                                                               \
     case DPV: {                                                                                                      \
         cudaError_t e = cudaFuncSetAttribute(km_fixup_kernel<DPV>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
