@@ -20,7 +20,8 @@ constexpr int kMaxGroups = 1024;
 constexpr int kProbeSplits = 32;
 constexpr int kSortChunk = 2048;   // rows per counting-sort chunk (matches the sort kernels)
 constexpr unsigned kSupportedFlags =
-    SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING;
+    SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED |
+    SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING;
 
 inline int pad16(int v) { return (v + 15) / 16 * 16; }
 inline int pad64(int v) { return (v + 63) / 64 * 64; }
@@ -119,9 +120,8 @@ sparsepr_status validate(const sparsepr_config* c) {
     if (c->kmeans_iters < 0 || c->kmeans_iters > 64) return SPARSEPR_ERR_INVALID_ARG;
     if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return SPARSEPR_ERR_INVALID_ARG;
     if (!(c->rho_exec > 0.f) || !isfinite(c->rho_exec)) return SPARSEPR_ERR_INVALID_ARG;
-    if (c->flags & ~(kSupportedFlags | SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED))
+    if (c->flags & ~kSupportedFlags)
         return SPARSEPR_ERR_INVALID_ARG;
-    if (c->flags & (SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED)) return SPARSEPR_ERR_UNSUPPORTED;
     if (!(c->flags & SPARSEPR_FLAG_HARD_DROP_ONLY)) {
         if (c->M < 1 || c->M > c->N) return SPARSEPR_ERR_INVALID_ARG;
         if (c->M > 64) return SPARSEPR_ERR_UNSUPPORTED;
@@ -321,18 +321,25 @@ sparsepr_status probe_fit_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     SPR_TRY(spr::launch_probe_residual(h->Odense, Osp, p->probe_pos, h->R, h->Xprobe, h->Hp, h->g, c.N, c.d,
                                        h->M, s));
     SPR_TRY(spr::launch_fit(h->R, h->Xprobe, p->weights, c.lambda, h->obar, h->Rbar, h->A, h->U, h->Bm, h->c0,
-                            h->rank, h->Hp, h->g, c.d, h->M, c.r, h->dev_status, s));
+                            h->rank, h->Hp, h->g, c.d, h->M, c.r, (c.flags & SPARSEPR_FLAG_RBAR_UNPROJECTED) != 0,
+                            h->dev_status, s));
     return SPARSEPR_OK;
 }
 
 sparsepr_status writeback_impl(sparsepr_handle h, const sparsepr_partition_t* p, const bf16* Osp,
-                               const float* U, const float* Bm, const float* c0, const float* Odense, bf16* O,
-                               cudaStream_t s) {
+                               const sparsepr_fit_t* f, bf16* O, cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
     const bool correct = h->M > 0;
-    SPR_TRY(spr::launch_writeback(Osp, p->qperm, U, Bm, c0, O, h->Hp, h->g, c.N, c.d, correct ? c.r : 1,
-                                  correct, s));
-    if (correct) SPR_TRY(spr::launch_probe_override(Odense, p->probe, O, h->Hp, h->g, c.N, c.d, h->M, s));
+    if (correct && (c.flags & SPARSEPR_FLAG_RIDGE_ONLY)) {
+        SPR_TRY(spr::launch_writeback_ridge(Osp, p->qperm, f->A, f->obar, f->Rbar, O, h->Hp, h->g, c.N, c.d,
+                                            h->num_sms, s));
+    } else {
+        const float* radd = (correct && (c.flags & SPARSEPR_FLAG_RBAR_UNPROJECTED)) ? f->Rbar : nullptr;
+        SPR_TRY(spr::launch_writeback(Osp, p->qperm, correct ? f->U : nullptr, correct ? f->Bm : nullptr,
+                                      correct ? f->c0 : nullptr, radd, O, h->Hp, h->g, c.N, c.d, correct ? c.r : 1,
+                                      correct, s));
+    }
+    if (correct) SPR_TRY(spr::launch_probe_override(f->Odense, p->probe, O, h->Hp, h->g, c.N, c.d, h->M, s));
     return SPARSEPR_OK;
 }
 
@@ -523,10 +530,11 @@ sparsepr_status sparsepr_writeback(sparsepr_handle h, const sparsepr_partition_t
     sparsepr_status st = check_partition(part, h->M > 0);
     if (st) return st;
     if (h->M && (!fit || !fit->U || !fit->Bm || !fit->c0 || !fit->Odense)) return SPARSEPR_ERR_INVALID_ARG;
+    if (h->M && (h->cfg.flags & (SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED)) &&
+        (!fit->A || !fit->obar || !fit->Rbar))
+        return SPARSEPR_ERR_INVALID_ARG;
     h->launches = 0;
-    return writeback_impl(h, part, static_cast<const bf16*>(Osp), fit ? fit->U : nullptr, fit ? fit->Bm : nullptr,
-                          fit ? fit->c0 : nullptr, fit ? fit->Odense : nullptr, static_cast<bf16*>(O),
-                          as_stream(stream));
+    return writeback_impl(h, part, static_cast<const bf16*>(Osp), fit, static_cast<bf16*>(O), as_stream(stream));
 }
 
 sparsepr_status sparsepr_attention(sparsepr_handle h, const void* Q, const void* K, const void* V, void* O,
@@ -553,7 +561,9 @@ sparsepr_status sparsepr_attention(sparsepr_handle h, const void* Q, const void*
     mark(h, 4, s);
     if ((st = probe_fit_impl(h, q, k, v, &part, h->Osp, s))) return st;
     mark(h, 5, s);
-    if ((st = writeback_impl(h, &part, h->Osp, h->U, h->Bm, h->c0, h->Odense, static_cast<bf16*>(O), s)))
+    sparsepr_fit_t fit;
+    fill_fit(h, &fit);
+    if ((st = writeback_impl(h, &part, h->Osp, &fit, static_cast<bf16*>(O), s)))
         return st;
     mark(h, 6, s);
     cudaEventRecord(h->done_ev, s);

@@ -36,7 +36,7 @@ constexpr int kFitWarps = kFitThreads / 32;
 __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     const float* __restrict__ Rg, const float* __restrict__ Xg, const float* __restrict__ wts,
     float lambda, float* obar, float* Rbar, float* A, float* U, float* Bm, float* c0,
-    int32_t* rank_out, int g, int d, int M, int r, int* status) {
+    int32_t* rank_out, int g, int d, int M, int r, int rbar_unprojected, int* status) {
     const int x = blockIdx.x, z = x / g, tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int Mp = (M + 1) & ~1;
@@ -237,7 +237,8 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
         }
         a1 = warp_sum(a1);
         a2 = warp_sum(a2);
-        if (lane == 0) c0[(long long)x * r + k] = a1 - a2;
+        // c0 = U^T Rbar - Bm obar; with Rbar added unprojected only the -Bm obar part
+        if (lane == 0) c0[(long long)x * r + k] = (rbar_unprojected ? 0.f : a1) - a2;
     }
     for (int c = tid; c < d; c += nt) {
         obar[(long long)x * d + c] = xb[c];
@@ -246,7 +247,8 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     if (tid == 0) rank_out[x] = rank;
 }
 
-// O[qperm[p]] = Osp[p] + U (c0 + Bm Osp[p]); one warp per group-major row. Each lane holds
+// O[qperm[p]] = Osp[p] + U (c0 + Bm Osp[p]) (+ Radd, when given: the residual mean added
+// unprojected); one warp per group-major row. Each lane holds
 // EPL consecutive elements; Bm and U^T are staged row-major in shared memory so every
 // vector load is conflict-free. The RP partial dot products are reduced by recursive
 // halving (RP/2 + ... + 1 + 1 shuffles); afterwards lane 2k holds t_k.
@@ -255,7 +257,8 @@ __global__ void __launch_bounds__(256) writeback_kernel(const bf16* __restrict__
                                                         const int32_t* __restrict__ qperm,
                                                         const float* __restrict__ U,
                                                         const float* __restrict__ Bm,
-                                                        const float* __restrict__ c0, bf16* O,
+                                                        const float* __restrict__ c0,
+                                                        const float* __restrict__ Radd, bf16* O,
                                                         int g, int N, int r, int correct) {
     constexpr int EPL = D / 32;
     static_assert(RP == 16 || RP == 32, "RP");
@@ -273,6 +276,9 @@ __global__ void __launch_bounds__(256) writeback_kernel(const bf16* __restrict__
         for (int t = threadIdx.x; t < RP; t += blockDim.x) sc[t] = t < r ? c0[(long long)x * r + t] : 0.f;
     }
     __syncthreads();
+    float radd[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) radd[e] = (correct && Radd) ? Radd[(long long)x * D + lane * EPL + e] : 0.f;
     const int32_t* perm = qperm + (long long)z * N;
     for (int p = blockIdx.x * 8 + warp; p < N; p += gridDim.x * 8) {
         const bf16* src = Osp + ((long long)x * N + p) * D + lane * EPL;
@@ -316,7 +322,7 @@ __global__ void __launch_bounds__(256) writeback_kernel(const bf16* __restrict__
                 for (int e = 0; e < EPL; ++e) delta[e] = fmaf(sUt[k * D + lane * EPL + e], t, delta[e]);
             }
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[e] += delta[e];
+            for (int e = 0; e < EPL; ++e) o[e] += delta[e] + radd[e];
         }
         bf16* dst = O + ((long long)x * N + perm[p]) * D + lane * EPL;
 #pragma unroll
@@ -330,6 +336,59 @@ __global__ void probe_override_kernel(const float* __restrict__ Od, const int32_
     const int x = blockIdx.y, m = blockIdx.x, c = threadIdx.x, z = x / g;
     const int row = probe[(long long)z * M + m];
     O[((long long)x * N + row) * d + c] = __float2bfloat16_rn(Od[((long long)x * M + m) * d + c]);
+}
+
+// Ridge correction without the subspace projection: O[qperm[p]] = o + Rbar + A (o - obar),
+// o = Osp[p]. A (d x d, row stride d + 1) and c = Rbar - A obar in shared memory; one warp per
+// group-major row, lane l computing outputs l, l + 32, ... (conflict-free A reads), the row
+// itself broadcast from a per-warp buffer.
+template <int D>
+__global__ void __launch_bounds__(256) writeback_ridge_kernel(const bf16* __restrict__ Osp,
+                                                              const int32_t* __restrict__ qperm,
+                                                              const float* __restrict__ A,
+                                                              const float* __restrict__ obar,
+                                                              const float* __restrict__ Rbar, bf16* O, int g,
+                                                              int N) {
+    constexpr int EPL = D / 32;
+    extern __shared__ float rsm[];
+    float* sA = rsm;                     // [D][D + 1]
+    float* sc = sA + D * (D + 1);        // [D]
+    float* so = sc + D;                  // [8 warps][D]
+    const int x = blockIdx.y, z = x / g;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float* Ax = A + (long long)x * D * D;
+    for (int t = threadIdx.x; t < D * D; t += blockDim.x) sA[(t / D) * (D + 1) + t % D] = Ax[t];
+    __syncthreads();
+    for (int j = threadIdx.x; j < D; j += blockDim.x) {
+        float acc = Rbar[(long long)x * D + j];
+        for (int c = 0; c < D; ++c) acc = fmaf(-sA[j * (D + 1) + c], obar[(long long)x * D + c], acc);
+        sc[j] = acc;
+    }
+    __syncthreads();
+    const int32_t* perm = qperm + (long long)z * N;
+    float* row = so + warp * D;
+    for (int p = blockIdx.x * 8 + warp; p < N; p += gridDim.x * 8) {
+        const bf16* src = Osp + ((long long)x * N + p) * D;
+        float o[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            o[e] = __bfloat162float(src[lane + 32 * e]);
+            row[lane + 32 * e] = o[e];
+        }
+        __syncwarp();
+        float acc[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = o[e] + sc[lane + 32 * e];
+        for (int c = 0; c < D; ++c) {
+            const float oc = row[c];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(sA[(lane + 32 * e) * (D + 1) + c], oc, acc[e]);
+        }
+        __syncwarp();
+        bf16* dst = O + ((long long)x * N + perm[p]) * D;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) dst[lane + 32 * e] = __float2bfloat16_rn(acc[e]);
+    }
 }
 
 }  // namespace
@@ -350,29 +409,53 @@ cudaError_t launch_probe_residual(const float* Odense, const bf16* Osp, const in
 
 cudaError_t launch_fit(const float* R, const float* Xp, const float* w, float lambda, float* obar,
                        float* Rbar, float* A, float* U, float* Bm, float* c0, int32_t* rank,
-                       int Hp, int g, int d, int M, int r, int* status, cudaStream_t s) {
+                       int Hp, int g, int d, int M, int r, bool rbar_unprojected, int* status, cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
     const size_t smem = fit_smem_bytes(d, M, r);
     cudaError_t e = cudaFuncSetAttribute(fit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fit_kernel<<<Hp, kFitThreads, smem, s>>>(R, Xp, w, lambda, obar, Rbar, A, U, Bm, c0, rank, g, d, M, r, status);
+    fit_kernel<<<Hp, kFitThreads, smem, s>>>(R, Xp, w, lambda, obar, Rbar, A, U, Bm, c0, rank, g, d, M, r,
+                                             rbar_unprojected ? 1 : 0, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float* U,
-                             const float* Bm, const float* c0, bf16* O, int Hp, int g, int N,
+                             const float* Bm, const float* c0, const float* Radd, bf16* O, int Hp, int g, int N,
                              int d, int r, bool correct, cudaStream_t s) {
     const int blocks = (N + 8 * 16 - 1) / (8 * 16);   // 16 rows per warp
     dim3 grid(blocks, Hp);
     const int cf = correct ? 1 : 0;
     if (r <= 16) {
-        if (d == 64) writeback_kernel<64, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
-        else if (d == 128) writeback_kernel<128, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
+        if (d == 64) writeback_kernel<64, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
+        else if (d == 128) writeback_kernel<128, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
         else return cudaErrorInvalidValue;
     } else {
-        if (d == 64) writeback_kernel<64, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
-        else if (d == 128) writeback_kernel<128, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, O, g, N, r, cf);
+        if (d == 64) writeback_kernel<64, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
+        else if (d == 128) writeback_kernel<128, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
         else return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_writeback_ridge(const bf16* Osp, const int32_t* qperm, const float* A, const float* obar,
+                                   const float* Rbar, bf16* O, int Hp, int g, int N, int d, int num_sms,
+                                   cudaStream_t s) {
+    int per = (4 * num_sms + Hp - 1) / Hp;
+    const int maxb = (N + 8 * 16 - 1) / (8 * 16);
+    if (per > maxb) per = maxb;
+    const dim3 grid(per, Hp);
+    const size_t smem = ((size_t)d * (d + 1) + d + 8 * d) * sizeof(float);
+    cudaError_t e;
+    if (d == 64) {
+        e = cudaFuncSetAttribute(writeback_ridge_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        writeback_ridge_kernel<64><<<grid, 256, smem, s>>>(Osp, qperm, A, obar, Rbar, O, g, N);
+    } else if (d == 128) {
+        e = cudaFuncSetAttribute(writeback_ridge_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        writeback_ridge_kernel<128><<<grid, 256, smem, s>>>(Osp, qperm, A, obar, Rbar, O, g, N);
+    } else {
+        return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

@@ -145,10 +145,15 @@ cudaError_t launch_probe_residual(const float* Odense, const bf16* Osp, const in
                                   cudaStream_t s);
 cudaError_t launch_fit(const float* R, const float* Xp, const float* w, float lambda, float* obar,
                        float* Rbar, float* A, float* U, float* Bm, float* c0, int32_t* rank,
-                       int Hp, int g, int d, int M, int r, int* status, cudaStream_t s);
+                       int Hp, int g, int d, int M, int r, bool rbar_unprojected, int* status, cudaStream_t s);
+// O = Osp + U (c0 + Bm Osp) (+ Radd [Hp][d] when non-null), scattered to the original order.
 cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float* U,
-                             const float* Bm, const float* c0, bf16* O, int Hp, int g, int N,
+                             const float* Bm, const float* c0, const float* Radd, bf16* O, int Hp, int g, int N,
                              int d, int r, bool correct, cudaStream_t s);
+// O = Osp + Rbar + A (Osp - obar) (ridge correction without the projection).
+cudaError_t launch_writeback_ridge(const bf16* Osp, const int32_t* qperm, const float* A, const float* obar,
+                                   const float* Rbar, bf16* O, int Hp, int g, int N, int d, int num_sms,
+                                   cudaStream_t s);
 cudaError_t launch_probe_override(const float* Odense, const int32_t* probe, bf16* O, int Hp,
                                   int g, int N, int d, int M, cudaStream_t s);
 

@@ -56,8 +56,8 @@ typedef enum sparsepr_status {
 
 /* Ablation switches (sparsepr_config.flags); the page's ablations compare them. */
 #define SPARSEPR_FLAG_HARD_DROP_ONLY    (1u << 0)  /* no probes, no correction; whole budget to the route */
-#define SPARSEPR_FLAG_RIDGE_ONLY        (1u << 1)  /* ridge correction without subspace projection */
-#define SPARSEPR_FLAG_RBAR_UNPROJECTED  (1u << 2)  /* project only A(o - obar), add Rbar unprojected */
+#define SPARSEPR_FLAG_RIDGE_ONLY        (1u << 1)  /* ablation: ridge correction Rbar + A(o - obar), no projection */
+#define SPARSEPR_FLAG_RBAR_UNPROJECTED  (1u << 2)  /* ablation: project only A(o - obar), add Rbar unprojected */
 #define SPARSEPR_FLAG_UNIFORM_WEIGHTS   (1u << 3)  /* probe weights 1 instead of group coverage */
 #define SPARSEPR_FLAG_TOPMASS           (1u << 4)  /* sparsepr_partition also writes the support diagnostic */
 #define SPARSEPR_FLAG_STAGE_TIMING      (1u << 8)  /* record per-stage CUDA events (sparsepr_get_stats) */

@@ -45,7 +45,7 @@ def _cfg(**kw):
     (dict(Gk=0), 1), (dict(Gq=2000), 1), (dict(Gk=1025, N=4096), 2), (dict(rK=65), 1), (dict(rQ=0), 1),
     (dict(M=0), 1), (dict(M=65), 2), (dict(r=0), 1), (dict(r=65), 1), (dict(lam=0.0), 1),
     (dict(rho_exec=0.0), 1), (dict(rho_exec=float("nan")), 1), (dict(kmeans_iters=-1), 1),
-    (dict(flags=1 << 20), 1), (dict(flags=spr.FLAG_RIDGE_ONLY), 2),
+    (dict(flags=1 << 20), 1),
 ])
 def test_create_rejects_bad_configs_without_gpu(kw, code):
     lib = spr.load_library()

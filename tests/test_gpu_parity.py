@@ -305,3 +305,34 @@ def test_support_diagnostic_matches_oracle(name):
         zo = res["partitions"][(z // w.Hkv, z % w.Hkv)].z
         k_o = np.array([round(oracle.top_mass_fraction(zo[s]) * w.N) for s in range(w.rK)])
         assert np.abs(k_gpu - k_o).max() <= max(2, 1e-3 * w.N), (k_gpu, k_o)
+
+
+
+@pytest.mark.parametrize("flag", ["FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED"])
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
+def test_ablation_corrections(name, flag):
+    """The two correction ablations of [probe] (ridge without the subspace projection; the
+    residual mean added unprojected) against the oracle, the oracle's partition and route handed
+    in to both sides."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+
+    class Cfg:
+        pass
+
+    cfg = Cfg()
+    for f in ("rK", "Gk", "Gq", "rQ", "M", "r", "lam", "rho", "kmeans_iters", "seed"):
+        setattr(cfg, f, getattr(w, f))
+    cfg.flags = getattr(oracle, flag)
+    ref = oracle.sparsepr_attention(Q, K, V, cfg, partitions=res["partitions"], routes=res["routes"])
+    pt, rt = partition_tensors(res, w), route_tensors(res, w)
+    with spr.SparsePR.from_workload(w, flags=getattr(spr, flag)) as h:
+        part, route = spr.partition_from_tensors(pt), spr.route_from_tensors(rt)
+        Qp, Kp, Vp, Osp, O = (torch.empty_like(t) for t in (q, k, v, q, q))
+        h.permute(q, k, v, part, Qp, Kp, Vp)
+        h.blocksparse_attn(Qp, Kp, Vp, part, route, Osp)
+        fit = h.probe_fit(q, k, v, part, Osp)
+        h.writeback(part, Osp, fit, O)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+    assert not np.allclose(ref["O"], res["O"])          # the ablation changes the output
+    assert_close(bf16_to_f64(O), ref["O"], f"{flag} output")
