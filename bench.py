@@ -389,6 +389,91 @@ def run_ours(args):
     return 0
 
 
+def run_stack(args):
+    """A stack of `--layers` calls (one per denoising-step layer: fresh seeded inputs, locality
+    drawn per layer), two handles on two streams so that consecutive layers overlap, captured
+    once in a CUDA graph and replayed. Times the stack eagerly on one stream, eagerly on two
+    streams and as the graph (each after warm-up, CUDA events, max over ranks)."""
+    import torch
+    import torch.distributed as dist
+
+    import free_block_sparse_sparsepr_b200 as spr
+    from synthetic import get_workload, video_qkv_device
+    from synthetic.workloads import stack_layer_locality
+
+    rank, world = dist_init("nccl" if torch.cuda.is_available() else "gloo")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = get_workload(args.workload)
+    L = args.layers
+    ins = [video_qkv_device(w, layer=1000 * rank + l, locality=stack_layer_locality(l, w.seed), device=str(dev))
+           for l in range(L)]
+    outs = [torch.empty_like(q) for q, _, _ in ins]
+    hs = [spr.SparsePR.from_workload(w) for _ in range(2)]
+    streams = [torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)]
+
+    def stack(two: bool):
+        cur = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(cur)
+        for s in streams:
+            s.wait_event(fork)
+        for l, (q, k, v) in enumerate(ins):
+            i = l % 2 if two else 0
+            with torch.cuda.stream(streams[i]):
+                hs[i].attention(q, k, v, outs[l])
+        for s in streams:
+            join = torch.cuda.Event()
+            join.record(s)
+            cur.wait_event(join)
+
+    def timed(fn, reps):
+        cur = torch.cuda.current_stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        a.record(cur)
+        for _ in range(reps):
+            fn()
+        b.record(cur)
+        torch.cuda.synchronize()
+        barrier()
+        return reduce_max(a.elapsed_time(b) / reps, dev)
+
+    for _ in range(max(1, args.warmup)):
+        stack(True)
+    torch.cuda.synchronize()
+    eager1 = timed(lambda: stack(False), 1)
+    eager2 = timed(lambda: stack(True), 1)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        stack(True)
+    for _ in range(args.warmup):
+        graph.replay()
+    with ClockSampler(local) as clk:
+        ms = timed(graph.replay, args.steps)
+    flops = w.dense_equiv_flops() * L
+    if rank == 0:
+        print(json.dumps({
+            "metric": f"SparsePR {L}-layer stack (CUDA graph, two streams): dense-equiv TFLOPS",
+            "value": whole_job_value(flops, world, ms), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "ms_per_call": ms / L, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (drawn on the GPU)",
+            "config": dict(workload_config(w, world), layers=L,
+                           locality="U[0.4, 1.2] per layer, fresh seeded inputs per layer"),
+            "eager_one_stream_ms_per_call": eager1 / L, "eager_two_streams_ms_per_call": eager2 / L,
+            "graph_two_streams_ms_per_call": ms / L, "gpu_launches": hs[0].last_launch_count() * L,
+            "clocks": clk.summary(),
+        }), flush=True)
+    del graph
+    for hh in hs:
+        hh.close()
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -399,6 +484,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="> 1: time a stack of this many calls as one CUDA graph (two streams)")
     return ap.parse_args(argv)
 
 
@@ -406,6 +493,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.layers > 1:
+        return run_stack(args)
     return run_ours(args)
 
 

@@ -87,3 +87,32 @@ def video_qkv(w, layer: int = 0, locality: float | None = None, threads: int | N
             K[b, h] = k
             V[b, h] = v
     return Q, K, V
+
+
+def video_qkv_device(w, layer: int = 0, locality: float | None = None, device: str = "cuda"):
+    """The same recipe drawn on the GPU with torch's generator, as bf16 tensors Q [B, Hq, N, d],
+    K, V [B, Hkv, N, d]. Its random streams differ from video_qkv's (same distributions, other
+    values); it serves stacks of many layers, whose inputs would take minutes on the host."""
+    import torch
+
+    loc = w.locality if locality is None else locality
+    amp = AMPLITUDE * LOCALITY_GAIN * loc ** LOCALITY_EXPONENT
+    pos = torch.from_numpy(_positions(w.T, w.Hg, w.Wg)).to(device=device, dtype=torch.float64)
+    N, d, g = w.N, w.d, w.g
+    Q = torch.empty((w.B, w.Hq, N, d), dtype=torch.bfloat16, device=device)
+    K = torch.empty((w.B, w.Hkv, N, d), dtype=torch.bfloat16, device=device)
+    V = torch.empty((w.B, w.Hkv, N, d), dtype=torch.bfloat16, device=device)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            seed = int(np.random.SeedSequence([w.seed, layer, b, h]).generate_state(1, dtype=np.uint64)[0] >> 1)
+            gen = torch.Generator(device=device).manual_seed(seed)
+            omega = torch.rand((N_FEATURES, 3), generator=gen, device=device, dtype=torch.float64) * 2.5 + 0.5
+            theta = torch.rand((N_FEATURES,), generator=gen, device=device, dtype=torch.float64) * (2.0 * np.pi)
+            G = torch.randn((N_FEATURES, d), generator=gen, device=device, dtype=torch.float64) * np.sqrt(1.0 / N_FEATURES)
+            phi = torch.cos(2.0 * np.pi * (pos @ omega.T) + theta)
+            base = (amp * (phi @ G)).float()
+            K[b, h] = (base + w.noise * torch.randn((N, d), generator=gen, device=device)).bfloat16()
+            for j in range(g):
+                Q[b, h * g + j] = (base + w.noise * torch.randn((N, d), generator=gen, device=device)).bfloat16()
+            V[b, h] = torch.randn((N, d), generator=gen, device=device).bfloat16()
+    return Q, K, V
