@@ -223,14 +223,14 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     // (2b) query coordinates and query groups
     st = query_logits(h, Q, h->chi, h->clo, h->koff, s);
     if (st) return st;
-    if (h->proj && spr::coords_proj_supported(h->DPy, h->Gkp)) {
+    if (h->proj && spr::coords_proj_supported(h->DPy, c.Gk, h->Gkp)) {
         // centring, projection and normalisation in one pass over the logits
-        SPR_TRY(spr::launch_coords_proj(h->u, h->projT, h->ycoord, P, h->g, N, c.Gk, h->Gkp, s));
+        SPR_TRY(spr::launch_coords_proj(h->u, h->projT, h->ycoord, P, h->g, N, c.Gk, h->Gkp, h->num_sms, s));
     } else {
         SPR_TRY(spr::launch_coords_center(h->u, h->uhi, h->ulo, h->ycoord, P, h->g, N, c.Gk, h->Gkp, h->DPy, h->proj,
                                           s));
     }
-    if (h->proj && !spr::coords_proj_supported(h->DPy, h->Gkp)) {
+    if (h->proj && !spr::coords_proj_supported(h->DPy, c.Gk, h->Gkp)) {
         spr::GemmArgs b;
         memset(&b, 0, sizeof(b));
         b.A1 = h->uhi; b.A2 = h->ulo; b.sA = (long long)N * h->Gkp; b.lda = h->Gkp;

@@ -82,9 +82,9 @@ cudaError_t launch_coords_center(const float* u, bf16* uhi, bf16* ulo, float* y,
                                  int N, int Gk, int Gkp, int DPy, bool proj, cudaStream_t s);
 cudaError_t launch_rows_normalize(float* y, int rows, int DP, cudaStream_t s);
 // Gk > rQ in one pass: y [P][N][DPy] = normalise((mean_h u - row mean) . projT^T) (DPy = 64).
-bool coords_proj_supported(int DPy, int Gkp);
+bool coords_proj_supported(int DPy, int Gk, int Gkp);
 cudaError_t launch_coords_proj(const float* u, const bf16* projT, float* y, int P, int g, int N, int Gk, int Gkp,
-                               cudaStream_t s);
+                               int num_sms, cudaStream_t s);
 // projT [DPy][Gkp] bf16 = +-1 with the sign of bit 0 of splitmix64(seed ^ (g*rQ + t)).
 cudaError_t launch_make_projection(bf16* projT, int Gk, int Gkp, int rQ, int DPy,
                                    unsigned long long seed, cudaStream_t s);

@@ -170,33 +170,52 @@ __global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int* counts
 }
 
 // bases[z][ch][g] = rows of group g in chunks < ch; off[z][g] = exclusive scan of group sizes.
-__global__ void sort_scan_kernel(const int* __restrict__ counts, int* bases, int32_t* off,
+__global__ void __launch_bounds__(1024) sort_scan_kernel(const int* __restrict__ counts, int* bases, int32_t* off,
                                  const int* done, int G, int nch) {
     const int z = blockIdx.x;
     if (done && done[z]) return;
     extern __shared__ int tot[];
+    __shared__ int wsum[32];
     for (int g = threadIdx.x; g < G; g += blockDim.x) {
         int s = 0;
         const int* cz = counts + (long long)z * nch * G + g;
         int* bz = bases + (long long)z * nch * G + g;
-        int ch = 0;
-        for (; ch + 4 <= nch; ch += 4) {
-            int v0 = cz[(long long)ch * G], v1 = cz[(long long)(ch + 1) * G];
-            int v2 = cz[(long long)(ch + 2) * G], v3 = cz[(long long)(ch + 3) * G];
-            bz[(long long)ch * G] = s; s += v0;
-            bz[(long long)(ch + 1) * G] = s; s += v1;
-            bz[(long long)(ch + 2) * G] = s; s += v2;
-            bz[(long long)(ch + 3) * G] = s; s += v3;
+        for (int ch0 = 0; ch0 < nch; ch0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = ch0 + e < nch ? cz[(long long)(ch0 + e) * G] : 0;   // 8 loads in flight
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (ch0 + e < nch) { bz[(long long)(ch0 + e) * G] = s; s += v[e]; }
         }
-        for (; ch < nch; ++ch) { int v = cz[(long long)ch * G]; bz[(long long)ch * G] = s; s += v; }
         tot[g] = s;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int s = 0;
-        for (int g = 0; g < G; ++g) { int v = tot[g]; off[(long long)z * (G + 1) + g] = s; s += v; }
-        off[(long long)z * (G + 1) + G] = s;
+    // exclusive scan of the group totals (G <= blockDim.x): warp scans, then the warp totals
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int v = t < G ? tot[t] : 0;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += n;
     }
+    if (lane == 31) wsum[w] = inc;
+    __syncthreads();
+    if (w == 0) {
+        const int nw = (blockDim.x + 31) >> 5;
+        int x = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += n;
+        }
+        wsum[lane] = x;   // inclusive scan of warp totals
+    }
+    __syncthreads();
+    const int base = w > 0 ? wsum[w - 1] : 0;
+    if (t < G) off[(long long)z * (G + 1) + t] = base + inc - v;
+    if (t == G - 1) off[(long long)z * (G + 1) + G] = base + inc;
 }
 
 // Stable scatter: position = off[g] + rows of g in earlier chunks + earlier sub-chunks of this
