@@ -147,7 +147,9 @@ __global__ void make_projection_kernel(bf16* projT, int Gk, int Gkp, int rQ, int
 }
 
 // Probe m of a KV head: position p = floor((m+1/2)N/M) of the sequence ordered by
-// (group, radial distance, original index). Rank counting inside the group.
+// (group, radial distance, original index). Inside the group the keys (radial bits, position)
+// are sorted in shared memory (bitonic; radial distances are >= 0, so their bits order
+// like the values) when the group fits, else ranked by counting.
 constexpr int kProbeSmem = 4096;
 __global__ void __launch_bounds__(256) probe_select_kernel(const int32_t* __restrict__ qperm,
                                                            const int32_t* __restrict__ qoff,
@@ -160,26 +162,43 @@ __global__ void __launch_bounds__(256) probe_select_kernel(const int32_t* __rest
     const int a = upper_index(off, Gq, p);
     const int lo = off[a], cnt = off[a + 1] - lo;
     const int k = (int)(p - lo);
-    __shared__ float sr[kProbeSmem];
-    __shared__ int si[kProbeSmem];
+    __shared__ unsigned long long key[kProbeSmem];
     const int32_t* perm = qperm + (long long)z * N + lo;
     const float* rad = radial + (long long)z * N;
-    const bool staged = cnt <= kProbeSmem;
-    if (staged) {
-        for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
-            int idx = perm[j];
-            si[j] = idx;
-            sr[j] = rad[idx];
+    if (cnt <= kProbeSmem) {
+        int len = 1;
+        while (len < cnt) len <<= 1;
+        for (int j = threadIdx.x; j < len; j += blockDim.x) {
+            // the position j breaks ties: inside a group positions follow the original index
+            key[j] = j < cnt ? ((unsigned long long)__float_as_uint(rad[perm[j]]) << 32) | (unsigned)j : ~0ull;
         }
+        __syncthreads();
+        for (int kk = 2; kk <= len; kk <<= 1)
+            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+                for (int t = threadIdx.x; t < len; t += blockDim.x) {
+                    const int u = t ^ jj;
+                    if (u > t) {
+                        const unsigned long long x = key[t], y = key[u];
+                        if ((x > y) == ((t & kk) == 0)) { key[t] = y; key[u] = x; }
+                    }
+                }
+                __syncthreads();
+            }
+        if (threadIdx.x == 0) {
+            const int j = (int)(key[k] & 0xffffffffull);
+            probe[(long long)z * M + m] = perm[j];
+            probe_pos[(long long)z * M + m] = lo + j;
+            probe_seq[(long long)z * M + m] = (int)p;
+        }
+        return;
     }
-    __syncthreads();
     for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
-        const int ij = staged ? si[j] : perm[j];
-        const float rj = staged ? sr[j] : rad[ij];
+        const int ij = perm[j];
+        const float rj = rad[ij];
         int rank = 0;
         for (int e = 0; e < cnt; ++e) {
-            const int ie = staged ? si[e] : perm[e];
-            const float re = staged ? sr[e] : rad[ie];
+            const int ie = perm[e];
+            const float re = rad[ie];
             rank += (re < rj || (re == rj && ie < ij)) ? 1 : 0;
         }
         if (rank == k) {

@@ -279,55 +279,86 @@ __global__ void __launch_bounds__(256) writeback_kernel(const bf16* __restrict__
     float radd[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) radd[e] = (correct && Radd) ? Radd[(long long)x * D + lane * EPL + e] : 0.f;
+    // kRW rows per warp and iteration: every Bm / U^T value read from shared memory serves kRW rows
+    constexpr int kRW = 4;
     const int32_t* perm = qperm + (long long)z * N;
-    for (int p = blockIdx.x * 8 + warp; p < N; p += gridDim.x * 8) {
-        const bf16* src = Osp + ((long long)x * N + p) * D + lane * EPL;
-        float o[EPL];
+    for (int p0 = (blockIdx.x * 8 + warp) * kRW; p0 < N; p0 += gridDim.x * 8 * kRW) {
+        float o[kRW][EPL];
 #pragma unroll
-        for (int e = 0; e < EPL; e += 2) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + e));
-            o[e] = f.x;
-            o[e + 1] = f.y;
+        for (int q = 0; q < kRW; ++q) {
+            const bf16* src = Osp + ((long long)x * N + p0 + q) * D + lane * EPL;
+#pragma unroll
+            for (int e = 0; e < EPL; e += 2) {
+                float2 f = make_float2(0.f, 0.f);
+                if (p0 + q < N) f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + e));
+                o[q][e] = f.x;
+                o[q][e + 1] = f.y;
+            }
         }
         if (correct) {
-            float a[RP];
+            float a[kRW][RP];
 #pragma unroll
             for (int k = 0; k < RP; ++k) {
-                float acc = 0.f;
+                float bk[EPL];
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) acc = fmaf(sB[k * D + lane * EPL + e], o[e], acc);
-                a[k] = acc;
+                for (int e = 0; e < EPL; ++e) bk[e] = sB[k * D + lane * EPL + e];
+#pragma unroll
+                for (int q = 0; q < kRW; ++q) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc = fmaf(bk[e], o[q][e], acc);
+                    a[q][k] = acc;
+                }
             }
             // Step with lane bit b: lanes with b set keep the upper half of the remaining
             // partials (adding the partner's upper half), the others the lower half.
+            float tk[kRW];
 #pragma unroll
-            for (int n = RP, bit = 16; n > 1; n >>= 1, bit >>= 1) {
-                const bool up = (lane & bit) != 0;
+            for (int q = 0; q < kRW; ++q) {
 #pragma unroll
-                for (int i = 0; i < n / 2; ++i) {
-                    const float send = up ? a[i] : a[i + n / 2];
-                    const float keep = up ? a[i + n / 2] : a[i];
-                    a[i] = keep + __shfl_xor_sync(kFull, send, bit);
+                for (int n = RP, bit = 16; n > 1; n >>= 1, bit >>= 1) {
+                    const bool up = (lane & bit) != 0;
+#pragma unroll
+                    for (int i = 0; i < n / 2; ++i) {
+                        const float send = up ? a[q][i] : a[q][i + n / 2];
+                        const float keep = up ? a[q][i + n / 2] : a[q][i];
+                        a[q][i] = keep + __shfl_xor_sync(kFull, send, bit);
+                    }
                 }
+                if (RP == 16) a[q][0] += __shfl_xor_sync(kFull, a[q][0], 1);   // lanes 2k, 2k+1 held halves
+                tk[q] = a[q][0];
             }
-            if (RP == 16) a[0] += __shfl_xor_sync(kFull, a[0], 1);   // lanes 2k, 2k+1 held halves of t_k
-            const float tk = a[0];
-            float delta[EPL];
+            float delta[kRW][EPL];
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) delta[e] = 0.f;
+            for (int q = 0; q < kRW; ++q)
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) delta[q][e] = 0.f;
 #pragma unroll
             for (int k = 0; k < RP; ++k) {
-                const float t = __shfl_sync(kFull, tk, (RP == 16) ? 2 * k : k) + sc[k];
+                float uk[EPL];
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) delta[e] = fmaf(sUt[k * D + lane * EPL + e], t, delta[e]);
+                for (int e = 0; e < EPL; ++e) uk[e] = sUt[k * D + lane * EPL + e];
+                const float ck = sc[k];
+#pragma unroll
+                for (int q = 0; q < kRW; ++q) {
+                    const float t = __shfl_sync(kFull, tk[q], (RP == 16) ? 2 * k : k) + ck;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) delta[q][e] = fmaf(uk[e], t, delta[q][e]);
+                }
             }
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[e] += delta[e] + radd[e];
-        }
-        bf16* dst = O + ((long long)x * N + perm[p]) * D + lane * EPL;
+            for (int q = 0; q < kRW; ++q)
 #pragma unroll
-        for (int e = 0; e < EPL; e += 2)
-            *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(o[e], o[e + 1]);
+                for (int e = 0; e < EPL; ++e) o[q][e] += delta[q][e] + radd[e];
+        }
+#pragma unroll
+        for (int q = 0; q < kRW; ++q) {
+            if (p0 + q >= N) break;
+            bf16* dst = O + ((long long)x * N + perm[p0 + q]) * D + lane * EPL;
+#pragma unroll
+            for (int e = 0; e < EPL; e += 2)
+                *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(o[q][e], o[q][e + 1]);
+        }
     }
 }
 
@@ -422,7 +453,7 @@ cudaError_t launch_fit(const float* R, const float* Xp, const float* w, float la
 cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float* U,
                              const float* Bm, const float* c0, const float* Radd, bf16* O, int Hp, int g, int N,
                              int d, int r, bool correct, cudaStream_t s) {
-    const int blocks = (N + 8 * 16 - 1) / (8 * 16);   // 16 rows per warp
+    const int blocks = (N + 8 * 16 - 1) / (8 * 16);   // 16 rows per warp (4 iterations of 4)
     dim3 grid(blocks, Hp);
     const int cf = correct ? 1 : 0;
     if (r <= 16) {
