@@ -64,6 +64,7 @@ __global__ void cell_scores_kernel(const float* __restrict__ u, const float* __r
 // ascending a, g) and a cost-weighted radix select finds the first cell whose inclusion would
 // exceed the remaining budget; it is kept iff its overshoot < the remaining undershoot.
 constexpr int kSelThreads = 1024;
+constexpr int kRadix = 2048;   // 11-bit digits
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     const float* __restrict__ scores, const int32_t* __restrict__ qoff, const int32_t* __restrict__ koff,
     int32_t* rowptr, int32_t* kg, int64_t* pairs, int Gq, int Gk, long long budget, int keep_all) {
@@ -73,7 +74,9 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     int* ks = qs + Gq;        // [Gk]
     int* mand = ks + Gk;      // [Gq]
     int* rowcnt = mand + Gq;  // [Gq]
-    __shared__ unsigned long long hist[256];
+    __shared__ unsigned long long hist[kRadix];
+    __shared__ int hcnt[kRadix];
+    __shared__ int s_unique;
     __shared__ long long red[32];
     __shared__ long long s_rem;
     __shared__ unsigned long long s_prefix, s_mask;
@@ -124,28 +127,42 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
         s_prefix = 0ull;
         s_mask = 0ull;
         s_found = keep_all ? 0 : 1;
+        s_unique = 0;
     }
     __syncthreads();
 
-    const long long ncell = (long long)Gq * Gk;
+    // Radix select over 64-bit keys (~score bits, cell index), 11 bits at a time from the top,
+    // weighted by cell cost; thread t visits the cells a * Gk + gk with gk = t % Gk (no division
+    // per cell). A digit bin holding a single candidate ends the descent: one more pass reads
+    // that candidate's full key.
+    const int gk0 = tid % Gk, astep = blockDim.x / Gk;
+    const bool lane_ok = tid < astep * Gk;
+    const bool gk_ok = ks[gk0] > 0;
     if (!keep_all) {
-        for (int shift = 56; shift >= 0; shift -= 8) {
-            for (int t = tid; t < 256; t += blockDim.x) hist[t] = 0ull;
+        bool unique = false;
+        for (int shift = 53; shift > -11 && !unique; shift -= 11) {
+            const int sh = shift > 0 ? shift : 0, bits = shift > 0 ? 11 : 11 + shift;
+            const unsigned long long dmask = (1ull << bits) - 1ull;
+            for (int t = tid; t < kRadix; t += blockDim.x) { hist[t] = 0ull; hcnt[t] = 0; }
             __syncthreads();
             const unsigned long long prefix = s_prefix, mask = s_mask;
-            for (long long c = tid; c < ncell; c += blockDim.x) {
-                const int a = (int)(c / Gk), gk = (int)(c % Gk);
-                if (qs[a] == 0 || ks[gk] == 0 || mand[a] == gk) continue;
-                const unsigned long long key =
-                    ((unsigned long long)(~__float_as_uint(S[c])) << 32) | (unsigned long long)c;
-                if ((key & mask) != prefix) continue;
-                atomicAdd(&hist[(key >> shift) & 255ull], (unsigned long long)((long long)qs[a] * ks[gk]));
+            if (lane_ok && gk_ok) {
+                for (int a = tid / Gk; a < Gq; a += astep) {
+                    if (qs[a] == 0 || mand[a] == gk0) continue;
+                    const long long c = (long long)a * Gk + gk0;
+                    const unsigned long long key =
+                        ((unsigned long long)(~__float_as_uint(S[c])) << 32) | (unsigned long long)c;
+                    if ((key & mask) != prefix) continue;
+                    const int dg = (int)((key >> sh) & dmask);
+                    atomicAdd(&hist[dg], (unsigned long long)((long long)qs[a] * ks[gk0]));
+                    atomicAdd(&hcnt[dg], 1);
+                }
             }
             __syncthreads();
             if (tid == 0) {
                 long long cum = 0;
                 int dsel = -1;
-                for (int dg = 0; dg < 256; ++dg) {
+                for (int dg = 0; dg <= (int)dmask; ++dg) {
                     long long h = (long long)hist[dg];
                     if (h > 0 && cum + h > s_rem) { dsel = dg; break; }
                     cum += h;
@@ -154,12 +171,28 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
                     s_found = 0;  // every remaining candidate fits in the budget
                 } else {
                     s_rem -= cum;
-                    s_prefix |= (unsigned long long)dsel << shift;
-                    s_mask |= 255ull << shift;
+                    s_prefix |= (unsigned long long)dsel << sh;
+                    s_mask |= dmask << sh;
+                    s_unique = hcnt[dsel] == 1;
                 }
             }
             __syncthreads();
             if (!s_found) break;
+            unique = s_unique;
+        }
+        if (s_found && unique) {
+            // the lone candidate under the prefix: its full key
+            const unsigned long long prefix = s_prefix, mask = s_mask;
+            if (lane_ok && gk_ok) {
+                for (int a = tid / Gk; a < Gq; a += astep) {
+                    if (qs[a] == 0 || mand[a] == gk0) continue;
+                    const long long c = (long long)a * Gk + gk0;
+                    const unsigned long long key =
+                        ((unsigned long long)(~__float_as_uint(S[c])) << 32) | (unsigned long long)c;
+                    if ((key & mask) == prefix) s_prefix = key;
+                }
+            }
+            __syncthreads();
         }
     }
     const int found = s_found;
