@@ -92,10 +92,12 @@ __global__ void __launch_bounds__(kAssignRows) km_assign_kernel(const float* __r
 }
 
 // New centroid = mean of its members in fp64, stored fp32; an empty group keeps its centroid.
-// One block per group: thread t reads feature quad t % (DP/4) (a float4) of the rows at
-// positions lo + slice, lo + slice + nslices, ... of the group (perm order), four rows in flight;
-// the slices are then summed in a fixed order, so the result does not depend on scheduling.
+// One block per group: the group's row indices (perm order) are staged in shared memory, then
+// thread t reads feature quad t % (DP/4) (a float4) of the rows at positions slice,
+// slice + nslices, ... of the group, eight rows in flight (no index load in the dependence
+// chain); the slices are summed in a fixed order, so the result does not depend on scheduling.
 constexpr int kUpdThreads = 256;
+constexpr int kUpdIdx = 2048;       // row indices staged per round
 template <int DP>
 __global__ void __launch_bounds__(kUpdThreads) km_update_kernel(const float* __restrict__ X,
                                                                 const int32_t* __restrict__ perm,
@@ -103,34 +105,41 @@ __global__ void __launch_bounds__(kUpdThreads) km_update_kernel(const float* __r
                                                                 const int* done, int n, int G) {
     constexpr int kQ = DP / 4;                       // float4 quads per row
     constexpr int kSl = kUpdThreads / kQ;            // row slices
+    constexpr int kU = 8;                            // rows in flight per slice
     const int z = blockIdx.y, g = blockIdx.x;
     if (done && done[z]) return;
     const int lo = off[(long long)z * (G + 1) + g], hi = off[(long long)z * (G + 1) + g + 1];
     if (hi <= lo) return;
     const int q = threadIdx.x % kQ, rs = threadIdx.x / kQ;
     __shared__ double red[kSl][DP];
-    if (rs < kSl) {
-        const int32_t* pz = perm + (long long)z * n;
-        const float4* xz = reinterpret_cast<const float4*>(X + (long long)z * n * DP) + q;
-        double a[4][4] = {};
-        int j = lo + rs;
-        for (; j + 3 * kSl < hi; j += 4 * kSl) {
-            int r[4];
+    __shared__ int sIdx[kUpdIdx];
+    const int32_t* pz = perm + (long long)z * n;
+    const float4* xz = reinterpret_cast<const float4*>(X + (long long)z * n * DP) + q;
+    double a[4][4] = {};
+    for (int base = lo; base < hi; base += kUpdIdx) {
+        const int cnt = min(kUpdIdx, hi - base);
+        __syncthreads();
+        for (int t = threadIdx.x; t < cnt; t += kUpdThreads) sIdx[t] = __ldg(pz + base + t);
+        __syncthreads();
+        if (rs < kSl) {
+            int j = rs;
+            for (; j + (kU - 1) * kSl < cnt; j += kU * kSl) {
+                float4 v[kU];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) r[u] = __ldg(pz + j + u * kSl);
-            float4 v[4];
+                for (int u = 0; u < kU; ++u) v[u] = __ldg(xz + (long long)sIdx[j + u * kSl] * kQ);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = __ldg(xz + (long long)r[u] * kQ);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                a[u][0] += (double)v[u].x; a[u][1] += (double)v[u].y;
-                a[u][2] += (double)v[u].z; a[u][3] += (double)v[u].w;
+                for (int u = 0; u < kU; ++u) {
+                    a[u & 3][0] += (double)v[u].x; a[u & 3][1] += (double)v[u].y;
+                    a[u & 3][2] += (double)v[u].z; a[u & 3][3] += (double)v[u].w;
+                }
+            }
+            for (; j < cnt; j += kSl) {
+                const float4 v = __ldg(xz + (long long)sIdx[j] * kQ);
+                a[0][0] += (double)v.x; a[0][1] += (double)v.y; a[0][2] += (double)v.z; a[0][3] += (double)v.w;
             }
         }
-        for (; j < hi; j += kSl) {
-            const float4 v = __ldg(xz + (long long)__ldg(pz + j) * kQ);
-            a[0][0] += (double)v.x; a[0][1] += (double)v.y; a[0][2] += (double)v.z; a[0][3] += (double)v.w;
-        }
+    }
+    if (rs < kSl) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) red[rs][4 * q + e] = (a[0][e] + a[1][e]) + (a[2][e] + a[3][e]);
     }

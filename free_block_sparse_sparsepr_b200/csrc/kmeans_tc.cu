@@ -312,26 +312,39 @@ __device__ __forceinline__ void split2(float v, bf16& a, bf16& b) {
 
 // X [rows][DP] fp32 -> two bf16 parts [rows][DP] (part q at X2 + q*stride) and ||x||^2 in fp32;
 // one warp per row.
+constexpr int kSplitRowsPerWarp = 4;
 __global__ void km_split_rows_kernel(const float* __restrict__ X, bf16* X2, long long stride, float* xx,
                                      long long rows, int DP) {
-    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const long long row0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kSplitRowsPerWarp;
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    float ss = 0.f;
+    if (row0 >= rows) return;
+    float v[kSplitRowsPerWarp][2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int c = lane + 32 * h;
-        if (c < DP) {
-            const float v = X[row * DP + c];
-            ss = fmaf(v, v, ss);
-            bf16 a, b;
-            split2(v, a, b);
-            X2[row * DP + c] = a;
-            X2[stride + row * DP + c] = b;
+    for (int q = 0; q < kSplitRowsPerWarp; ++q)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = lane + 32 * h;
+            v[q][h] = (row0 + q < rows && c < DP) ? __ldg(X + (row0 + q) * DP + c) : 0.f;
         }
+#pragma unroll
+    for (int q = 0; q < kSplitRowsPerWarp; ++q) {
+        const long long row = row0 + q;
+        if (row >= rows) break;
+        float ss = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = lane + 32 * h;
+            ss = fmaf(v[q][h], v[q][h], ss);
+            if (c < DP) {
+                bf16 a, b;
+                split2(v[q][h], a, b);
+                X2[row * DP + c] = a;
+                X2[stride + row * DP + c] = b;
+            }
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) xx[row] = ss;
     }
-    ss = warp_sum(ss);
-    if (lane == 0) xx[row] = ss;
 }
 
 // C [P][G][DP] fp32 -> two bf16 parts [P][G16][64] (zero past G and DP, part q at C2 + q*stride)
@@ -490,7 +503,9 @@ void km_grid(int P, int n, int num_sms, int* per, int* cap) {
 
 cudaError_t launch_km_split_rows(const float* X, bf16* X2, float* xx, int P, int n, int DP, cudaStream_t s) {
     const long long rows = (long long)P * n;
-    km_split_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(X, X2, rows * DP, xx, rows, DP);
+    const long long per_block = 8ll * kSplitRowsPerWarp;
+    km_split_rows_kernel<<<(unsigned)((rows + per_block - 1) / per_block), 256, 0, s>>>(X, X2, rows * DP, xx, rows,
+                                                                                        DP);
     return cudaGetLastError();
 }
 
