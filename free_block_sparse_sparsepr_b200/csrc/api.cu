@@ -343,7 +343,7 @@ sparsepr_status writeback_impl(sparsepr_handle h, const sparsepr_partition_t* p,
         const float* radd = (correct && (c.flags & SPARSEPR_FLAG_RBAR_UNPROJECTED)) ? f->Rbar : nullptr;
         SPR_TRY(spr::launch_writeback(Osp, p->qperm, correct ? f->U : nullptr, correct ? f->Bm : nullptr,
                                       correct ? f->c0 : nullptr, radd, O, h->Hp, h->g, c.N, c.d, correct ? c.r : 1,
-                                      correct, s));
+                                      correct, h->num_sms, s));
     }
     if (correct) SPR_TRY(spr::launch_probe_override(f->Odense, p->probe, O, h->Hp, h->g, c.N, c.d, h->M, s));
     return SPARSEPR_OK;

@@ -25,7 +25,10 @@ __device__ __forceinline__ void split3(float v, float& a, float& b, float& c) {
     c = r - b;
 }
 
-__global__ void __launch_bounds__(kWarps * 32) coords_proj_kernel(const float* __restrict__ u,
+// kOneHead: g == 1, so the next 16 columns' loads are issued before this step's MMAs (a
+// register double buffer); with several heads their sum is formed as the loads arrive.
+template <bool kOneHead>
+__global__ void __launch_bounds__(kWarps * 32, 5) coords_proj_kernel(const float* __restrict__ u,
                                                                   const bf16* __restrict__ projT, float* y, int g,
                                                                   int N, int Gk, int Gkp) {
     extern __shared__ __align__(16) unsigned char cp_raw[];
@@ -57,17 +60,30 @@ __global__ void __launch_bounds__(kWarps * 32) coords_proj_kernel(const float* _
 #pragma unroll
             for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
         float sa = 0.f, sb = 0.f;
-#pragma unroll 2
-        for (int k0 = 0; k0 < Gkp; k0 += 16) {
+        // the four float2 of the lane's A fragment at column step k0 (rows ra / rb, columns c0 / c1)
+        auto load_step = [&](int k0, float2 (&x)[4]) {
             const int c0 = k0 + (lane & 3) * 2, c1 = c0 + 8;
-            float2 x[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            for (int j = 0; j < g; ++j) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) x[q] = make_float2(0.f, 0.f);
+            for (int j = 0; j < (kOneHead ? 1 : g); ++j) {
                 const float* ua = u + (((long long)z * g + j) * N + ra) * Gk;
                 const float* ub = ua + 8ll * Gk;
-                if (va && c0 < Gk) { const float2 t = *reinterpret_cast<const float2*>(ua + c0); x[0].x += t.x; x[0].y += t.y; }
-                if (vb && c0 < Gk) { const float2 t = *reinterpret_cast<const float2*>(ub + c0); x[1].x += t.x; x[1].y += t.y; }
-                if (va && c1 < Gk) { const float2 t = *reinterpret_cast<const float2*>(ua + c1); x[2].x += t.x; x[2].y += t.y; }
-                if (vb && c1 < Gk) { const float2 t = *reinterpret_cast<const float2*>(ub + c1); x[3].x += t.x; x[3].y += t.y; }
+                if (va && c0 < Gk) { const float2 t = __ldg(reinterpret_cast<const float2*>(ua + c0)); x[0].x += t.x; x[0].y += t.y; }
+                if (vb && c0 < Gk) { const float2 t = __ldg(reinterpret_cast<const float2*>(ub + c0)); x[1].x += t.x; x[1].y += t.y; }
+                if (va && c1 < Gk) { const float2 t = __ldg(reinterpret_cast<const float2*>(ua + c1)); x[2].x += t.x; x[2].y += t.y; }
+                if (vb && c1 < Gk) { const float2 t = __ldg(reinterpret_cast<const float2*>(ub + c1)); x[3].x += t.x; x[3].y += t.y; }
+            }
+        };
+        float2 xn[4];
+        if (kOneHead) load_step(0, xn);
+        for (int k0 = 0; k0 < Gkp; k0 += 16) {
+            float2 x[4];
+            if (kOneHead) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) x[q] = xn[q];
+                if (k0 + 16 < Gkp) load_step(k0 + 16, xn);
+            } else {
+                load_step(k0, x);
             }
             uint32_t af[3][4];
 #pragma unroll
@@ -133,13 +149,21 @@ bool coords_proj_supported(int DPy, int Gk, int Gkp) {
 cudaError_t launch_coords_proj(const float* u, const bf16* projT, float* y, int P, int g, int N, int Gk, int Gkp,
                                int num_sms, cudaStream_t s) {
     const size_t smem = (size_t)kOut * (Gkp + 8) * sizeof(bf16) + kOut * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(coords_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = g == 1 ? coords_proj_kernel<true> : coords_proj_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int tiles = (N + 15) / 16;
-    int per = (8 * num_sms + P - 1) / P;
+    // persistent CTAs: as many as fit on the GPU at once (a second, partial wave would double
+    // the time of the slowest CTA)
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    int per = occ * num_sms / P;
+    if (per < 1) per = 1;
     const int maxper = (tiles + kWarps - 1) / kWarps;
     if (per > maxper) per = maxper;
-    coords_proj_kernel<<<dim3(per, P), kWarps * 32, smem, s>>>(u, projT, y, g, N, Gk, Gkp);
+    kern<<<dim3(per, P), kWarps * 32, smem, s>>>(u, projT, y, g, N, Gk, Gkp);
     return cudaGetLastError();
 }
 

@@ -33,11 +33,14 @@ __global__ void probe_residual_kernel(const float* __restrict__ Od, const bf16* 
 //   Bm = U^T A, c0 = U^T Rbar - Bm xbar  so that the correction is U (c0 + Bm o).
 constexpr int kFitThreads = 512;
 constexpr int kFitWarps = kFitThreads / 32;
+template <int D>
 __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     const float* __restrict__ Rg, const float* __restrict__ Xg, const float* __restrict__ wts,
     float lambda, float* obar, float* Rbar, float* A, float* U, float* Bm, float* c0,
-    int32_t* rank_out, int g, int d, int M, int r, int rbar_unprojected, int* status) {
-    const int x = blockIdx.x, z = x / g, tid = threadIdx.x, nt = blockDim.x;
+    int32_t* rank_out, int g, int M, int r, int rbar_unprojected, int* status) {
+    constexpr int d = D;
+    constexpr int nt = kFitThreads;
+    const int x = blockIdx.x, z = x / g, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int Mp = (M + 1) & ~1;
     const int ld = d + 1;            // padded row stride: column-wise walks hit distinct banks
@@ -53,6 +56,7 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
     float* yb = xb + d;              // [d]
     float* nrm = yb + d;             // [M]
     int* sel = reinterpret_cast<int*>(nrm + M);   // [r]
+    float* inv_diag = nrm;           // [M] 1 / L[j][j] during the solves (nrm is written after them)
     __shared__ float sW;
     __shared__ int s_rank, s_rot;
 
@@ -86,96 +90,168 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
         Y[m * ld + c] = sw[m] * (Y[m * ld + c] - yb[c]);
     }
     __syncthreads();
-    // Km = Xs Xs^T + lambda I: one warp per entry, lanes over the d columns
-    for (int e = warp; e < M * M; e += kFitWarps) {
-        const int i = e / M, j = e % M;
-        if (j > i) continue;
-        float acc = 0.f;
-        for (int c = lane; c < d; c += 32) acc = fmaf(X[i * ld + c], X[j * ld + c], acc);
-        acc = warp_sum(acc);
-        if (lane == 0) {
-            Km[i * M + j] = acc + (i == j ? lambda : 0.f);
-            Km[j * M + i] = acc + (i == j ? lambda : 0.f);
+    // Km = Xs Xs^T + lambda I, lower triangle, in 2 x 2 register blocks (rows past M read as 0)
+    {
+        const int Mb = (M + 1) / 2, nb = Mb * (Mb + 1) / 2;
+        for (int e = tid; e < nb; e += nt) {
+            int ib = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+            while (ib * (ib + 1) / 2 > e) --ib;
+            while ((ib + 1) * (ib + 2) / 2 <= e) ++ib;
+            const int jb = e - ib * (ib + 1) / 2;
+            const int i0 = 2 * ib, j0 = 2 * jb;
+            const bool i1ok = i0 + 1 < M, j1ok = j0 + 1 < M;
+            float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+            for (int c = 0; c < d; ++c) {
+                const float xi0 = X[i0 * ld + c], xj0 = X[j0 * ld + c];
+                const float xi1 = i1ok ? X[(i0 + 1) * ld + c] : 0.f, xj1 = j1ok ? X[(j0 + 1) * ld + c] : 0.f;
+                a00 = fmaf(xi0, xj0, a00);
+                a01 = fmaf(xi0, xj1, a01);
+                a10 = fmaf(xi1, xj0, a10);
+                a11 = fmaf(xi1, xj1, a11);
+            }
+            Km[i0 * M + j0] = a00 + (i0 == j0 ? lambda : 0.f);
+            if (j1ok && j0 + 1 <= i0) Km[i0 * M + j0 + 1] = a01;
+            if (i1ok) Km[(i0 + 1) * M + j0] = a10;
+            if (i1ok && j1ok) Km[(i0 + 1) * M + j0 + 1] = a11 + (i0 == j0 ? lambda : 0.f);
         }
     }
     __syncthreads();
-    // Cholesky Km = L L^T (lower triangle, in place)
+    // Cholesky Km = L L^T (lower triangle, in place), right-looking: scale column j, then
+    // update the trailing triangle
     for (int j = 0; j < M; ++j) {
-        if (warp == 0) {
-            float s = 0.f;
-            for (int k = lane; k < j; k += 32) s = fmaf(Km[j * M + k], Km[j * M + k], s);
-            s = Km[j * M + j] - warp_sum(s);
-            if (lane == 0) {
-                if (!(s > 0.f)) { set_status(status, kDevBounds); s = 1e-30f; }
-                Km[j * M + j] = sqrtf(s);
+        float djj = Km[j * M + j];
+        if (!(djj > 0.f)) {
+            if (tid == 0) set_status(status, kDevBounds);
+            djj = 1e-30f;
+        }
+        const float dj = sqrtf(djj);
+        for (int i = j + 1 + tid; i < M; i += nt) Km[i * M + j] = Km[i * M + j] / dj;
+        __syncthreads();
+        if (tid == 0) Km[j * M + j] = dj;
+        {
+            const int k = j + 1 + (tid & 63);
+            if (k < M) {
+                const float lk = Km[k * M + j];
+#pragma unroll 4
+                for (int i = j + 1 + (tid >> 6); i < M; i += nt / 64)
+                    if (k <= i) Km[i * M + k] = fmaf(-Km[i * M + j], lk, Km[i * M + k]);
             }
         }
         __syncthreads();
-        for (int i = j + 1 + tid; i < M; i += nt) {
-            float s = Km[i * M + j];
-            for (int k = 0; k < j; ++k) s -= Km[i * M + k] * Km[j * M + k];
-            Km[i * M + j] = s / Km[j * M + j];
-        }
-        __syncthreads();
     }
-    // Z = Km^-1 Xs, column by column, in place in X
-    for (int c = tid; c < d; c += nt) {
-        for (int m = 0; m < M; ++m) {
-            float s = X[m * ld + c];
-            for (int k = 0; k < m; ++k) s -= Km[m * M + k] * X[k * ld + c];
-            X[m * ld + c] = s / Km[m * M + m];
+    for (int t = tid; t < M; t += nt) inv_diag[t] = 1.f / Km[t * M + t];
+    __syncthreads();
+    // Z = Km^-1 Xs, in place in X: L y = Xs then L^T z = y. Each column is owned by kLpc lanes
+    // of one warp (rows interleaved among them), so the substitutions need only warp barriers.
+    {
+        constexpr int lpc = nt / d;                  // lanes per column (4 at d = 128, 8 at d = 64)
+        const int col = tid / lpc, rs = tid % lpc;
+        for (int jj = 0; jj < M; ++jj) {
+            __syncwarp();
+            const float yj = X[jj * ld + col] * inv_diag[jj];
+            __syncwarp();
+            if ((jj & (lpc - 1)) == rs) X[jj * ld + col] = yj;
+            const int i0 = jj + 1 + ((rs - jj - 1) & (lpc - 1));
+#pragma unroll 4
+            for (int i = i0; i < M; i += lpc) X[i * ld + col] = fmaf(-Km[i * M + jj], yj, X[i * ld + col]);
         }
         for (int m = M - 1; m >= 0; --m) {
-            float s = X[m * ld + c];
-            for (int k = m + 1; k < M; ++k) s -= Km[k * M + m] * X[k * ld + c];
-            X[m * ld + c] = s / Km[m * M + m];
+            __syncwarp();
+            const float zm = X[m * ld + col] * inv_diag[m];
+            __syncwarp();
+            if ((m & (lpc - 1)) == rs) X[m * ld + col] = zm;
+#pragma unroll 4
+            for (int k = rs; k < m; k += lpc) X[k * ld + col] = fmaf(-Km[m * M + k], zm, X[k * ld + col]);
         }
     }
     __syncthreads();
+    // A = Ys^T Z (d x d): each thread a 4 x (d/16) register tile, columns c2 interleaved by 16
     float* Ax = A + (long long)x * d * d;
-    for (int t = tid; t < d * d; t += nt) {
-        const int c = t / d, c2 = t % d;
-        float acc = 0.f;
-        for (int m = 0; m < M; ++m) acc = fmaf(Y[m * ld + c], X[m * ld + c2], acc);
-        Ax[t] = acc;
-    }
-    // One-sided Jacobi on the columns of W (round-robin disjoint pairs, one warp per pair)
-    for (int sweep = 0; sweep < 12; ++sweep) {
-        if (tid == 0) s_rot = 0;
-        __syncthreads();
-        for (int k = 0; k < Mp - 1; ++k) {
-            for (int i = warp; i < Mp / 2; i += kFitWarps) {
-                const int a1 = (i == 0) ? 0 : ((i - 1 + k) % (Mp - 1)) + 1;
-                const int b1 = ((Mp - 2 - i + k) % (Mp - 1)) + 1;
-                const int pc = min(a1, b1), qc = max(a1, b1);
-                if (qc >= M) continue;
-                float al = 0.f, be = 0.f, ga = 0.f;
-                for (int c = lane; c < d; c += 32) {
-                    const float u1 = Wc[pc * ld + c], u2 = Wc[qc * ld + c];
-                    al = fmaf(u1, u1, al);
-                    be = fmaf(u2, u2, be);
-                    ga = fmaf(u1, u2, ga);
-                }
-                al = warp_sum(al);
-                be = warp_sum(be);
-                ga = warp_sum(ga);
-                if (fabsf(ga) > 1e-7f * sqrtf(al * be) && ga != 0.f) {
-                    const float zeta = (be - al) / (2.f * ga);
-                    const float tt = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(zeta * zeta + 1.f));
-                    const float cs = 1.f / sqrtf(tt * tt + 1.f), sn = tt * cs;
-                    for (int c = lane; c < d; c += 32) {
-                        const float u1 = Wc[pc * ld + c], u2 = Wc[qc * ld + c];
-                        Wc[pc * ld + c] = cs * u1 - sn * u2;
-                        Wc[qc * ld + c] = sn * u1 + cs * u2;
-                    }
-                    if (lane == 0) s_rot = 1;
-                }
+    {
+        const int ne = d / 16;
+        for (int t = tid; t < (d / 4) * 16; t += nt) {
+            const int cb = t / 16, c2b = t % 16;
+            float acc[4][8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[q][e] = 0.f;
+            for (int m = 0; m < M; ++m) {
+                float yv[4], zv[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) yv[q] = Y[m * ld + 4 * cb + q];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) zv[e] = e < ne ? X[m * ld + c2b + 16 * e] : 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[q][e] = fmaf(yv[q], zv[e], acc[q][e]);
             }
-            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (e < ne) Ax[(long long)(4 * cb + q) * d + c2b + 16 * e] = acc[q][e];
         }
-        const int rotated = s_rot;   // read by every thread before thread 0 resets it
-        __syncthreads();
-        if (!rotated) break;
+    }
+    // One-sided Jacobi on the columns of W (round-robin disjoint pairs, one half-warp per pair:
+    // every pair of a round at once). Round k pairs column a(i, k) with b(i, k); both indices
+    // advance by one (mod Mp - 1) from round to round.
+    {
+        const int hw = tid >> 4, hl = tid & 15;
+        constexpr int kE = D / 16;                   // elements of a column per lane
+        // a pair counts as orthogonal once |u1.u2| <= sqrt(d) eps |u1||u2|, the rounding level of
+        // an fp32 dot product of length d
+        const float jtol = sqrtf((float)d) * FLT_EPSILON, jtol2 = jtol * jtol;
+        const int np = Mp / 2, nm = Mp - 1;
+        for (int sweep = 0; sweep < 16; ++sweep) {
+            if (tid == 0) s_rot = 0;
+            __syncthreads();
+            int ia = hw == 0 ? 0 : hw - 1, ib = (Mp - 2 - hw) % nm;   // (i - 1 + k), (Mp - 2 - i + k) mod nm at k = 0
+            if (ib < 0) ib += nm;
+            for (int k = 0; k < nm; ++k) {
+                const int a1 = hw == 0 ? 0 : ia + 1, b1 = ib + 1;
+                const int pc = min(a1, b1), qc = max(a1, b1);
+                const bool valid = hw < np && qc < M;
+                float u1[kE], u2[kE];
+                float al = 0.f, be = 0.f, ga = 0.f;
+#pragma unroll
+                for (int e = 0; e < kE; ++e) {
+                    u1[e] = valid ? Wc[pc * ld + hl + 16 * e] : 0.f;
+                    u2[e] = valid ? Wc[qc * ld + hl + 16 * e] : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < kE; ++e) {
+                    al = fmaf(u1[e], u1[e], al);
+                    be = fmaf(u2[e], u2[e], be);
+                    ga = fmaf(u1[e], u2[e], ga);
+                }
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) {
+                    al += __shfl_xor_sync(kFull, al, o);
+                    be += __shfl_xor_sync(kFull, be, o);
+                    ga += __shfl_xor_sync(kFull, ga, o);
+                }
+                if (valid && ga != 0.f && ga * ga > jtol2 * (al * be)) {
+                    // tan of the rotation angle: the smaller root of t^2 + 2 zeta t - 1 = 0
+                    const float zeta = __fdividef(be - al, 2.f * ga);
+                    const float tt = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
+                    const float cs = rsqrtf(fmaf(tt, tt, 1.f)), sn = tt * cs;
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) {
+                        Wc[pc * ld + hl + 16 * e] = cs * u1[e] - sn * u2[e];
+                        Wc[qc * ld + hl + 16 * e] = sn * u1[e] + cs * u2[e];
+                    }
+                    if (hl == 0) s_rot = 1;
+                }
+                ia = ia + 1 == nm ? 0 : ia + 1;
+                ib = ib + 1 == nm ? 0 : ib + 1;
+                __syncthreads();
+            }
+            const int rotated = s_rot;   // read by every thread before thread 0 resets it
+            __syncthreads();
+            if (!rotated) break;
+        }
     }
     // column norms = singular values; top r (descending, ties -> lower index) and the rank
     for (int m = warp; m < M; m += kFitWarps) {
@@ -221,11 +297,20 @@ __global__ void __launch_bounds__(kFitThreads) fit_kernel(
         U[(long long)x * d * r + t] = val;
     }
     __syncthreads();
+    // Bm = U^T A = (Ys U)^T Z: T = Ys U (M x r, in Km's space, free since the solves), then T^T Z
+    float* T = Km;
+    for (int t = tid; t < M * r; t += nt) {
+        const int m = t / r, k = t % r;
+        float acc = 0.f;
+        for (int c = 0; c < d; ++c) acc = fmaf(Y[m * ld + c], Us[c * r + k], acc);
+        T[t] = acc;
+    }
+    __syncthreads();
     float* Bx = Bm + (long long)x * r * d;
     for (int t = tid; t < r * d; t += nt) {
         const int k = t / d, c2 = t % d;
         float acc = 0.f;
-        for (int c = 0; c < d; ++c) acc = fmaf(Us[c * r + k], Ax[(long long)c * d + c2], acc);
+        for (int m = 0; m < M; ++m) acc = fmaf(T[m * r + k], X[m * ld + c2], acc);
         Bx[t] = acc;
     }
     __syncthreads();
@@ -442,30 +527,45 @@ cudaError_t launch_fit(const float* R, const float* Xp, const float* w, float la
                        float* Rbar, float* A, float* U, float* Bm, float* c0, int32_t* rank,
                        int Hp, int g, int d, int M, int r, bool rbar_unprojected, int* status, cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
+    if (M > 64) return cudaErrorInvalidValue;
     const size_t smem = fit_smem_bytes(d, M, r);
-    cudaError_t e = cudaFuncSetAttribute(fit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fit_kernel<<<Hp, kFitThreads, smem, s>>>(R, Xp, w, lambda, obar, Rbar, A, U, Bm, c0, rank, g, d, M, r,
-                                             rbar_unprojected ? 1 : 0, status);
-    return cudaGetLastError();
+    auto run = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<Hp, kFitThreads, smem, s>>>(R, Xp, w, lambda, obar, Rbar, A, U, Bm, c0, rank, g, M, r,
+                                           rbar_unprojected ? 1 : 0, status);
+        return cudaGetLastError();
+    };
+    if (d == 64) return run(fit_kernel<64>);
+    if (d == 128) return run(fit_kernel<128>);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float* U,
                              const float* Bm, const float* c0, const float* Radd, bf16* O, int Hp, int g, int N,
-                             int d, int r, bool correct, cudaStream_t s) {
-    const int blocks = (N + 8 * 16 - 1) / (8 * 16);   // 16 rows per warp (4 iterations of 4)
-    dim3 grid(blocks, Hp);
+                             int d, int r, bool correct, int num_sms, cudaStream_t s) {
     const int cf = correct ? 1 : 0;
+    // persistent CTAs (one full wave): each stages Bm and U^T once for thousands of rows
+    auto run = [&](auto kern) -> cudaError_t {
+        int occ = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0);
+        if (e != cudaSuccess) return e;
+        if (occ < 1) occ = 1;
+        int per = occ * num_sms / Hp;
+        const int maxb = (N + 8 * 4 - 1) / (8 * 4);    // 8 warps x 4 rows per iteration
+        if (per > maxb) per = maxb;
+        if (per < 1) per = 1;
+        kern<<<dim3(per, Hp), 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
+        return cudaGetLastError();
+    };
     if (r <= 16) {
-        if (d == 64) writeback_kernel<64, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
-        else if (d == 128) writeback_kernel<128, 16><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
-        else return cudaErrorInvalidValue;
+        if (d == 64) return run(writeback_kernel<64, 16>);
+        if (d == 128) return run(writeback_kernel<128, 16>);
     } else {
-        if (d == 64) writeback_kernel<64, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
-        else if (d == 128) writeback_kernel<128, 32><<<grid, 256, 0, s>>>(Osp, qperm, U, Bm, c0, Radd, O, g, N, r, cf);
-        else return cudaErrorInvalidValue;
+        if (d == 64) return run(writeback_kernel<64, 32>);
+        if (d == 128) return run(writeback_kernel<128, 32>);
     }
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_writeback_ridge(const bf16* Osp, const int32_t* qperm, const float* A, const float* obar,

@@ -153,7 +153,7 @@ cudaError_t launch_fit(const float* R, const float* Xp, const float* w, float la
 // O = Osp + U (c0 + Bm Osp) (+ Radd [Hp][d] when non-null), scattered to the original order.
 cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float* U,
                              const float* Bm, const float* c0, const float* Radd, bf16* O, int Hp, int g, int N,
-                             int d, int r, bool correct, cudaStream_t s);
+                             int d, int r, bool correct, int num_sms, cudaStream_t s);
 // O = Osp + Rbar + A (Osp - obar) (ridge correction without the projection).
 cudaError_t launch_writeback_ridge(const bf16* Osp, const int32_t* qperm, const float* A, const float* obar,
                                    const float* Rbar, bf16* O, int Hp, int g, int N, int d, int num_sms,

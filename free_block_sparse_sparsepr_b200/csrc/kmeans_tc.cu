@@ -380,6 +380,7 @@ __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long
 // to the lowest group. Corrects the label and the count of rows that moved.
 constexpr int kFixThreads = 512;
 constexpr int kFixSplit = 4;   // blocks per assignment CTA's region
+constexpr int kFixLd = kMaxG + 1;
 template <int DP>
 __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __restrict__ fix,
                                                                const int* __restrict__ fix_count,
@@ -392,11 +393,13 @@ __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __res
     if (done && done[z]) return;
     const int cta = z * gridDim.x + blockIdx.x;
     const int cnt = fix_count[cta];
-    if (cnt == 0) return;
+    if (blockIdx.z * (kFixThreads / 32) >= cnt) return;     // no flagged row for this block
     extern __shared__ float fsm[];
-    float* sC = fsm;                          // [DP][kMaxG], k-major
-    float* sCC = fsm + DP * kMaxG;            // [kMaxG]
-    for (int t = threadIdx.x; t < G * DP; t += blockDim.x) sC[(t % DP) * kMaxG + t / DP] = C[(long long)z * G * DP + t];
+    // k-major centroids with a padded row (kFixLd = kMaxG + 1 floats): the transposing stores
+    // and the per-lane column reads of the fp64 pass both hit distinct banks
+    float* sC = fsm;                          // [DP][kFixLd]
+    float* sCC = fsm + DP * kFixLd;           // [kMaxG]
+    for (int t = threadIdx.x; t < G * DP; t += blockDim.x) sC[(t % DP) * kFixLd + t / DP] = C[(long long)z * G * DP + t];
     for (int t = threadIdx.x; t < kMaxG; t += blockDim.x) sCC[t] = t < G ? cc[(long long)z * G32 + t] : 0.f;
     __syncthreads();
     float cmax2 = 0.f;
@@ -425,8 +428,8 @@ __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __res
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int k = 0; k < DP; k += 2) {
-                a0 = fmaf(x[k], sC[k * kMaxG + g], a0);
-                a1 = fmaf(x[k + 1], sC[(k + 1) * kMaxG + g], a1);
+                a0 = fmaf(x[k], sC[k * kFixLd + g], a0);
+                a1 = fmaf(x[k + 1], sC[(k + 1) * kFixLd + g], a1);
             }
             const float d = g < G ? fmaf(-2.f, a0 + a1, xx + sCC[g]) : INFINITY;
             dg[j] = d;
@@ -445,8 +448,8 @@ __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __res
             while (m) {
                 const int g = 32 * j + __ffs(m) - 1;
                 m &= m - 1;
-                const double ca = lane < DP ? (double)sC[lane * kMaxG + g] : 0.0;
-                const double cb = lane + 32 < DP ? (double)sC[(lane + 32) * kMaxG + g] : 0.0;
+                const double ca = lane < DP ? (double)sC[lane * kFixLd + g] : 0.0;
+                const double cb = lane + 32 < DP ? (double)sC[(lane + 32) * kFixLd + g] : 0.0;
                 const double xc = warp_sum_d(xa * ca + xb * cb);
                 const double ccd = warp_sum_d(ca * ca + cb * cb);
                 const float d = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
@@ -548,7 +551,7 @@ cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* 
     int per, cap;
     km_grid(P, n, num_sms, &per, &cap);
     const int G32 = (G + 31) / 32 * 32;
-    const size_t smem = ((size_t)DP * kMaxG + kMaxG) * sizeof(float);
+    const size_t smem = ((size_t)DP * kFixLd + kMaxG) * sizeof(float);
     const dim3 grid(per, P, kFixSplit);
 #define SPR_FIXUP(DPV)                                                                                               \
     case DPV: {                                                                                                      \

@@ -118,6 +118,21 @@ def test_handed_in_partition_and_route(name):
                 if len(s) > w.r and s[w.r - 1] > 1.2 * s[w.r]:       # projector well defined
                     Ug = fv["U"][x].cpu().numpy().astype(np.float64)
                     assert np.abs(Ug @ Ug.T - f.U @ f.U.T).max() < 5e-2
+                # the fit on the GPU's own probe rows, against the oracle's closed forms in fp64:
+                # the ridge map A, Bm = U^T A with the GPU's U, and the residual subspace
+                Xg = fv["Osp"][x].cpu().numpy().astype(np.float64)
+                Rg = fv["R"][x].cpu().numpy().astype(np.float64)
+                wz = pt["weights"][b * w.Hkv + hq // w.g].cpu().numpy().astype(np.float64)
+                A_ref, xb_ref, yb_ref = oracle.ridge_fit(Xg, Rg, wz, w.lam)
+                scale = max(1e-3, np.abs(A_ref).max())
+                assert np.abs(fv["A"][x].cpu().numpy() - A_ref).max() <= 2e-3 * scale, "ridge map"
+                assert np.abs(fv["obar"][x].cpu().numpy() - xb_ref).max() <= 1e-5 * max(1.0, np.abs(xb_ref).max())
+                Ug = fv["U"][x].cpu().numpy().astype(np.float64)
+                Bm_ref = Ug.T @ A_ref
+                assert np.abs(fv["Bm"][x].cpu().numpy() - Bm_ref).max() <= 2e-3 * scale, "Bm"
+                U_ref, s_ref = oracle.residual_subspace(Rg, wz, w.r)
+                if len(s_ref) > w.r and s_ref[w.r - 1] > 1.2 * s_ref[w.r]:
+                    assert np.abs(Ug @ Ug.T - U_ref @ U_ref.T).max() < 1e-3, "residual subspace"
         # (7) correction and write-back
         O = torch.empty_like(q)
         h.writeback(part, Osp, fit, O)
