@@ -52,7 +52,8 @@ constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kStages, kBarEK = kBarV + kS
               kBarS = kBarEV + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2,
               kNumBars = kBarMma + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;          // tmem base (u32), abort flag (int)
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;          // + slack to align the base to 1024
+constexpr int kOffML = kOffMisc + 16;                      // split mode: tile 1's running max and sum [2][128]
+constexpr int kSmemBytes = kOffML + 2 * kBM * 4 + 1024;   // + slack to align the base to 1024
 
 enum { kModeSparse = 0, kModeDense = 1 };
 
@@ -197,6 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         ntk = (p.N + kBN - 1) / kBN;
     }
     const bool two = qn1 > 0;
+    // split mode: a lone query tile with two or more key tiles. Both softmax warpgroups take
+    // the same rows, warpgroup t the key tiles j with j % 2 == t, and warpgroup 0 merges the two
+    // partial softmax states at the end, so the tensor core still alternates between two S tiles.
+    const bool split = !two && ntk >= 2;
 
     // ---- set-up: barriers (thread 0), TMEM (warp 9)
     if (threadIdx.x == 0) {
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         bool ok = __all_sync(kFull, tc::mbar_wait(bar(kBarQ), 0, abort_flag));
         auto issue_S = [&](int t, int j) {
             const uint32_t kb = sK + (j % kStages) * 2 * kRegion;
-            const uint32_t qb = sQ + t * 2 * kRegion;
+            const uint32_t qb = sQ + (split ? 0 : t) * 2 * kRegion;
 #pragma unroll
             for (int k = 0; k < kD / 16; ++k) {
                 const uint32_t off = (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
@@ -286,6 +291,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             tc::commit(bar(kBarS + t));
         };
         int j = 0;
+        if (split) {
+            // S_0(0) and S_1(1) first; then per key tile j (softmax t = j % 2): PV_t(j) and S_t(j + 2)
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = __all_sync(kFull, tc::mbar_wait(bar(kBarK + t), 0, abort_flag));
+                if (!ok) break;
+                tc::fence_after_sync();
+                if (lane == 0) {
+                    issue_S(t, t);
+                    tc::commit(bar(kBarEK + t));
+                }
+                __syncwarp();
+            }
+            for (; ok && j < ntk; ++j) {
+                const int t = j & 1, s = j % kStages;
+                const bool nh = j + 2 < ntk;
+                if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kStages) & 1, abort_flag))) break;
+                if (nh && !__all_sync(kFull, tc::mbar_wait(bar(kBarK + ((j + 2) % kStages)), ((j + 2) / kStages) & 1,
+                                                          abort_flag)))
+                    break;
+                if (!__all_sync(kFull, tc::mbar_wait(bar(kBarP + t), (j >> 1) & 1, abort_flag))) break;
+                tc::fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t vb = sV + s * 2 * kRegion;
+                    const uint32_t pt = tmem + (uint32_t)(t * 128);
+#pragma unroll
+                    for (int k = 0; k < kBN / 16; ++k)
+                        tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
+                                       tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
+                                       (j >= 2 || k > 0) ? 1u : 0u);
+                    tc::commit(bar(kBarEV + s));
+                    if (nh) {
+                        issue_S(t, j + 2);
+                        tc::commit(bar(kBarEK + (j + 2) % kStages));
+                    } else {
+                        tc::commit(bar(kBarO + t));
+                    }
+                }
+                __syncwarp();
+            }
+            have = false;
+        }
         if (ok && have) {
             ok = __all_sync(kFull, tc::mbar_wait(bar(kBarK), 0, abort_flag));
             if (ok) {
@@ -339,19 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // ================= softmax warpgroup t: thread r <-> row r of tile t <-> TMEM lane r
         const int t = warp >> 2;
         const int r = threadIdx.x & 127;
-        const int qn = t == 0 ? qn0 : qn1;
+        const int qn = (t == 0 || split) ? qn0 : qn1;
+        float* sML = reinterpret_cast<float*>(sbase + kOffML);   // split mode: [0][r] max, [1][r] sum of tile 1
         if (qn > 0) {
             const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
             const uint32_t tS = tmem + (uint32_t)(t * 128) + lane_off;
             const uint32_t tO = tmem + 256 + (uint32_t)(t * 128) + lane_off;
             const float c_log2 = p.scale_log2;
+            // this warpgroup's key tiles: all of them, or (split mode) every other one from t
+            const int kj0 = split ? t : 0, kjs = split ? 2 : 1;
+            const int nloc = split ? (ntk - t + 1) / 2 : ntk;
             int j = 0;
             float m_run = -INFINITY, l_run = 0.f;
             bool ok = true;
-            int lim_next = ntk > 0 ? key_tile(p, MODE, klist, 0).y : 0;
-            for (; j < ntk; ++j) {
+            int lim_next = nloc > 0 ? key_tile(p, MODE, klist, kj0).y : 0;
+            for (; j < nloc; ++j) {
                 const int lim = lim_next;
-                if (j + 1 < ntk) lim_next = key_tile(p, MODE, klist, j + 1).y;   // prefetch
+                if (j + 1 < nloc) lim_next = key_tile(p, MODE, klist, kj0 + (j + 1) * kjs).y;   // prefetch
                 // every TMEM access below is warp-collective: decisions are made warp-uniform
                 const bool got_s = tc::mbar_wait(bar(kBarS + t), j & 1, abort_flag);
                 if (!__all_sync(kFull, got_s)) { ok = false; break; }
@@ -442,6 +492,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tc::mbar_arrive(bar(kBarP + t));
             }
             // epilogue: O / l, bf16 row store, lse
+            if (split) {
+                // tile 1 hands its running max and sum to warpgroup 0, which reads both O_0 and O_1
+                // from TMEM (the same lanes) and writes the merged rows
+                if (t == 1) {
+                    sML[r] = m_run;
+                    sML[kBM + r] = l_run;
+                }
+                tc::named_bar_sync(1, 2 * kBM);
+                if (t == 0) {
+                    bool got = false;
+                    if (ok) got = tc::mbar_wait(bar(kBarO), 0, abort_flag) && tc::mbar_wait(bar(kBarO + 1), 0, abort_flag);
+                    if (__all_sync(kFull, got)) {
+                        tc::fence_after_sync();
+                        const float m1 = sML[r], l1 = sML[kBM + r];
+                        const float mm = fmaxf(m_run, m1);
+                        const float f0 = mm == -INFINITY ? 0.f : exp2f(m_run - mm);
+                        const float f1 = mm == -INFINITY ? 0.f : exp2f(m1 - mm);
+                        const float l = l_run * f0 + l1 * f1;
+                        const float inv = l > 0.f ? 1.f / l : 0.f;
+                        const float a0 = f0 * inv, a1 = f1 * inv;
+                        bf16* orow = p.O + ((long long)x * p.N + qlo + r) * kD;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t o0[32], o1[32];
+                            tc::tmem_ld32(tO + 32 * c, o0);
+                            tc::tmem_ld32(tO + 128 + 32 * c, o1);
+                            tc::tmem_wait_ld();
+                            tc::regs_after_wait(o0);
+                            tc::regs_after_wait(o1);
+                            if (r < qn) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    uint32_t w[4];
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int i0 = 8 * q + 2 * e;
+                                        __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                                            fmaf(__uint_as_float(o0[i0]), a0, __uint_as_float(o1[i0]) * a1),
+                                            fmaf(__uint_as_float(o0[i0 + 1]), a0, __uint_as_float(o1[i0 + 1]) * a1));
+                                        w[e] = *reinterpret_cast<uint32_t*>(&b2);
+                                    }
+                                    *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+                                }
+                            }
+                        }
+                        if (r < qn && p.lse) p.lse[(long long)x * p.N + qlo + r] = (mm + log2f(l)) * kLn2;
+                    }
+                }
+            } else {
             bool got_last = false;
             if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO + t), 0, abort_flag);
             if (j > 0 && __all_sync(kFull, got_last)) {
@@ -474,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 bf16* orow = p.O + ((long long)x * p.N + qlo + t * kBM + r) * kD;
                 for (int c = 0; c < kD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
                 if (p.lse) p.lse[(long long)x * p.N + qlo + t * kBM + r] = -INFINITY;
+            }
             }
         }
     }
