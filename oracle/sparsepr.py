@@ -53,6 +53,7 @@ import numpy as np
 __all__ = [
     "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS",
     "sample_rows", "splitmix64", "rademacher_projection", "response_features", "top_mass_fraction",
+    "top_mass_count", "top_mass_set", "SHARED_ROWS", "shared_rows", "shared_support",
     "sq_dists_f32", "kmeans_assign", "kmeans_update", "kmeans", "group_means",
     "stable_group_order", "query_coordinates", "query_logits", "cell_scores", "select_cells",
     "route_csr", "probe_rows", "coverage_weights", "sparse_attention", "dense_attention_rows",
@@ -160,6 +161,61 @@ def top_mass_fraction(z_row: np.ndarray, mass: float = 0.9) -> float:
     c = np.cumsum(p)
     k = int(np.searchsorted(c, mass * c[-1], side="left")) + 1
     return min(k, len(p)) / len(p)
+
+
+def top_mass_count(z_row: np.ndarray, mass: float = 0.9) -> int:
+    """The key count behind top_mass_fraction: keys taken in descending probability until their
+    softmax mass first reaches `mass` of the total ([support])."""
+    z = np.asarray(z_row, dtype=np.float64)
+    p = np.exp(z - z.max())
+    c = np.cumsum(np.sort(p)[::-1])
+    k = int(np.searchsorted(c, mass * c[-1], side="left")) + 1
+    return min(k, len(p))
+
+
+def top_mass_set(z_row: np.ndarray, mass: float = 0.9) -> np.ndarray:
+    """Boolean mask of a row's 90%-mass support: the keys whose logit is at least the k-th
+    largest, k = top_mass_count (reading: keys tied with the k-th largest logit all count)."""
+    z = np.asarray(z_row, dtype=np.float64)
+    k = top_mass_count(z, mass)
+    tau = np.sort(z)[::-1][k - 1]
+    return z >= tau
+
+
+SHARED_ROWS = 8     # queries that share one route in the shared-support diagnostic
+
+
+def shared_rows(lo: int, hi: int, R: int = SHARED_ROWS) -> np.ndarray:
+    """Group-major positions of the rows of a query group [lo, hi) that stand for it in the
+    shared-support diagnostic: min(R, size) systematic positions lo + floor((m + 1/2) size / R')."""
+    size = hi - lo
+    Rp = min(R, size)
+    m = np.arange(Rp, dtype=np.int64)
+    return lo + ((2 * m + 1) * size) // (2 * Rp)
+
+
+def shared_support(Qg: np.ndarray, Kh: np.ndarray, qperm: np.ndarray, qoff: np.ndarray,
+                   R: int = SHARED_ROWS, mass: float = 0.9):
+    """Shared-route support ([support]): a route serves every query of its group, so it must
+    cover the union of their 90%-mass key sets. For each query group a, the rows of shared_rows
+    (row m in query head m mod g of the KV group; Qg [g, N, d], Kh [N, d] fp64) each get their
+    90%-mass set over all N keys (top_mass_set of q.k / sqrt(d)); returns the union's size / N
+    per group [Gq] (0 for an empty group) and each row's own count / N [Gq, R] (0 past R')."""
+    g, N, d = Qg.shape
+    Gq = len(qoff) - 1
+    union = np.zeros(Gq, dtype=np.float64)
+    single = np.zeros((Gq, R), dtype=np.float64)
+    for a in range(Gq):
+        lo, hi = int(qoff[a]), int(qoff[a + 1])
+        if hi <= lo:
+            continue
+        mask = np.zeros(N, dtype=bool)
+        for m, pos in enumerate(shared_rows(lo, hi, R)):
+            z = (Qg[m % g, int(qperm[pos])] @ Kh.T) / math.sqrt(d)
+            mask |= top_mass_set(z, mass)
+            single[a, m] = top_mass_count(z, mass) / N
+        union[a] = mask.sum() / N
+    return union, single
 
 
 # --------------------------------------------------------------------------------------
