@@ -373,14 +373,15 @@ __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long
     if (lane == 0) cc[(long long)z * G32 + g] = g < G ? ss : kFar;
 }
 
-// Exact pass over the flagged rows: kFixSplit blocks per assignment CTA (each with the
-// centroids staged in shared memory k-major), one warp per row, the row in registers. Candidates are the groups whose fp32
+// Exact pass over the flagged rows: kFixSplit blocks per assignment CTA's region, one thread
+// per row, the row in registers and the centroids staged row-major in shared memory (every
+// centroid read is a broadcast to the warp). Candidates are the groups whose fp32
 // ||x||^2 - 2 x.c + ||c||^2 (error below 2^-19 (||x||^2 + ||c||^2)) is within 1e-4 (d + ||x||^2
-// + max ||c||^2) of the smallest; each gets the fp32 value of its fp64 distance, argmin with ties
-// to the lowest group. Corrects the label and the count of rows that moved.
-constexpr int kFixThreads = 512;
-constexpr int kFixSplit = 4;   // blocks per assignment CTA's region
-constexpr int kFixLd = kMaxG + 1;
+// + max ||c||^2) of the smallest: the four smallest are kept while scanning, and only a row with
+// more candidates than that scans again. Each candidate gets the fp32 value of its fp64
+// distance, argmin with ties to the lowest group. Corrects the label and the moved count.
+constexpr int kFixThreads = 128;
+constexpr int kFixSplit = 2;   // blocks per assignment CTA's region
 template <int DP>
 __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __restrict__ fix,
                                                                const int* __restrict__ fix_count,
@@ -393,76 +394,94 @@ __global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __res
     if (done && done[z]) return;
     const int cta = z * gridDim.x + blockIdx.x;
     const int cnt = fix_count[cta];
-    if (blockIdx.z * (kFixThreads / 32) >= cnt) return;     // no flagged row for this block
-    extern __shared__ float fsm[];
-    // k-major centroids with a padded row (kFixLd = kMaxG + 1 floats): the transposing stores
-    // and the per-lane column reads of the fp64 pass both hit distinct banks
-    float* sC = fsm;                          // [DP][kFixLd]
-    float* sCC = fsm + DP * kFixLd;           // [kMaxG]
-    for (int t = threadIdx.x; t < G * DP; t += blockDim.x) sC[(t % DP) * kFixLd + t / DP] = C[(long long)z * G * DP + t];
-    for (int t = threadIdx.x; t < kMaxG; t += blockDim.x) sCC[t] = t < G ? cc[(long long)z * G32 + t] : 0.f;
+    if (blockIdx.z * kFixThreads >= cnt) return;            // no flagged row for this block
+    extern __shared__ __align__(16) float fsm[];
+    float* sC = fsm;                          // [G][DP]
+    float* sCC = fsm + (size_t)G * DP;        // [G]
+    {
+        const float4* src = reinterpret_cast<const float4*>(C + (long long)z * G * DP);
+        float4* dst = reinterpret_cast<float4*>(sC);
+        for (int t = threadIdx.x; t < G * DP / 4; t += kFixThreads) dst[t] = __ldg(src + t);
+        for (int t = threadIdx.x; t < G; t += kFixThreads) sCC[t] = cc[(long long)z * G32 + t];
+    }
     __syncthreads();
     float cmax2 = 0.f;
     for (int g = 0; g < G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
     const int4* reg = fix + (long long)cta * fix_cap;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // blockIdx.z of gridDim.z blocks share the region, each warp taking every (warps * blocks)th row
-    for (int w = blockIdx.z * (kFixThreads / 32) + warp; w < cnt; w += gridDim.z * (kFixThreads / 32)) {
+    for (int w = blockIdx.z * kFixThreads + threadIdx.x; w < cnt; w += gridDim.z * kFixThreads) {
         const int4 h = reg[w];
         const long long o = h.x;
-        const float* xr = X + o * DP;
+        const float4* xr4 = reinterpret_cast<const float4*>(X + o * DP);
         float x[DP];
 #pragma unroll
-        for (int k = 0; k < DP; k += 4) {
-            const float4 q = __ldg(reinterpret_cast<const float4*>(xr + k));
-            x[k] = q.x; x[k + 1] = q.y; x[k + 2] = q.z; x[k + 3] = q.w;
+        for (int k = 0; k < DP / 4; ++k) {
+            const float4 q = __ldg(xr4 + k);
+            x[4 * k] = q.x; x[4 * k + 1] = q.y; x[4 * k + 2] = q.z; x[4 * k + 3] = q.w;
         }
         float xx = 0.f;
 #pragma unroll
         for (int k = 0; k < DP; ++k) xx = fmaf(x[k], x[k], xx);
-        float dg[kMaxG / 32];
-        float dmin = INFINITY;
+        auto dist32 = [&](int g) -> float {
+            const float4* c4 = reinterpret_cast<const float4*>(sC + g * DP);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int j = 0; j < kMaxG / 32; ++j) {
-            const int g = lane + 32 * j;
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int k = 0; k < DP; k += 2) {
-                a0 = fmaf(x[k], sC[k * kFixLd + g], a0);
-                a1 = fmaf(x[k + 1], sC[(k + 1) * kFixLd + g], a1);
+            for (int k = 0; k < DP / 4; ++k) {
+                const float4 c = c4[k];
+                a0 = fmaf(x[4 * k], c.x, a0);
+                a1 = fmaf(x[4 * k + 1], c.y, a1);
+                a2 = fmaf(x[4 * k + 2], c.z, a2);
+                a3 = fmaf(x[4 * k + 3], c.w, a3);
             }
-            const float d = g < G ? fmaf(-2.f, a0 + a1, xx + sCC[g]) : INFINITY;
-            dg[j] = d;
-            dmin = fminf(dmin, d);
+            return fmaf(-2.f, (a0 + a1) + (a2 + a3), xx + sCC[g]);
+        };
+        // the four smallest fp32 distances (ascending) and their groups
+        float t0 = INFINITY, t1 = INFINITY, t2 = INFINITY, t3 = INFINITY;
+        int i0 = 0, i1 = 0, i2 = 0, i3 = 0;
+#pragma unroll 1
+        for (int g = 0; g < G; ++g) {
+            const float d = dist32(g);
+            if (d < t3) {
+                if (d < t1) {
+                    t3 = t2; i3 = i2; t2 = t1; i2 = i1;
+                    if (d < t0) { t1 = t0; i1 = i0; t0 = d; i0 = g; }
+                    else { t1 = d; i1 = g; }
+                } else if (d < t2) { t3 = t2; i3 = i2; t2 = d; i2 = g; }
+                else { t3 = d; i3 = g; }
+            }
         }
-        dmin = warp_min(dmin);
-        const float thr = dmin + 1e-4f * (fabsf(dmin) + xx + cmax2);
-        const double xa = lane < DP ? (double)xr[lane] : 0.0;
-        const double xb = lane + 32 < DP ? (double)xr[lane + 32] : 0.0;
-        const double xxd = warp_sum_d(xa * xa + xb * xb);
+        const float thr = t0 + 1e-4f * (fabsf(t0) + xx + cmax2);
+        double xxd = 0.0;
+#pragma unroll
+        for (int k = 0; k < DP; ++k) xxd = fma((double)x[k], (double)x[k], xxd);
         float best = INFINITY;
         int bg = h.z;
+        auto exact = [&](int g) {
+            const float* cg = sC + g * DP;
+            double xc = 0.0, ccd = 0.0;
 #pragma unroll
-        for (int j = 0; j < kMaxG / 32; ++j) {
-            uint32_t m = __ballot_sync(kFull, dg[j] <= thr);
-            while (m) {
-                const int g = 32 * j + __ffs(m) - 1;
-                m &= m - 1;
-                const double ca = lane < DP ? (double)sC[lane * kFixLd + g] : 0.0;
-                const double cb = lane + 32 < DP ? (double)sC[(lane + 32) * kFixLd + g] : 0.0;
-                const double xc = warp_sum_d(xa * ca + xb * cb);
-                const double ccd = warp_sum_d(ca * ca + cb * cb);
-                const float d = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
-                if (d < best) { best = d; bg = g; }
+            for (int k = 0; k < DP; ++k) {
+                const double c = (double)cg[k];
+                xc = fma((double)x[k], c, xc);
+                ccd = fma(c, c, ccd);
             }
+            const float d = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
+            if (d < best || (d == best && g < bg)) { best = d; bg = g; }
+        };
+        // candidates: the (at most three) kept groups within thr, or, when the fourth smallest is
+        // within thr too, every group within thr (found by scanning again)
+        const bool all = t3 <= thr;
+        const int ncand = all ? G : 1 + (t1 <= thr ? 1 : 0) + (t2 <= thr ? 1 : 0);
+#pragma unroll 1
+        for (int q = 0; q < ncand; ++q) {
+            const int g = all ? q : (q == 0 ? i0 : (q == 1 ? i1 : i2));
+            if (all && !(dist32(g) <= thr)) continue;
+            exact(g);
         }
-        if (lane == 0) {
-            labels[o] = bg;
-            const int prev = h.y;
-            if (prev >= 0) {
-                const int dmoved = (prev != bg ? 1 : 0) - (prev != h.z ? 1 : 0);
-                if (dmoved) atomicAdd(&changed[z], dmoved);
-            }
+        labels[o] = bg;
+        const int prev = h.y;
+        if (prev >= 0) {
+            const int dmoved = (prev != bg ? 1 : 0) - (prev != h.z ? 1 : 0);
+            if (dmoved) atomicAdd(&changed[z], dmoved);
         }
     }
 }
@@ -551,7 +570,7 @@ cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* 
     int per, cap;
     km_grid(P, n, num_sms, &per, &cap);
     const int G32 = (G + 31) / 32 * 32;
-    const size_t smem = ((size_t)DP * kFixLd + kMaxG) * sizeof(float);
+    const size_t smem = ((size_t)G * DP + G) * sizeof(float);
     const dim3 grid(per, P, kFixSplit);
 #define SPR_FIXUP(DPV)                                                                                               \
     case DPV: {                                                                                                      \
