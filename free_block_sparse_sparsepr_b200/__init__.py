@@ -61,6 +61,8 @@ class SparsePRError(RuntimeError):
         self.code = code
 
 
+SHARED_ROWS = 8   # rows per query group in the shared-support diagnostic (SPARSEPR_SHARED_ROWS)
+
 _lib = None
 
 
@@ -100,6 +102,9 @@ def load_library() -> ctypes.CDLL:
         "sparsepr_device_status": (st, [H, ctypes.POINTER(ctypes.c_int)]),
         "sparsepr_last_launch_count": (st, [H, ctypes.POINTER(ctypes.c_int)]),
         "sparsepr_set_stage_events": (st, [H, ctypes.c_void_p]),
+        "sparsepr_shared_support_workspace": (st, [H, ctypes.POINTER(ctypes.c_size_t),
+                                                   ctypes.POINTER(ctypes.c_size_t)]),
+        "sparsepr_shared_support": (st, [H, _p, _p, ctypes.POINTER(Partition), _p, _p, _p, ctypes.c_size_t, _p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -227,6 +232,25 @@ class SparsePR:
                                                                  ctypes.byref(part), _ptr(Osp), ctypes.byref(out),
                                                                  _stream(stream)))
         return out
+
+    def shared_support(self, Q, K, part: Partition, max_workspace_bytes: int = 8 << 30, stream=None):
+        """Shared-route support diagnostic: (row_frac [B*Hkv, Gq, SHARED_ROWS], union_frac
+        [B*Hkv, Gq]) as fp32 device tensors; the workspace (device memory through torch) holds
+        as many KV heads' logits per pass as max_workspace_bytes allows (at least one)."""
+        import torch
+
+        lo, hi = ctypes.c_size_t(), ctypes.c_size_t()
+        _check("sparsepr_shared_support_workspace",
+               self.lib.sparsepr_shared_support_workspace(self.h, ctypes.byref(lo), ctypes.byref(hi)))
+        nbytes = max(lo.value, min(hi.value, max_workspace_bytes))
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        P = self.cfg.B * self.cfg.Hkv
+        row_frac = torch.empty((P, self.cfg.Gq, SHARED_ROWS), dtype=torch.float32, device="cuda")
+        union_frac = torch.empty((P, self.cfg.Gq), dtype=torch.float32, device="cuda")
+        _check("sparsepr_shared_support",
+               self.lib.sparsepr_shared_support(self.h, _ptr(Q), _ptr(K), ctypes.byref(part), _ptr(row_frac),
+                                                _ptr(union_frac), _ptr(ws), nbytes, _stream(stream)))
+        return row_frac, union_frac
 
     def writeback(self, part: Partition, Osp, fit: Fit | None, O, stream=None):
         _check("sparsepr_writeback", self.lib.sparsepr_writeback(self.h, ctypes.byref(part), _ptr(Osp),

@@ -473,6 +473,58 @@ sparsepr_status sparsepr_partition(sparsepr_handle h, const void* Q, const void*
     return SPARSEPR_OK;
 }
 
+namespace {
+constexpr int kShared = SPARSEPR_SHARED_ROWS;
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+size_t shared_rows_bytes(sparsepr_handle h) {
+    return align256((size_t)h->P * h->cfg.Gq * kShared * h->cfg.d * sizeof(bf16));
+}
+size_t shared_head_bytes(sparsepr_handle h) {
+    return align256((size_t)h->cfg.Gq * kShared * h->cfg.N * sizeof(float));
+}
+}  // namespace
+
+sparsepr_status sparsepr_shared_support_workspace(sparsepr_handle h, size_t* min_bytes, size_t* all_bytes) {
+    if (!h || (!min_bytes && !all_bytes)) return SPARSEPR_ERR_INVALID_ARG;
+    if (min_bytes) *min_bytes = shared_rows_bytes(h) + shared_head_bytes(h);
+    if (all_bytes) *all_bytes = shared_rows_bytes(h) + (size_t)h->P * shared_head_bytes(h);
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_shared_support(sparsepr_handle h, const void* Q, const void* K,
+                                        const sparsepr_partition_t* part, float* row_frac, float* union_frac,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!h || !aligned16(Q) || !aligned16(K) || !row_frac || !union_frac || !aligned16(workspace))
+        return SPARSEPR_ERR_INVALID_ARG;
+    if (!part || !part->qperm || !part->qoff) return SPARSEPR_ERR_INVALID_ARG;
+    const sparsepr_config& c = h->cfg;
+    const size_t rows_b = shared_rows_bytes(h), head_b = shared_head_bytes(h);
+    if (workspace_bytes < rows_b + head_b) return SPARSEPR_ERR_WORKSPACE;
+    int hc = (int)((workspace_bytes - rows_b) / head_b);
+    if (hc > h->P) hc = h->P;
+    h->launches = 0;
+    cudaStream_t s = as_stream(stream);
+    bf16* Qsh = static_cast<bf16*>(workspace);
+    float* Z = reinterpret_cast<float*>(static_cast<char*>(workspace) + rows_b);
+    const long long ldz = (long long)(head_b / sizeof(float)) / ((long long)c.Gq * kShared);
+    SPR_TRY(spr::launch_shared_rows(static_cast<const bf16*>(Q), part->qperm, part->qoff, Qsh, h->P, h->g, c.N, c.d,
+                                    c.Gq, s));
+    for (int z0 = 0; z0 < h->P; z0 += hc) {
+        const int nz = h->P - z0 < hc ? h->P - z0 : hc;
+        spr::GemmArgs a;
+        memset(&a, 0, sizeof(a));
+        a.A1 = Qsh + (size_t)z0 * c.Gq * kShared * c.d; a.sA = (long long)c.Gq * kShared * c.d; a.lda = c.d;
+        a.B1 = static_cast<const bf16*>(K) + (size_t)z0 * c.N * c.d; a.sB = (long long)c.N * c.d; a.ldb = c.d;
+        a.bdiv = 1;
+        a.C = Z; a.sC = (long long)c.Gq * kShared * ldz; a.ldc = (int)ldz;
+        a.M = c.Gq * kShared; a.N = c.N; a.K = c.d; a.batch = nz;
+        a.alpha = (float)(1.0 / sqrt((double)c.d));
+        SPR_TRY(spr::launch_gemm_bf16(a, s));
+        SPR_TRY(spr::launch_shared_support(Z, ldz, part->qoff, row_frac, union_frac, z0, nz, c.N, c.Gq, s));
+    }
+    return SPARSEPR_OK;
+}
+
 sparsepr_status sparsepr_route(sparsepr_handle h, const void* Q, const sparsepr_partition_t* part,
                                sparsepr_route_t* out, void* stream) {
     if (!h || !aligned16(Q) || !out) return SPARSEPR_ERR_INVALID_ARG;

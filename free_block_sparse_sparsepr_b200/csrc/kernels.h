@@ -71,6 +71,13 @@ cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long coun
 // Support diagnostic: out[z][s] = (smallest k whose k largest exp(F[.][s] - max) hold 90% of the
 // row's softmax mass) / N, for s < S; F [P][N][DP] fp32 (DP a multiple of 8, S <= DP).
 cudaError_t launch_topmass(const float* F, float* out, int P, int N, int DP, int S, cudaStream_t s);
+// Shared-route support: Qsh [P][Gq][8][d] bf16 gathered rows (zero past R' of each group), then
+// for KV heads z0..z0+nz-1 the row-major logits Z [nz][Gq*8][ldz] give row_frac [P][Gq][8] and
+// union_frac [P][Gq].
+cudaError_t launch_shared_rows(const bf16* Q, const int32_t* qperm, const int32_t* qoff, bf16* Qsh, int P, int g,
+                               int N, int d, int Gq, cudaStream_t s);
+cudaError_t launch_shared_support(const float* Z, long long ldz, const int32_t* qoff, float* row_frac,
+                                  float* union_frac, int z0, int nz, int N, int Gq, cudaStream_t s);
 
 // ---------------------------------------------------------------- responses and coordinates
 // Qs[z][s][:] = Q[b][h*g + s%g][floor((s+1/2)N/S)][:] for s < S, zero rows up to DP.

@@ -285,6 +285,32 @@ sparsepr_status sparsepr_attention(sparsepr_handle h, const void* Q, const void*
 sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const void* K,
                                         const void* V, void* O, void* stream);
 
+/*
+ * Shared-route support diagnostic [support paragraph: a route shared by the
+ * queries of a group must cover the union of their supports]. For every query
+ * group a of every KV head z, up to SPARSEPR_SHARED_ROWS rows stand for the
+ * group: its group-major positions lo + floor((m + 1/2) size / R'),
+ * R' = min(SPARSEPR_SHARED_ROWS, size), row m taken in query head m mod (Hq/Hkv).
+ * Each row's logits against all N keys (q.k/sqrt(d), fp32) give its 90%-mass
+ * set (keys in descending logit until 90% of the softmax mass is reached; every
+ * key tied with the last one counts) and its count.
+ *   row_frac   [B*Hkv][Gq][SPARSEPR_SHARED_ROWS] fp32, device: each row's count / N
+ *              (0 past R')
+ *   union_frac [B*Hkv][Gq] fp32, device: |union of the R' sets| / N (0 for an
+ *              empty group)
+ *   workspace  caller-owned device memory of at least the `min_bytes` that
+ *              sparsepr_shared_support_workspace reports (16-byte aligned); more
+ *              (up to `all_bytes`) lets more KV heads run per pass.
+ * `part` may be handle-owned or handed in (only qperm and qoff are read).
+ * Not part of the attention call; it writes no handle state. Returns
+ * SPARSEPR_ERR_WORKSPACE when the workspace is too small.
+ */
+#define SPARSEPR_SHARED_ROWS 8
+sparsepr_status sparsepr_shared_support_workspace(sparsepr_handle h, size_t* min_bytes, size_t* all_bytes);
+sparsepr_status sparsepr_shared_support(sparsepr_handle h, const void* Q, const void* K,
+                                        const sparsepr_partition_t* part, float* row_frac, float* union_frac,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Dense softmax attention (scale 1/sqrt(d)) of every query over all keys: the baseline. */
 sparsepr_status sparsepr_dense_attn(sparsepr_handle h, const void* Q, const void* K, const void* V,
                                     void* O, void* stream);

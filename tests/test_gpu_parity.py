@@ -323,6 +323,37 @@ def test_support_diagnostic_matches_oracle(name):
 
 
 
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000", "ragged_gqa_n1500_g40"])
+def test_shared_support_matches_oracle(name):
+    """The shared-route support diagnostic ([support]) on the GPU's own partition against the
+    oracle's definition in fp64: each row's 90%-mass key count within max(2, 1e-3 N) keys (fp32
+    logits and mass sums move the crossing across near-equal weights), the union within that
+    per row; the result does not depend on how many KV heads share a workspace pass."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    P, g, R = w.B * w.Hkv, w.g, spr.SHARED_ROWS
+    with spr.SparsePR.from_workload(w) as h:
+        part = h.partition(q, k)
+        rf_all, uf_all = h.shared_support(q, k, part)
+        rf_one, uf_one = h.shared_support(q, k, part, max_workspace_bytes=0)   # one KV head per pass
+        torch.cuda.synchronize()
+        pv = {n: t.cpu().numpy() for n, t in h.partition_views(part).items()}
+    rf, uf = rf_all.cpu().numpy(), uf_all.cpu().numpy()
+    tol = max(2.0, 1e-3 * w.N)
+    assert np.abs(rf_one.cpu().numpy() - rf).max() * w.N <= tol
+    assert np.abs(uf_one.cpu().numpy() - uf).max() * w.N <= R * tol
+    for z in range(P):
+        b, hk = divmod(z, w.Hkv)
+        Qg = bf16_to_f64(q[b, hk * g:(hk + 1) * g])
+        Kh = bf16_to_f64(k[b, hk])
+        u_ref, s_ref = oracle.shared_support(Qg, Kh, pv["qperm"][z], pv["qoff"][z])
+        assert np.abs(rf[z] - s_ref).max() * w.N <= tol, (z, np.abs(rf[z] - s_ref).max() * w.N)
+        assert np.abs(uf[z] - u_ref).max() * w.N <= R * tol, (z, np.abs(uf[z] - u_ref).max() * w.N)
+        sizes = np.diff(pv["qoff"][z])
+        assert np.all(rf[z][np.arange(R)[None, :] >= np.minimum(sizes, R)[:, None]] == 0)
+        ok = sizes > 0
+        assert np.all(uf[z][ok] + 1e-6 >= rf[z][ok].max(axis=1))        # the union covers every row's set
+
+
 @pytest.mark.parametrize("flag", ["FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED"])
 @pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
 def test_ablation_corrections(name, flag):
