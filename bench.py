@@ -474,6 +474,64 @@ def run_stack(args):
     return 0
 
 
+def run_sharded(args):
+    """One call split by KV heads over the ranks (strong scaling): every rank draws the same
+    seeded inputs, runs its shard of heads, and the output is all-gathered over NCCL. Times the
+    sharded call alone and the call followed by the gather (CUDA events, max over ranks); value
+    is the whole call's dense-equivalent FLOPs over the slower of the two rank times."""
+    import torch
+    import torch.distributed as dist
+
+    from free_block_sparse_sparsepr_b200.sharding import ShardedSparsePR, head_range
+    from synthetic import get_workload, video_qkv_device
+
+    rank, world = dist_init("nccl" if torch.cuda.is_available() else "gloo")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = get_workload(args.workload)
+    Q, K, V = video_qkv_device(w, layer=0, locality=w.locality, device=str(dev))
+    sh = ShardedSparsePR(w.B, w.Hq, w.Hkv, w.N, w.d, Gk=w.Gk, Gq=w.Gq, block=w.block, rK=w.rK, rQ=w.rQ, M=w.M,
+                         r=w.r, kmeans_iters=w.kmeans_iters, lam=w.lam, rho_exec=w.rho, seed=w.seed)
+
+    def timed(fn, reps):
+        cur = torch.cuda.current_stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        a.record(cur)
+        for _ in range(reps):
+            fn()
+        b.record(cur)
+        torch.cuda.synchronize()
+        barrier()
+        return reduce_max(a.elapsed_time(b) / reps, dev)
+
+    for _ in range(max(3, args.warmup)):
+        sh.attention(Q, K, V, gather=world > 1)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = timed(lambda: sh.attention(Q, K, V), args.steps)
+    ms_gather = timed(lambda: sh.attention(Q, K, V, gather=True), args.steps) if world > 1 else ms
+    launches = sh.handle.last_launch_count() if sh.handle is not None else 0
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC + " (one call sharded by KV heads)",
+            "value": w.dense_equiv_flops() / (ms * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_with_gather": ms_gather,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (drawn on the GPU)",
+            "config": dict(workload_config(w, world), parallelism=f"heads{world}",
+                           heads_per_rank=[hi - lo for lo, hi in (head_range(w.B * w.Hkv, world, r)
+                                                                  for r in range(world))]),
+            "gpu_launches": launches, "clocks": clk.summary(),
+        }), flush=True)
+    sh.close()
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -486,6 +544,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--layers", type=int, default=1,
                     help="> 1: time a stack of this many calls as one CUDA graph (two streams)")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="split one call's KV heads over the ranks and all-gather O (strong scaling)")
     return ap.parse_args(argv)
 
 
@@ -495,6 +555,8 @@ def main(argv=None):
         return run_reference(args)
     if args.layers > 1:
         return run_stack(args)
+    if args.shard_heads:
+        return run_sharded(args)
     return run_ours(args)
 
 

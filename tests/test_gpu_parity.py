@@ -354,6 +354,27 @@ def test_shared_support_matches_oracle(name):
         assert np.all(uf[z][ok] + 1e-6 >= rf[z][ok].max(axis=1))        # the union covers every row's set
 
 
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
+def test_head_shards_reproduce_the_call(name):
+    """Head sharding: every step is per KV head, so running the KV heads in shards (each shard
+    its own handle, as each rank of a head-sharded group would) reproduces the unsharded call
+    bit for bit."""
+    from free_block_sparse_sparsepr_b200.sharding import ShardedSparsePR
+
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    kw = dict(Gk=w.Gk, Gq=w.Gq, block=w.block, rK=w.rK, rQ=w.rQ, M=w.M, r=w.r, kmeans_iters=w.kmeans_iters,
+              lam=w.lam, rho_exec=w.rho, seed=w.seed)
+    with spr.SparsePR.from_workload(w) as h:
+        O_full = h.attention(q, k, v).reshape(w.B * w.Hq, w.N, w.d)
+    world = min(3, w.B * w.Hkv)
+    parts = []
+    for rank in range(world):
+        with ShardedSparsePR(w.B, w.Hq, w.Hkv, w.N, w.d, world=world, rank=rank, **kw) as sh:
+            parts.append(sh.attention(q, k, v).clone())
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts), O_full)
+
+
 @pytest.mark.parametrize("flag", ["FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED"])
 @pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
 def test_ablation_corrections(name, flag):

@@ -72,3 +72,76 @@ def test_two_gloo_ranks():
     line = json.loads(o0.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _dense_heads(q, k, v):
+    """Plain softmax attention per query head (q [n*g, N, d], k, v [n, N, d]), fp64 on CPU."""
+    import torch
+
+    g = q.shape[0] // k.shape[0]
+    kk = k.repeat_interleave(g, dim=0)
+    vv = v.repeat_interleave(g, dim=0)
+    s = (q @ kk.transpose(1, 2)) / q.shape[-1] ** 0.5
+    return torch.softmax(s, dim=-1) @ vv
+
+
+def _shard_worker(rank, world, port, out, B, Hq, Hkv):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+
+    from free_block_sparse_sparsepr_b200.sharding import ShardedSparsePR
+
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        N, d = 24, 8
+        gen = torch.Generator().manual_seed(11)                     # same full inputs on every rank
+        Q = torch.randn(B, Hq, N, d, generator=gen, dtype=torch.float64)
+        K = torch.randn(B, Hkv, N, d, generator=gen, dtype=torch.float64)
+        V = torch.randn(B, Hkv, N, d, generator=gen, dtype=torch.float64)
+        sh = ShardedSparsePR(B, Hq, Hkv, N, d, compute=_dense_heads)
+        O_local = sh.attention(Q, K, V)
+        O_all = sh.attention(Q, K, V, gather=True)
+        ref = _dense_heads(Q.reshape(B * Hq, N, d), K.reshape(B * Hkv, N, d), V.reshape(B * Hkv, N, d))
+        out.put((rank, sh.lo, sh.hi, bool(torch.equal(O_all, ref)),
+                 bool(torch.equal(O_local, ref[sh.lo * (Hq // Hkv): sh.hi * (Hq // Hkv)]))))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,B,Hq,Hkv", [(2, 1, 8, 2), (3, 2, 8, 4), (4, 1, 6, 3)])
+def test_head_sharded_gather(world, B, Hq, Hkv):
+    """Head sharding on gloo ranks: shards tile the flattened KV heads (sizes within one, a rank
+    may hold none), each rank's output is its slice of the unsharded result, and the all-gather
+    returns the whole output in head order on every rank."""
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, out, B, Hq, Hkv)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(out.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    P = B * Hkv
+    assert res[0][1] == 0 and res[-1][2] == P
+    assert all(res[i][2] == res[i + 1][1] for i in range(world - 1))
+    sizes = [hi - lo for _, lo, hi, _, _ in res]
+    assert max(sizes) - min(sizes) <= 1
+    assert all(r[3] and r[4] for r in res)
+
+
+def test_head_range_tiles():
+    from free_block_sparse_sparsepr_b200.sharding import head_range
+
+    for P in (1, 5, 24, 64):
+        for world in (1, 2, 3, 8):
+            ranges = [head_range(P, world, r) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == P
+            assert all(ranges[i][1] == ranges[i + 1][0] for i in range(world - 1))
+            assert max(b - a for a, b in ranges) - min(b - a for a, b in ranges) <= 1
