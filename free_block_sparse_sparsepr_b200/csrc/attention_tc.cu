@@ -17,7 +17,9 @@
 // occupied only after PV_t(j) in issue order; its completion also tells softmax t that
 // PV_t(j) is done, so O_t may be rescaled and P_t(j+1) written.
 // Key tiles are cut from merged runs of consecutive kept key groups; keys past a run's end
-// (the next group's, or zero fill past the tensor) are masked to -inf.
+// (the next group's, or zero fill past the tensor) are masked to -inf. A tile with at most 64
+// valid keys is a half tile: its S and PV MMAs run with 64 keys and the softmax neither loads
+// nor writes the other half.
 #include <cuda.h>
 #include <float.h>
 #include <math.h>
@@ -275,18 +277,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     } else if (warp == 9) {
         // ================= MMA issuer
         const uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0);
+        const uint32_t idS64 = tc::idesc_bf16_f32(kBM, 64, 0);   // half tile: at most 64 valid keys
         const uint32_t idO = tc::idesc_bf16_f32(kBM, kD, 1);
+        // PV k-steps of key tile j (16 keys each): 4 for a half tile, else 8
+        auto pv_steps = [&](int j) { return key_tile(p, MODE, klist, j).y <= 64 ? 4 : kBN / 16; };
         const int ntiles = two ? 2 : 1;
         bool have = ntk > 0;
         bool ok = __all_sync(kFull, tc::mbar_wait(bar(kBarQ), 0, abort_flag));
         auto issue_S = [&](int t, int j) {
             const uint32_t kb = sK + (j % kStages) * 2 * kRegion;
             const uint32_t qb = sQ + (split ? 0 : t) * 2 * kRegion;
+            const uint32_t id = key_tile(p, MODE, klist, j).y <= 64 ? idS64 : idS;
 #pragma unroll
             for (int k = 0; k < kD / 16; ++k) {
                 const uint32_t off = (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
                 tc::mma_f16_ss(tmem + (uint32_t)(t * 128), tc::smem_desc_sw128(qb + off, 16, 1024),
-                               tc::smem_desc_sw128(kb + off, 16, 1024), idS, k > 0 ? 1u : 0u);
+                               tc::smem_desc_sw128(kb + off, 16, 1024), id, k > 0 ? 1u : 0u);
             }
             tc::commit(bar(kBarS + t));
         };
@@ -315,11 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (lane == 0) {
                     const uint32_t vb = sV + s * 2 * kRegion;
                     const uint32_t pt = tmem + (uint32_t)(t * 128);
+                    const int nk = pv_steps(j);
 #pragma unroll
                     for (int k = 0; k < kBN / 16; ++k)
-                        tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
-                                       tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
-                                       (j >= 2 || k > 0) ? 1u : 0u);
+                        if (k < nk)
+                            tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
+                                           tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
+                                           (j >= 2 || k > 0) ? 1u : 0u);
                     tc::commit(bar(kBarEV + s));
                     if (nh) {
                         issue_S(t, j + 2);
@@ -356,11 +364,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (lane == 0) {
                     const uint32_t vb = sV + s * 2 * kRegion;
                     const uint32_t pt = tmem + (uint32_t)(t * 128);       // P_t packed in S_t's columns
+                    const int nk = pv_steps(j);
 #pragma unroll
                     for (int k = 0; k < kBN / 16; ++k)
-                        tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
-                                       tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
-                                       (j > 0 || k > 0) ? 1u : 0u);
+                        if (k < nk)
+                            tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
+                                           tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
+                                           (j > 0 || k > 0) ? 1u : 0u);
                     const bool last = t + 1 == ntiles;
                     if (last) tc::commit(bar(kBarEV + s));                  // V(j) read by every PV
                     if (nhave) {
@@ -422,21 +432,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     slow = __any_sync(kFull, mx0 > thr);
                     if (!slow) exp_half(sv, c_log2, -m_run, pk0, ps);
                 }
-                {
+                if (lim > 64) {
                     uint32_t sv[2][32];
                     load_half(tS, 1, lim, sv, mx1);
                     slow = slow || __any_sync(kFull, mx1 > thr);
                     if (!slow) {
                         uint32_t pk1[32];
-                        if (lim > 64) exp_half(sv, c_log2, -m_run, pk1, ps);
-                        else
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) pk1[e] = 0u;    // all keys of this half masked
+                        exp_half(sv, c_log2, -m_run, pk1, ps);
                         tc::tmem_st16(tS, pk0);
                         tc::tmem_st16(tS + 16, pk0 + 16);
                         tc::tmem_st16(tS + 32, pk1);
                         tc::tmem_st16(tS + 48, pk1 + 16);
                     }
+                } else if (!slow) {
+                    // a half tile (S and PV run with 64 keys): P of the first 64 keys only
+                    tc::tmem_st16(tS, pk0);
+                    tc::tmem_st16(tS + 16, pk0 + 16);
                 }
                 if (slow) {
                     // some row's max moved by more than 2^8: new per-row max, rescale O and l
