@@ -52,6 +52,7 @@ import numpy as np
 
 __all__ = [
     "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS",
+    "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "PROBE_SEED_SALT", "probe_rows_uniform", "probe_rows_random",
     "sample_rows", "splitmix64", "rademacher_projection", "response_features", "top_mass_fraction",
     "top_mass_count", "top_mass_set", "SHARED_ROWS", "shared_rows", "shared_support",
     "sq_dists_f32", "kmeans_assign", "kmeans_update", "kmeans", "group_means",
@@ -67,6 +68,9 @@ FLAG_HARD_DROP_ONLY = 1 << 0    # no probes, no correction; the whole budget goe
 FLAG_RIDGE_ONLY = 1 << 1        # ridge correction without the subspace projection
 FLAG_RBAR_UNPROJECTED = 1 << 2  # project only the feature-dependent part A(o - obar)
 FLAG_UNIFORM_WEIGHTS = 1 << 3   # all probe weights 1 instead of group-coverage weights
+FLAG_PROBES_UNIFORM = 1 << 5    # probes on a uniform grid of the original token order
+FLAG_PROBES_RANDOM = 1 << 6     # probes drawn at random (seeded)
+PROBE_SEED_SALT = 0x70726F6265  # "probe": separates the probe draws from other uses of the seed
 
 _MASK64 = (1 << 64) - 1
 
@@ -486,6 +490,39 @@ def probe_rows(qgroup: np.ndarray, radial: np.ndarray, M: int):
     return seq[pos].astype(np.int32), pos.astype(np.int32)
 
 
+def _by_sequence_position(rows: np.ndarray, qperm: np.ndarray):
+    """The rows with their group-major positions (index in qperm), in ascending position."""
+    inv = np.empty(len(qperm), dtype=np.int64)
+    inv[np.asarray(qperm, dtype=np.int64)] = np.arange(len(qperm))
+    pos = inv[np.asarray(rows, dtype=np.int64)]
+    o = np.argsort(pos, kind="stable")
+    return np.asarray(rows)[o].astype(np.int32), pos[o].astype(np.int32)
+
+
+def probe_rows_uniform(qperm: np.ndarray, M: int):
+    """Ablation of [probe] (uniform spatio-temporal sampling): the rows floor((m + 1/2) N / M) of
+    the original token order, a uniform grid over (t, h, w) in t-major order, returned in
+    group-major order with their sequence positions (for the coverage weights)."""
+    return _by_sequence_position(sample_rows(len(qperm), M), qperm)
+
+
+def probe_rows_random(qperm: np.ndarray, M: int, seed: int):
+    """Ablation of [probe] (random sampling): M distinct rows from the SplitMix64 stream of state
+    s = seed xor PROBE_SEED_SALT (output i = splitmix64(s + i * 0x9E3779B97F4A7C15)), each output
+    taken mod N, an output equal to an earlier one skipped; returned in group-major order with
+    their sequence positions."""
+    N = len(qperm)
+    s = (int(seed) ^ PROBE_SEED_SALT) & _MASK64
+    rows, seen, i = [], set(), 0
+    while len(rows) < M:
+        c = splitmix64((s + i * 0x9E3779B97F4A7C15) & _MASK64) % N
+        i += 1
+        if c not in seen:
+            seen.add(c)
+            rows.append(c)
+    return _by_sequence_position(np.array(rows, dtype=np.int64), qperm)
+
+
 def coverage_weights(pos: np.ndarray, qoff: np.ndarray, M: int, N: int) -> np.ndarray:
     """Group-coverage weight of each probe, normalised to mean 1 ([probe]).
 
@@ -643,9 +680,15 @@ def partition_head(Qg: np.ndarray, Kh: np.ndarray, cfg) -> HeadPartition:
     kperm, koff = stable_group_order(kgroup, cfg.Gk)
     qperm, qoff = stable_group_order(qgroup, cfg.Gq)
     M = _n_probes(cfg)
+    flags = getattr(cfg, "flags", 0)
     if M:
-        probe, pseq = probe_rows(qgroup, radial, M)
-        if getattr(cfg, "flags", 0) & FLAG_UNIFORM_WEIGHTS:
+        if flags & FLAG_PROBES_UNIFORM:
+            probe, pseq = probe_rows_uniform(qperm, M)
+        elif flags & FLAG_PROBES_RANDOM:
+            probe, pseq = probe_rows_random(qperm, M, getattr(cfg, "seed", 0))
+        else:
+            probe, pseq = probe_rows(qgroup, radial, M)
+        if flags & FLAG_UNIFORM_WEIGHTS:
             w = np.ones(M)
         else:
             w = coverage_weights(pseq, qoff, M, N)

@@ -8,6 +8,8 @@ import pytest
 
 import oracle
 
+GOLDEN = __file__.rsplit("/", 1)[0] + "/golden/splitmix64.txt"
+
 
 def _brute_set(z, mass=0.9):
     """Independent restatement: walk the keys by descending weight with plain Python, stop at
@@ -82,3 +84,22 @@ def test_shared_support_identical_and_disjoint_rows():
     Q[0, np.arange(N), np.arange(N) % d] = 1.0         # query i points at key i
     union, single = oracle.shared_support(Q, Kh, qperm, qoff)
     assert union[0] * N == 8 and np.allclose(single[0] * N, 1)   # disjoint one-key sets add up
+
+
+def test_alternative_probe_samplers():
+    """The probe-sampling ablations of [probe]: the uniform grid is the original rows
+    floor((m + 1/2) N / M); the random draw follows its stated generator (first draws checked
+    against SplitMix64's published outputs from state 0, tests/golden/splitmix64.txt, when the
+    seed cancels the salt), gives M
+    distinct rows, and both come back in group-major order with their positions in qperm."""
+    rng = np.random.default_rng(9)
+    N, M = 500, 16
+    qperm = rng.permutation(N)
+    rows, pos = oracle.probe_rows_uniform(qperm, M)
+    assert sorted(rows) == [(2 * m + 1) * N // (2 * M) for m in range(M)]
+    assert np.all(np.diff(pos) > 0) and np.array_equal(qperm[pos], rows)
+    rows, pos = oracle.probe_rows_random(qperm, M, seed=oracle.PROBE_SEED_SALT)   # state 0
+    gold = [int(line.split()[1], 16) for line in open(GOLDEN).read().splitlines() if line.startswith("0x")]
+    first = [g % N for g in gold]                                            # published first outputs
+    assert set(first) <= set(rows.tolist())
+    assert len(set(rows.tolist())) == M and np.all(np.diff(pos) > 0) and np.array_equal(qperm[pos], rows)
