@@ -20,6 +20,8 @@ FLAG_RIDGE_ONLY = 1 << 1
 FLAG_RBAR_UNPROJECTED = 1 << 2
 FLAG_UNIFORM_WEIGHTS = 1 << 3
 FLAG_TOPMASS = 1 << 4
+FLAG_PROBES_UNIFORM = 1 << 5     # ablation: probes on a uniform grid of the original token order
+FLAG_PROBES_RANDOM = 1 << 6      # ablation: probes drawn at random (seeded SplitMix64)
 FLAG_STAGE_TIMING = 1 << 8
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace allocation failed",
@@ -378,4 +380,5 @@ def route_from_tensors(t: dict) -> Route:
 __all__ = ["SparsePR", "SparsePRError", "Config", "Partition", "Route", "Fit", "Stats", "load_library",
            "header_functions", "partition_from_tensors", "route_from_tensors", "device_view", "LIB_PATH",
            "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS", "FLAG_TOPMASS",
+           "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "SHARED_ROWS",
            "FLAG_STAGE_TIMING"]

@@ -21,7 +21,8 @@ constexpr int kProbeSplits = 32;
 constexpr int kSortChunk = 2048;   // rows per counting-sort chunk (matches the sort kernels)
 constexpr unsigned kSupportedFlags =
     SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED |
-    SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING;
+    SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING |
+    SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM;
 
 inline int pad16(int v) { return (v + 15) / 16 * 16; }
 inline int pad64(int v) { return (v + 63) / 64 * 64; }
@@ -121,6 +122,8 @@ sparsepr_status validate(const sparsepr_config* c) {
     if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return SPARSEPR_ERR_INVALID_ARG;
     if (!(c->rho_exec > 0.f) || !isfinite(c->rho_exec)) return SPARSEPR_ERR_INVALID_ARG;
     if (c->flags & ~kSupportedFlags)
+        return SPARSEPR_ERR_INVALID_ARG;
+    if ((c->flags & SPARSEPR_FLAG_PROBES_UNIFORM) && (c->flags & SPARSEPR_FLAG_PROBES_RANDOM))
         return SPARSEPR_ERR_INVALID_ARG;
     if (!(c->flags & SPARSEPR_FLAG_HARD_DROP_ONLY)) {
         if (c->M < 1 || c->M > c->N) return SPARSEPR_ERR_INVALID_ARG;
@@ -242,9 +245,14 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     }
     st = kmeans(h, h->ycoord, h->DPy, c.Gq, h->qgroup, h->radial, h->qperm, h->qoff, s);
     if (st) return st;
-    // probe rows (stratified, radial order) and their coverage weights
+    // probe rows (stratified, radial order; or an ablation's grid / random draws) and their weights
     if (h->M) {
-        SPR_TRY(spr::launch_probe_select(h->qperm, h->qoff, h->radial, h->probe, h->probe_pos, h->probe_seq,
+        if (c.flags & (SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM))
+            SPR_TRY(spr::launch_probe_alt(h->qperm, h->qoff, h->qgroup, h->probe, h->probe_pos, h->probe_seq, P, N,
+                                          c.Gq, h->M, (c.flags & SPARSEPR_FLAG_PROBES_RANDOM) != 0, c.seed,
+                                          h->dev_status, s));
+        else
+            SPR_TRY(spr::launch_probe_select(h->qperm, h->qoff, h->radial, h->probe, h->probe_pos, h->probe_seq,
                                          P, N, c.Gq, h->M, s));
         SPR_TRY(spr::launch_probe_weights(h->qoff, h->probe_seq, h->weights, P, N, c.Gq, h->M,
                                           (c.flags & SPARSEPR_FLAG_UNIFORM_WEIGHTS) != 0, s));

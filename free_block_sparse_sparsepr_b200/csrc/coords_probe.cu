@@ -209,6 +209,65 @@ __global__ void __launch_bounds__(256) probe_select_kernel(const int32_t* __rest
     }
 }
 
+// Probe-sampling ablations of [probe]: the rows of a uniform grid over the original token order
+// (floor((m + 1/2) N / M)), or M distinct rows from the SplitMix64 stream of state
+// seed ^ 0x70726F6265 (output i = splitmix64(state + i * 0x9E3779B97F4A7C15), taken mod N,
+// repeats skipped). Each row's group-major position is found in its group's slice of qperm, and
+// the probes are stored in ascending position (that position also drives the coverage weights).
+constexpr unsigned long long kProbeSalt = 0x70726F6265ull;
+constexpr int kMaxProbeRows = 64;
+__global__ void __launch_bounds__(kMaxProbeRows) probe_alt_kernel(const int32_t* __restrict__ qperm,
+                                                                  const int32_t* __restrict__ qoff,
+                                                                  const int32_t* __restrict__ qgroup,
+                                                                  int32_t* probe, int32_t* probe_pos,
+                                                                  int32_t* probe_seq, int N, int Gq, int M,
+                                                                  int random, unsigned long long seed, int* status) {
+    const int z = blockIdx.x, m = threadIdx.x;
+    __shared__ int rows[kMaxProbeRows];
+    __shared__ int pos[kMaxProbeRows];
+    if (random) {
+        if (m == 0) {
+            const unsigned long long st = seed ^ kProbeSalt;
+            int got = 0;
+            // the stream repeats a row rarely; the bound only guards against M close to N
+            const long long cap = 64ll * N + 4096;
+            for (long long i = 0; got < M && i < cap; ++i) {
+                const int c = (int)(splitmix64(st + (unsigned long long)i * 0x9E3779B97F4A7C15ull) %
+                                    (unsigned long long)N);
+                bool dup = false;
+                for (int e = 0; e < got; ++e) dup |= rows[e] == c;
+                if (!dup) rows[got++] = c;
+            }
+            for (; got < M; ++got) {            // only past the bound: flag it and fill distinct rows
+                set_status(status, kDevBounds);
+                rows[got] = got;
+            }
+        }
+    } else if (m < M) {
+        rows[m] = (int)sample_pos(m, N, M);
+    }
+    __syncthreads();
+    int r = 0, p = 0;
+    if (m < M) {
+        r = rows[m];
+        const int a = qgroup[(long long)z * N + r];
+        const int lo = qoff[(long long)z * (Gq + 1) + a], hi = qoff[(long long)z * (Gq + 1) + a + 1];
+        const int32_t* pz = qperm + (long long)z * N;
+        p = lo;
+        for (int j = lo; j < hi; ++j)
+            if (pz[j] == r) { p = j; break; }
+        pos[m] = p;
+    }
+    __syncthreads();
+    if (m < M) {
+        int rank = 0;
+        for (int e = 0; e < M; ++e) rank += pos[e] < p ? 1 : 0;
+        probe[(long long)z * M + rank] = r;
+        probe_pos[(long long)z * M + rank] = p;
+        probe_seq[(long long)z * M + rank] = p;
+    }
+}
+
 // Coverage weight of probe m: its group's size split over the group's probes, plus the
 // sizes of probe-less groups whose nearest probe (sequence distance, ties -> lower m) is m.
 __global__ void probe_weights_kernel(const int32_t* __restrict__ qoff,
@@ -282,6 +341,16 @@ cudaError_t launch_probe_select(const int32_t* qperm, const int32_t* qoff, const
                                 int N, int Gq, int M, cudaStream_t s) {
     if (M <= 0) return cudaSuccess;
     probe_select_kernel<<<dim3(M, P), 256, 0, s>>>(qperm, qoff, radial, probe, probe_pos, probe_seq, N, Gq, M);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_probe_alt(const int32_t* qperm, const int32_t* qoff, const int32_t* qgroup, int32_t* probe,
+                             int32_t* probe_pos, int32_t* probe_seq, int P, int N, int Gq, int M, bool random,
+                             unsigned long long seed, int* status, cudaStream_t s) {
+    if (M <= 0) return cudaSuccess;
+    if (M > kMaxProbeRows || M > N) return cudaErrorInvalidValue;
+    probe_alt_kernel<<<P, kMaxProbeRows, 0, s>>>(qperm, qoff, qgroup, probe, probe_pos, probe_seq, N, Gq, M,
+                                                 random ? 1 : 0, seed, status);
     return cudaGetLastError();
 }
 

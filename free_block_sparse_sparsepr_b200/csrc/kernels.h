@@ -101,6 +101,10 @@ cudaError_t launch_make_projection(bf16* projT, int Gk, int Gkp, int rQ, int DPy
 cudaError_t launch_probe_select(const int32_t* qperm, const int32_t* qoff, const float* radial,
                                 int32_t* probe, int32_t* probe_pos, int32_t* probe_seq, int P,
                                 int N, int Gq, int M, cudaStream_t s);
+// Probe-sampling ablations: uniform grid of the original order, or seeded SplitMix64 draws.
+cudaError_t launch_probe_alt(const int32_t* qperm, const int32_t* qoff, const int32_t* qgroup, int32_t* probe,
+                             int32_t* probe_pos, int32_t* probe_seq, int P, int N, int Gq, int M, bool random,
+                             unsigned long long seed, int* status, cudaStream_t s);
 cudaError_t launch_probe_weights(const int32_t* qoff, const int32_t* probe_seq, float* w, int P,
                                  int N, int Gq, int M, bool uniform, cudaStream_t s);
 

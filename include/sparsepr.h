@@ -60,6 +60,10 @@ typedef enum sparsepr_status {
 #define SPARSEPR_FLAG_RBAR_UNPROJECTED  (1u << 2)  /* ablation: project only A(o - obar), add Rbar unprojected */
 #define SPARSEPR_FLAG_UNIFORM_WEIGHTS   (1u << 3)  /* probe weights 1 instead of group coverage */
 #define SPARSEPR_FLAG_TOPMASS           (1u << 4)  /* sparsepr_partition also writes the support diagnostic */
+#define SPARSEPR_FLAG_PROBES_UNIFORM    (1u << 5)  /* ablation: probes at rows floor((m+1/2)N/M) of the original order */
+#define SPARSEPR_FLAG_PROBES_RANDOM     (1u << 6)  /* ablation: M distinct rows from the SplitMix64 stream of state
+                                                      seed ^ 0x70726F6265, each output mod N (repeats skipped);
+                                                      at most one of the two probe flags */
 #define SPARSEPR_FLAG_STAGE_TIMING      (1u << 8)  /* record per-stage CUDA events (sparsepr_get_stats) */
 
 /*

@@ -375,6 +375,62 @@ def test_head_shards_reproduce_the_call(name):
     assert torch.equal(torch.cat(parts), O_full)
 
 
+@pytest.mark.parametrize("flag", ["FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM"])
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
+def test_probe_sampling_ablations(name, flag):
+    """The probe-sampling ablations of [probe]: the GPU's probe rows, positions and coverage
+    weights equal the oracle's sampler applied to the GPU's own query groups (exact rows and
+    positions); with the oracle's partition carrying those probes handed in to both sides, the
+    corrected output matches the oracle."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    seed = w.seed
+    with spr.SparsePR.from_workload(w, flags=getattr(spr, flag)) as h:
+        part = h.partition(q, k)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+        pv = {n: t.cpu().numpy() for n, t in h.partition_views(part).items()}
+
+    def sample(qperm):
+        if flag == "FLAG_PROBES_UNIFORM":
+            return oracle.probe_rows_uniform(qperm, w.M)
+        return oracle.probe_rows_random(qperm, w.M, seed)
+
+    for z in range(w.B * w.Hkv):
+        rows, pos = sample(pv["qperm"][z])
+        assert np.array_equal(pv["probe"][z], rows)
+        assert np.array_equal(pv["probe_pos"][z], pos)
+        wref = oracle.coverage_weights(pos, pv["qoff"][z], w.M, w.N)
+        assert np.abs(pv["weights"][z] - wref).max() < 1e-4 * max(1.0, wref.max())
+    # end to end on the oracle's partition with the ablation's probes
+    parts = {}
+    for key, hp in res["partitions"].items():
+        rows, pos = sample(hp.qperm)
+        parts[key] = oracle.HeadPartition(hp.kgroup, hp.qgroup, hp.kcent, hp.kperm, hp.koff, hp.qperm, hp.qoff,
+                                          hp.radial, rows, pos, oracle.coverage_weights(pos, hp.qoff, w.M, w.N),
+                                          hp.features, hp.z, hp.ycoord)
+
+    class Cfg:
+        pass
+
+    cfg = Cfg()
+    for f in ("rK", "Gk", "Gq", "rQ", "M", "r", "lam", "rho", "kmeans_iters", "seed"):
+        setattr(cfg, f, getattr(w, f))
+    cfg.flags = getattr(oracle, flag)
+    ref = oracle.sparsepr_attention(Q, K, V, cfg, partitions=parts, routes=res["routes"])
+    res2 = dict(res, partitions=parts)
+    pt, rt = partition_tensors(res2, w), route_tensors(res, w)
+    with spr.SparsePR.from_workload(w, flags=getattr(spr, flag)) as h:
+        part, route = spr.partition_from_tensors(pt), spr.route_from_tensors(rt)
+        Qp, Kp, Vp, Osp, O = (torch.empty_like(t) for t in (q, k, v, q, q))
+        h.permute(q, k, v, part, Qp, Kp, Vp)
+        h.blocksparse_attn(Qp, Kp, Vp, part, route, Osp)
+        fit = h.probe_fit(q, k, v, part, Osp)
+        h.writeback(part, Osp, fit, O)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+    assert_close(bf16_to_f64(O), ref["O"], f"{flag} output")
+
+
 @pytest.mark.parametrize("flag", ["FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED"])
 @pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
 def test_ablation_corrections(name, flag):
