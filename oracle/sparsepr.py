@@ -52,7 +52,7 @@ import numpy as np
 
 __all__ = [
     "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS",
-    "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "PROBE_SEED_SALT", "probe_rows_uniform", "probe_rows_random",
+    "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "FLAG_SEMANTIC_PARTITION", "PROBE_SEED_SALT", "probe_rows_uniform", "probe_rows_random",
     "sample_rows", "splitmix64", "rademacher_projection", "response_features", "top_mass_fraction",
     "top_mass_count", "top_mass_set", "SHARED_ROWS", "shared_rows", "shared_support",
     "sq_dists_f32", "kmeans_assign", "kmeans_update", "kmeans", "group_means",
@@ -70,6 +70,7 @@ FLAG_RBAR_UNPROJECTED = 1 << 2  # project only the feature-dependent part A(o - 
 FLAG_UNIFORM_WEIGHTS = 1 << 3   # all probe weights 1 instead of group-coverage weights
 FLAG_PROBES_UNIFORM = 1 << 5    # probes on a uniform grid of the original token order
 FLAG_PROBES_RANDOM = 1 << 6     # probes drawn at random (seeded)
+FLAG_SEMANTIC_PARTITION = 1 << 7   # ablation: k-means on the raw keys and the raw mean query
 PROBE_SEED_SALT = 0x70726F6265  # "probe": separates the probe draws from other uses of the seed
 
 _MASK64 = (1 << 64) - 1
@@ -673,9 +674,17 @@ def partition_head(Qg: np.ndarray, Kh: np.ndarray, cfg) -> HeadPartition:
     """
     N = Kh.shape[0]
     z, F = response_features(Qg, Kh, cfg.rK)
-    kgroup, _, _ = kmeans(F, cfg.Gk, cfg.kmeans_iters)
-    kcent = group_means(Kh, kgroup, cfg.Gk)
-    _, y = query_coordinates(Qg, kcent, cfg.rQ, getattr(cfg, "seed", 0))
+    if getattr(cfg, "flags", 0) & FLAG_SEMANTIC_PARTITION:
+        # ablation ([partition]: grouping by activations instead of responses): k-means on the
+        # raw keys, and on the mean query of the KV group, both as fp32 rows
+        F = _to_f32(Kh)
+        y = _to_f32(Qg.mean(axis=0))
+        kgroup, _, _ = kmeans(F, cfg.Gk, cfg.kmeans_iters)
+        kcent = group_means(Kh, kgroup, cfg.Gk)
+    else:
+        kgroup, _, _ = kmeans(F, cfg.Gk, cfg.kmeans_iters)
+        kcent = group_means(Kh, kgroup, cfg.Gk)
+        _, y = query_coordinates(Qg, kcent, cfg.rQ, getattr(cfg, "seed", 0))
     qgroup, _, radial = kmeans(y, cfg.Gq, cfg.kmeans_iters)
     kperm, koff = stable_group_order(kgroup, cfg.Gk)
     qperm, qoff = stable_group_order(qgroup, cfg.Gq)

@@ -103,3 +103,30 @@ def test_alternative_probe_samplers():
     first = [g % N for g in gold]                                            # published first outputs
     assert set(first) <= set(rows.tolist())
     assert len(set(rows.tolist())) == M and np.all(np.diff(pos) > 0) and np.array_equal(qperm[pos], rows)
+
+
+def test_semantic_partition_groups_raw_activations():
+    """The semantic-partition ablation of [partition]: key groups are the k-means of the raw
+    keys (recovered exactly on planted, well separated key clusters, whatever the queries), and
+    query groups the k-means of the raw mean query of the KV group."""
+    from synthetic import get_workload
+
+    rng = np.random.default_rng(2)
+    g, N, d, G = 2, 128, 16, 4
+    centers = rng.standard_normal((G, d)) * 20.0
+    lab = np.repeat(np.arange(G), N // G)
+    Kh = centers[lab] + rng.standard_normal((N, d)) * 0.1
+    qc = rng.standard_normal((G, d)) * 20.0
+    rows = np.arange(N)
+    qlab = (rows // 16 + rows // 64) % G          # another partition; the k-means seed rows fall in distinct clusters
+    Qg = np.stack([qc[qlab] + rng.standard_normal((N, d)) * 0.1 for _ in range(g)])
+    import types
+
+    base = get_workload("tiny_n1024")
+    cfg = types.SimpleNamespace(rK=base.rK, rQ=base.rQ, Gk=G, Gq=G, M=8, r=4, kmeans_iters=10, seed=0,
+                                flags=oracle.FLAG_SEMANTIC_PARTITION)
+    hp = oracle.partition_head(Qg, Kh, cfg)
+    same = lambda a, b: all(len(set(b[a == v])) == 1 for v in np.unique(a)) and len(np.unique(a)) == len(np.unique(b))
+    assert same(hp.kgroup, lab) and same(hp.qgroup, qlab)
+    assert np.allclose(hp.features, Kh.astype(np.float32))
+    assert np.allclose(hp.ycoord, Qg.mean(axis=0).astype(np.float32))
