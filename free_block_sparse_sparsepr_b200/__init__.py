@@ -22,6 +22,7 @@ FLAG_UNIFORM_WEIGHTS = 1 << 3
 FLAG_TOPMASS = 1 << 4
 FLAG_PROBES_UNIFORM = 1 << 5     # ablation: probes on a uniform grid of the original token order
 FLAG_PROBES_RANDOM = 1 << 6      # ablation: probes drawn at random (seeded SplitMix64)
+FLAG_SEMANTIC_PARTITION = 1 << 7  # ablation: k-means on the raw keys and the raw mean query
 FLAG_STAGE_TIMING = 1 << 8
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace allocation failed",
@@ -324,7 +325,7 @@ class SparsePR:
              "kcent": device_view(part.kcent, (P, c.Gk, c.d), torch.float32),
              "radial": device_view(part.radial, (P, N), torch.float32)}
         if part.features:
-            DP = (c.rK + 15) // 16 * 16
+            DP = c.d if c.flags & FLAG_SEMANTIC_PARTITION else (c.rK + 15) // 16 * 16
             v["features"] = device_view(part.features, (P, N, DP), torch.float32)
         if part.topmass:
             v["topmass"] = device_view(part.topmass, (P, c.rK), torch.float32)
@@ -380,5 +381,5 @@ def route_from_tensors(t: dict) -> Route:
 __all__ = ["SparsePR", "SparsePRError", "Config", "Partition", "Route", "Fit", "Stats", "load_library",
            "header_functions", "partition_from_tensors", "route_from_tensors", "device_view", "LIB_PATH",
            "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS", "FLAG_TOPMASS",
-           "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "SHARED_ROWS",
+           "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "FLAG_SEMANTIC_PARTITION", "SHARED_ROWS",
            "FLAG_STAGE_TIMING"]

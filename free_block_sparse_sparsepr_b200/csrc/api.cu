@@ -22,7 +22,7 @@ constexpr int kSortChunk = 2048;   // rows per counting-sort chunk (matches the 
 constexpr unsigned kSupportedFlags =
     SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED |
     SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING |
-    SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM;
+    SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM | SPARSEPR_FLAG_SEMANTIC_PARTITION;
 
 inline int pad16(int v) { return (v + 15) / 16 * 16; }
 inline int pad64(int v) { return (v + 63) / 64 * 64; }
@@ -74,6 +74,7 @@ struct sparsepr_handle_s {
     float *kmxx = nullptr, *kmcc = nullptr;
     int4* kmfix = nullptr;
     int* kmfix_count = nullptr;
+    bool semantic = false;   // ablation: k-means on the raw activations
     int launches = 0;
     int device = 0;
     int num_sms = 148;
@@ -125,6 +126,8 @@ sparsepr_status validate(const sparsepr_config* c) {
         return SPARSEPR_ERR_INVALID_ARG;
     if ((c->flags & SPARSEPR_FLAG_PROBES_UNIFORM) && (c->flags & SPARSEPR_FLAG_PROBES_RANDOM))
         return SPARSEPR_ERR_INVALID_ARG;
+    if ((c->flags & SPARSEPR_FLAG_SEMANTIC_PARTITION) && (c->flags & SPARSEPR_FLAG_TOPMASS))
+        return SPARSEPR_ERR_INVALID_ARG;
     if (!(c->flags & SPARSEPR_FLAG_HARD_DROP_ONLY)) {
         if (c->M < 1 || c->M > c->N) return SPARSEPR_ERR_INVALID_ARG;
         if (c->M > 64) return SPARSEPR_ERR_UNSUPPORTED;
@@ -153,7 +156,7 @@ long long budget_pairs(const sparsepr_config& c, int M) {
 sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t* labels, float* dist,
                        int32_t* perm, int32_t* off, cudaStream_t s) {
     const int P = h->P, n = h->cfg.N;
-    const bool tc = spr::km_tc_supported(G);
+    const bool tc = spr::km_tc_supported(G) && DP <= 64;
     auto assign = [&](bool first, const int* done) -> cudaError_t {
         if (!tc) return spr::launch_km_assign(X, h->kmC, labels, dist, h->km_changed, done, P, n, G, DP, first, s);
         cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC2, h->kmcc, P, G, DP, s);
@@ -205,9 +208,30 @@ sparsepr_status query_logits(sparsepr_handle h, const bf16* Q, const bf16* chi, 
     return SPARSEPR_OK;
 }
 
+sparsepr_status probes_impl(sparsepr_handle h, cudaStream_t s);
+
+// Semantic-partition ablation ([partition]): key groups from the raw keys and query groups from
+// the raw mean query of each KV group (fp32 rows of width d), everything after as in the
+// response-coupled partition; the query logits are still formed for the routing.
+sparsepr_status partition_semantic(sparsepr_handle h, const bf16* Q, const bf16* K, cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    const int P = h->P, N = c.N, d = c.d;
+    SPR_TRY(spr::launch_mean_heads_f32(K, h->features, P, 1, N, d, s));
+    sparsepr_status st = kmeans(h, h->features, d, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s);
+    if (st) return st;
+    SPR_TRY(spr::launch_group_mean_bf16(K, h->kperm, h->koff, h->kcent, h->chi, h->clo, P, N, c.Gk, d, s));
+    st = query_logits(h, Q, h->chi, h->clo, h->koff, s);
+    if (st) return st;
+    SPR_TRY(spr::launch_mean_heads_f32(Q, h->ycoord, P, h->g, N, d, s));
+    st = kmeans(h, h->ycoord, d, c.Gq, h->qgroup, h->radial, h->qperm, h->qoff, s);
+    if (st) return st;
+    return probes_impl(h, s);
+}
+
 sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
     const int P = h->P, N = c.N, d = c.d;
+    if (h->semantic) return partition_semantic(h, Q, K, s);
     // (1) sampled responses: F[z] = K[z] . Qs[z]^T / sqrt(d)
     SPR_TRY(spr::launch_gather_samples(Q, h->Qs, c.B, c.Hq, c.Hkv, N, d, c.rK, h->DPk, s));
     spr::GemmArgs a;
@@ -245,7 +269,13 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     }
     st = kmeans(h, h->ycoord, h->DPy, c.Gq, h->qgroup, h->radial, h->qperm, h->qoff, s);
     if (st) return st;
-    // probe rows (stratified, radial order; or an ablation's grid / random draws) and their weights
+    return probes_impl(h, s);
+}
+
+// Probe rows (stratified, radial order; or an ablation's grid / random draws) and their weights.
+sparsepr_status probes_impl(sparsepr_handle h, cudaStream_t s) {
+    const sparsepr_config& c = h->cfg;
+    const int P = h->P, N = c.N;
     if (h->M) {
         if (c.flags & (SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM))
             SPR_TRY(spr::launch_probe_alt(h->qperm, h->qoff, h->qgroup, h->probe, h->probe_pos, h->probe_seq, P, N,
@@ -392,10 +422,11 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     h->Hp = c.B * c.Hq;
     h->g = c.Hq / c.Hkv;
     h->M = (c.flags & SPARSEPR_FLAG_HARD_DROP_ONLY) ? 0 : c.M;
-    h->DPk = pad16(c.rK);
+    h->semantic = (c.flags & SPARSEPR_FLAG_SEMANTIC_PARTITION) != 0;
+    h->DPk = h->semantic ? c.d : pad16(c.rK);
     h->proj = c.Gk > c.rQ;
     h->Dy = h->proj ? c.rQ : c.Gk;
-    h->DPy = pad16(h->Dy);
+    h->DPy = h->semantic ? c.d : pad16(h->Dy);
     h->Gkp = pad64(c.Gk);
     h->nch = (c.N + kSortChunk - 1) / kSortChunk;
     h->Gmax = c.Gk > c.Gq ? c.Gk : c.Gq;
@@ -413,7 +444,7 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     A_(kgroup, P * N); A_(qgroup, P * N); A_(kperm, P * N); A_(koff, P * (Gk + 1));
     A_(qperm, P * N); A_(qoff, P * (Gq + 1)); A_(probe, P * M); A_(probe_pos, P * M); A_(probe_seq, P * M);
     A_(kcent, P * Gk * d); A_(radial, P * N); A_(weights, P * M); A_(features, P * N * h->DPk); A_(topmass, P * c.rK);
-    A_(ycoord, P * N * h->DPy); A_(kdist, P * N); A_(kmC, P * h->Gmax * 64);
+    A_(ycoord, P * N * h->DPy); A_(kdist, P * N); A_(kmC, P * h->Gmax * (size_t)(h->DPk > 64 || h->DPy > 64 ? (h->DPk > h->DPy ? h->DPk : h->DPy) : 64));
     A_(counts, P * h->nch * h->Gmax); A_(bases, P * h->nch * h->Gmax); A_(km_changed, P); A_(km_done, P);
     A_(Qs, P * h->DPk * d); A_(chi, P * Gk * d); A_(clo, P * Gk * d);
     A_(u, Hp * N * Gk); A_(ulse, Hp * N);

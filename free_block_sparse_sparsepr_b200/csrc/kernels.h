@@ -23,7 +23,9 @@ struct GemmArgs {
 cudaError_t launch_gemm_bf16(const GemmArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- k-means + group-major order
-// X: [P][n][DP] fp32 rows (DP in {16,32,48,64}); C: [P][G][DP]; labels/dist: [P][n].
+// X: [P][n][DP] fp32 rows (DP in {16,32,48,64,128}); C: [P][G][DP]; labels/dist: [P][n].
+// dst [P][N][d] fp32 = mean over the g query heads of src [P*g][N][d] bf16 (g = 1: widening copy).
+cudaError_t launch_mean_heads_f32(const bf16* src, float* dst, int P, int g, int N, int d, cudaStream_t s);
 cudaError_t launch_km_seed(const float* X, float* C, int P, int n, int G, int DP, cudaStream_t s);
 cudaError_t launch_km_assign(const float* X, const float* C, int32_t* labels, float* dist,
                              int* changed, const int* done, int P, int n, int G, int DP, bool first,

@@ -13,7 +13,7 @@ namespace {
 constexpr int kSortSub = 256;       // rows per sub-chunk (one row per thread)
 constexpr int kSortChunk = 2048;    // rows per counting-sort chunk (one CTA, 8 sub-chunks in order)
 constexpr int kAssignRows = 128;    // rows per assignment CTA (one row per thread)
-constexpr int kAssignCent = 128;    // centroids staged in shared memory per pass
+constexpr int kAssignCentMax = 128; // centroids staged in shared memory per pass (64 at D = 128)
 
 __global__ void km_seed_kernel(const float* X, float* C, int n, int G, int DP) {
     const int z = blockIdx.x;
@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kAssignRows) km_assign_kernel(const float* __r
                                                                 int32_t* labels, float* dist,
                                                                 int* changed, const int* done,
                                                                 int n, int G, int first) {
+    constexpr int kAssignCent = DP > 64 ? 64 : kAssignCentMax;
     const int z = blockIdx.y;
     if (done && done[z]) return;
     __shared__ __align__(16) float sC[kAssignCent * DP];
@@ -297,7 +298,27 @@ __global__ void split_bf16_kernel(const float* x, bf16* hi, bf16* lo, long long 
     lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
+// dst[z][i][c] = (1/g) sum_j src[z * g + j][i][c] in fp32 (g = 1: the rows widened to fp32).
+__global__ void mean_heads_f32_kernel(const bf16* __restrict__ src, float* dst, int g, long long per_head) {
+    const int z = blockIdx.y;
+    const float inv = 1.f / (float)g;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < per_head;
+         t += (long long)gridDim.x * blockDim.x) {
+        float a = 0.f;
+        for (int j = 0; j < g; ++j) a += __bfloat162float(src[((long long)z * g + j) * per_head + t]);
+        dst[(long long)z * per_head + t] = g == 1 ? a : a * inv;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_mean_heads_f32(const bf16* src, float* dst, int P, int g, int N, int d, cudaStream_t s) {
+    const long long per_head = (long long)N * d;
+    long long blocks = (per_head + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    mean_heads_f32_kernel<<<dim3((unsigned)blocks, P), 256, 0, s>>>(src, dst, g, per_head);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_km_seed(const float* X, float* C, int P, int n, int G, int DP, cudaStream_t s) {
     km_seed_kernel<<<P, 256, 0, s>>>(X, C, n, G, DP);
@@ -313,6 +334,7 @@ cudaError_t launch_km_assign(const float* X, const float* C, int32_t* labels, fl
         case 32: km_assign_kernel<32><<<grid, kAssignRows, 0, s>>>(X, C, labels, dist, changed, done, n, G, first); break;
         case 48: km_assign_kernel<48><<<grid, kAssignRows, 0, s>>>(X, C, labels, dist, changed, done, n, G, first); break;
         case 64: km_assign_kernel<64><<<grid, kAssignRows, 0, s>>>(X, C, labels, dist, changed, done, n, G, first); break;
+        case 128: km_assign_kernel<128><<<grid, kAssignRows, 0, s>>>(X, C, labels, dist, changed, done, n, G, first); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -326,6 +348,7 @@ cudaError_t launch_km_update(const float* X, const int32_t* perm, const int32_t*
         case 32: km_update_kernel<32><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
         case 48: km_update_kernel<48><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
         case 64: km_update_kernel<64><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
+        case 128: km_update_kernel<128><<<grid, kUpdThreads, 0, s>>>(X, perm, off, C, done, n, G); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

@@ -64,6 +64,10 @@ typedef enum sparsepr_status {
 #define SPARSEPR_FLAG_PROBES_RANDOM     (1u << 6)  /* ablation: M distinct rows from the SplitMix64 stream of state
                                                       seed ^ 0x70726F6265, each output mod N (repeats skipped);
                                                       at most one of the two probe flags */
+#define SPARSEPR_FLAG_SEMANTIC_PARTITION (1u << 7) /* ablation: key groups by k-means on the raw keys, query
+                                                      groups on the raw mean query of the KV group (fp32 rows
+                                                      of width d; `features` then holds the keys); not with
+                                                      SPARSEPR_FLAG_TOPMASS */
 #define SPARSEPR_FLAG_STAGE_TIMING      (1u << 8)  /* record per-stage CUDA events (sparsepr_get_stats) */
 
 /*

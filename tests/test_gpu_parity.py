@@ -375,6 +375,56 @@ def test_head_shards_reproduce_the_call(name):
     assert torch.equal(torch.cat(parts), O_full)
 
 
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
+def test_semantic_partition_ablation(name):
+    """The semantic-partition ablation of [partition] (k-means on the raw keys and the raw mean
+    query): the GPU's groups agree with the oracle's where the assignment margin is clear, its
+    group-major orders are the stable sort of its own labels, and with the oracle's semantic
+    partition handed in to both sides the corrected output matches the oracle."""
+    import types
+
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    cfg = types.SimpleNamespace(rK=w.rK, Gk=w.Gk, Gq=w.Gq, rQ=w.rQ, M=w.M, r=w.r, lam=w.lam, rho=w.rho,
+                                kmeans_iters=w.kmeans_iters, seed=w.seed, flags=oracle.FLAG_SEMANTIC_PARTITION)
+    with spr.SparsePR.from_workload(w, flags=spr.FLAG_SEMANTIC_PARTITION) as h:
+        part = h.partition(q, k)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+        pv = {n: t.cpu().numpy() for n, t in h.partition_views(part).items()}
+    parts = {}
+    for b in range(w.B):
+        for hk in range(w.Hkv):
+            z = b * w.Hkv + hk
+            Qg = bf16_to_f64(q[b, hk * w.g:(hk + 1) * w.g])
+            Kh = bf16_to_f64(k[b, hk])
+            po = oracle.partition_head(Qg, Kh, cfg)
+            parts[(b, hk)] = po
+            assert np.array_equal(pv["features"][z], po.features)          # the raw keys, widened
+            _, Ck, _ = oracle.kmeans(po.features, w.Gk, w.kmeans_iters)
+            mk = kmeans_margin(po.features, Ck) > 1e-3
+            assert (pv["kgroup"][z] == po.kgroup)[mk].mean() >= 0.99
+            _, Cq, _ = oracle.kmeans(po.ycoord, w.Gq, w.kmeans_iters)
+            mq = kmeans_margin(po.ycoord, Cq) > 1e-3
+            assert (pv["qgroup"][z] == po.qgroup)[mq].mean() >= 0.99
+            for lab, perm in ((pv["kgroup"][z], pv["kperm"][z]), (pv["qgroup"][z], pv["qperm"][z])):
+                assert np.array_equal(perm, np.argsort(lab, kind="stable"))
+    routes = {key: oracle.route_head(bf16_to_f64(q[key[0], key[1] * w.g:(key[1] + 1) * w.g]), hp, cfg)
+              for key, hp in parts.items()}
+    ref = oracle.sparsepr_attention(Q, K, V, cfg, partitions=parts, routes=routes)
+    res2 = dict(res, partitions=parts, routes=routes)
+    pt, rt = partition_tensors(res2, w), route_tensors(res2, w)
+    with spr.SparsePR.from_workload(w, flags=spr.FLAG_SEMANTIC_PARTITION) as h:
+        part, route = spr.partition_from_tensors(pt), spr.route_from_tensors(rt)
+        Qp, Kp, Vp, Osp, O = (torch.empty_like(t) for t in (q, k, v, q, q))
+        h.permute(q, k, v, part, Qp, Kp, Vp)
+        h.blocksparse_attn(Qp, Kp, Vp, part, route, Osp)
+        fit = h.probe_fit(q, k, v, part, Osp)
+        h.writeback(part, Osp, fit, O)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+    assert_close(bf16_to_f64(O), ref["O"], "semantic-partition output")
+
+
 @pytest.mark.parametrize("flag", ["FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM"])
 @pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
 def test_probe_sampling_ablations(name, flag):
