@@ -52,7 +52,8 @@ import numpy as np
 
 __all__ = [
     "FLAG_HARD_DROP_ONLY", "FLAG_RIDGE_ONLY", "FLAG_RBAR_UNPROJECTED", "FLAG_UNIFORM_WEIGHTS",
-    "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "FLAG_SEMANTIC_PARTITION", "PROBE_SEED_SALT", "probe_rows_uniform", "probe_rows_random",
+    "FLAG_PROBES_UNIFORM", "FLAG_PROBES_RANDOM", "FLAG_SEMANTIC_PARTITION", "PROBE_SEED_SALT",
+    "affine_diagnostics", "probe_rows_uniform", "probe_rows_random",
     "sample_rows", "splitmix64", "rademacher_projection", "response_features", "top_mass_fraction",
     "top_mass_count", "top_mass_set", "SHARED_ROWS", "shared_rows", "shared_support",
     "sq_dists_f32", "kmeans_assign", "kmeans_update", "kmeans", "group_means",
@@ -599,6 +600,23 @@ def residual_subspace(R: np.ndarray, w: np.ndarray, r: int):
         return U[:, :0], s
     rank = int((s > s[0] * max(Rw.shape) * np.finfo(np.float64).eps).sum())
     return U[:, : min(r, rank)], s
+
+
+def affine_diagnostics(Os: np.ndarray, Od: np.ndarray):
+    """How affine the hard-drop residual of one query head is ([partition] diagnostics, judged
+    against dense outputs): R = Od - Os over all rows, and the least-squares affine map of the
+    sparse output R ~ A Os + b (no penalty). Returns
+      explained  = 1 - SSE / sum ||R_i - mean R||^2   (affine-explainable fraction)
+      orthogonal = SSE / sum ||R_i||^2                 (affine-orthogonal energy)
+    with SSE the residual energy of that fit (reading: the page names both and gives no formula)."""
+    Os = np.asarray(Os, dtype=np.float64)
+    R = np.asarray(Od, dtype=np.float64) - Os
+    X = np.concatenate([Os, np.ones((Os.shape[0], 1))], axis=1)
+    beta, *_ = np.linalg.lstsq(X, R, rcond=None)
+    sse = float(((R - X @ beta) ** 2).sum())
+    centred = float(((R - R.mean(axis=0)) ** 2).sum())
+    total = float((R ** 2).sum())
+    return 1.0 - sse / centred, sse / total
 
 
 def correction(Os: np.ndarray, U: np.ndarray, A: np.ndarray, obar: np.ndarray, Rbar: np.ndarray,

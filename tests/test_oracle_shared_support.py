@@ -130,3 +130,24 @@ def test_semantic_partition_groups_raw_activations():
     assert same(hp.kgroup, lab) and same(hp.qgroup, qlab)
     assert np.allclose(hp.features, Kh.astype(np.float32))
     assert np.allclose(hp.ycoord, Qg.mean(axis=0).astype(np.float32))
+
+
+def test_affine_diagnostics_planted():
+    """Residual = affine map of the sparse output + a part orthogonal to every affine function of
+    it: the fit recovers the map, so the unexplained energy is exactly that part's energy."""
+    rng = np.random.default_rng(4)
+    n, d = 400, 6
+    Os = rng.standard_normal((n, d))
+    A = rng.standard_normal((d, d))
+    b = rng.standard_normal(d)
+    X = np.concatenate([Os, np.ones((n, 1))], axis=1)
+    E = rng.standard_normal((n, d))
+    Qx, _ = np.linalg.qr(X)
+    E -= Qx @ (Qx.T @ E)                                   # orthogonal to the columns of [Os, 1]
+    R = Os @ A.T + b + E
+    explained, orthogonal = oracle.affine_diagnostics(Os, Os + R)
+    sse = (E ** 2).sum()
+    assert explained == pytest.approx(1 - sse / ((R - R.mean(axis=0)) ** 2).sum(), rel=1e-9)
+    assert orthogonal == pytest.approx(sse / (R ** 2).sum(), rel=1e-9)
+    ex0, or0 = oracle.affine_diagnostics(Os, Os + Os @ A.T + b)       # purely affine residual
+    assert ex0 == pytest.approx(1.0, abs=1e-12) and or0 == pytest.approx(0.0, abs=1e-12)
