@@ -108,6 +108,8 @@ def load_library() -> ctypes.CDLL:
         "sparsepr_shared_support_workspace": (st, [H, ctypes.POINTER(ctypes.c_size_t),
                                                    ctypes.POINTER(ctypes.c_size_t)]),
         "sparsepr_shared_support": (st, [H, _p, _p, ctypes.POINTER(Partition), _p, _p, _p, ctypes.c_size_t, _p]),
+        "sparsepr_affine_diagnostics_workspace": (st, [H, ctypes.POINTER(ctypes.c_size_t)]),
+        "sparsepr_affine_diagnostics": (st, [H, _p, _p, _p, _p, ctypes.c_size_t, _p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -254,6 +256,30 @@ class SparsePR:
                self.lib.sparsepr_shared_support(self.h, _ptr(Q), _ptr(K), ctypes.byref(part), _ptr(row_frac),
                                                 _ptr(union_frac), _ptr(ws), nbytes, _stream(stream)))
         return row_frac, union_frac
+
+    def affine_diagnostics(self, Q, K, V, stream=None):
+        """Affine-explainable fraction and affine-orthogonal energy of each query head's hard-drop
+        residual (dense output minus the uncorrected sparse output), as a [B*Hq, 2] fp64 device
+        tensor; runs the partition, routing, sparse attention and the dense baseline."""
+        import torch
+
+        part = self.partition(Q, K, stream)
+        route = self.route(Q, part, stream)
+        Qp, Kp, Vp, Osp = (torch.empty_like(t) for t in (Q, K, V, Q))
+        self.permute(Q, K, V, part, Qp, Kp, Vp, stream)
+        self.blocksparse_attn(Qp, Kp, Vp, part, route, Osp, None, stream)
+        Os, Od = torch.empty_like(Q), torch.empty_like(Q)
+        self.writeback(part, Osp, None, Os, stream)
+        self.dense_attn(Q, K, V, Od, stream)
+        n = ctypes.c_size_t()
+        _check("sparsepr_affine_diagnostics_workspace",
+               self.lib.sparsepr_affine_diagnostics_workspace(self.h, ctypes.byref(n)))
+        ws = torch.empty(n.value, dtype=torch.uint8, device="cuda")
+        out = torch.empty((self.cfg.B * self.cfg.Hq, 2), dtype=torch.float64, device="cuda")
+        _check("sparsepr_affine_diagnostics",
+               self.lib.sparsepr_affine_diagnostics(self.h, _ptr(Os), _ptr(Od), _ptr(out), _ptr(ws), n.value,
+                                                    _stream(stream)))
+        return out, Os, Od
 
     def writeback(self, part: Partition, Osp, fit: Fit | None, O, stream=None):
         _check("sparsepr_writeback", self.lib.sparsepr_writeback(self.h, ctypes.byref(part), _ptr(Osp),

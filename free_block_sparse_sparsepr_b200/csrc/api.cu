@@ -373,7 +373,7 @@ sparsepr_status probe_fit_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
 sparsepr_status writeback_impl(sparsepr_handle h, const sparsepr_partition_t* p, const bf16* Osp,
                                const sparsepr_fit_t* f, bf16* O, cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
-    const bool correct = h->M > 0;
+    const bool correct = h->M > 0 && f != nullptr;
     if (correct && (c.flags & SPARSEPR_FLAG_RIDGE_ONLY)) {
         SPR_TRY(spr::launch_writeback_ridge(Osp, p->qperm, f->A, f->obar, f->Rbar, O, h->Hp, h->g, c.N, c.d,
                                             h->num_sms, s));
@@ -523,6 +523,24 @@ size_t shared_head_bytes(sparsepr_handle h) {
 }
 }  // namespace
 
+sparsepr_status sparsepr_affine_diagnostics_workspace(sparsepr_handle h, size_t* bytes) {
+    if (!h || !bytes) return SPARSEPR_ERR_INVALID_ARG;
+    *bytes = spr::affine_diag_workspace(h->Hp, h->cfg.d);
+    return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_affine_diagnostics(sparsepr_handle h, const void* Os, const void* Od, double* out,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+    if (!h || !aligned16(Os) || !aligned16(Od) || !out || !workspace) return SPARSEPR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 7u) != 0) return SPARSEPR_ERR_INVALID_ARG;
+    if (workspace_bytes < spr::affine_diag_workspace(h->Hp, h->cfg.d)) return SPARSEPR_ERR_WORKSPACE;
+    h->launches = 0;
+    SPR_TRY(spr::launch_affine_diag(static_cast<const bf16*>(Os), static_cast<const bf16*>(Od), out, workspace,
+                                    h->Hp, h->cfg.N, h->cfg.d, h->dev_status, as_stream(stream)));
+    ++h->launches;   // the Gram and the solve kernels
+    return SPARSEPR_OK;
+}
+
 sparsepr_status sparsepr_shared_support_workspace(sparsepr_handle h, size_t* min_bytes, size_t* all_bytes) {
     if (!h || (!min_bytes && !all_bytes)) return SPARSEPR_ERR_INVALID_ARG;
     if (min_bytes) *min_bytes = shared_rows_bytes(h) + shared_head_bytes(h);
@@ -626,8 +644,8 @@ sparsepr_status sparsepr_writeback(sparsepr_handle h, const sparsepr_partition_t
     if (!h || !aligned16(Osp) || !aligned16(O)) return SPARSEPR_ERR_INVALID_ARG;
     sparsepr_status st = check_partition(part, h->M > 0);
     if (st) return st;
-    if (h->M && (!fit || !fit->U || !fit->Bm || !fit->c0 || !fit->Odense)) return SPARSEPR_ERR_INVALID_ARG;
-    if (h->M && (h->cfg.flags & (SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED)) &&
+    if (h->M && fit && (!fit->U || !fit->Bm || !fit->c0 || !fit->Odense)) return SPARSEPR_ERR_INVALID_ARG;
+    if (h->M && fit && (h->cfg.flags & (SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED)) &&
         (!fit->A || !fit->obar || !fit->Rbar))
         return SPARSEPR_ERR_INVALID_ARG;
     h->launches = 0;

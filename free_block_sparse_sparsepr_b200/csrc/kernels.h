@@ -73,6 +73,10 @@ cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long coun
 // Support diagnostic: out[z][s] = (smallest k whose k largest exp(F[.][s] - max) hold 90% of the
 // row's softmax mass) / N, for s < S; F [P][N][DP] fp32 (DP a multiple of 8, S <= DP).
 cudaError_t launch_topmass(const float* F, float* out, int P, int N, int DP, int S, cudaStream_t s);
+// Affine diagnostics: per query head, [explained fraction, orthogonal energy] of R = Od - Os.
+size_t affine_diag_workspace(int Hp, int d);
+cudaError_t launch_affine_diag(const bf16* Os, const bf16* Od, double* out, void* ws, int Hp, int N, int d,
+                               int* status, cudaStream_t s);
 // Shared-route support: Qsh [P][Gq][8][d] bf16 gathered rows (zero past R' of each group), then
 // for KV heads z0..z0+nz-1 the row-major logits Z [nz][Gq*8][ldz] give row_frac [P][Gq][8] and
 // union_frac [P][Gq].

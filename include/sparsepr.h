@@ -273,6 +273,8 @@ sparsepr_status sparsepr_probe_fit(sparsepr_handle h, const void* Q, const void*
  * Step (7) [probe and execution paragraphs]: O[qperm[p]] = Osp[p] + delta(Osp[p])
  * for every group-major row p, then the probe rows are overwritten with
  * their dense outputs. O: bf16 [B][Hq][N][d], original order, caller-owned.
+ * fit = NULL: the rows only return to the original order (no correction, no
+ * probe override), e.g. for sparsepr_affine_diagnostics.
  */
 sparsepr_status sparsepr_writeback(sparsepr_handle h, const sparsepr_partition_t* part,
                                    const void* Osp, const sparsepr_fit_t* fit, void* O, void* stream);
@@ -318,6 +320,24 @@ sparsepr_status sparsepr_shared_support_workspace(sparsepr_handle h, size_t* min
 sparsepr_status sparsepr_shared_support(sparsepr_handle h, const void* Q, const void* K,
                                         const sparsepr_partition_t* part, float* row_frac, float* union_frac,
                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Affine diagnostics of the hard-drop residual [partition paragraph: the residual of a
+ * response-coupled partition is closer to an affine function of the sparse output]. For every
+ * query head x, R = Od - Os over all N rows and the least-squares affine fit R ~ A Os + b
+ * (fp64 throughout). out[2x] = 1 - SSE / sum_i ||R_i - mean R||^2 (affine-explainable
+ * fraction), out[2x+1] = SSE / sum_i ||R_i||^2 (affine-orthogonal energy); NaN (and
+ * SPARSEPR_DEV_BOUNDS in the device status) if [Os, 1] is rank deficient.
+ *   Os, Od     bf16 [B][Hq][N][d], device, original row order: the uncorrected sparse output
+ *              (e.g. sparsepr_blocksparse_attn followed by sparsepr_writeback with fit = NULL)
+ *              and the dense output (sparsepr_dense_attn)
+ *   out        double [B*Hq][2], device
+ *   workspace  caller-owned device memory of sparsepr_affine_diagnostics_workspace bytes
+ *              (8-byte aligned)
+ */
+sparsepr_status sparsepr_affine_diagnostics_workspace(sparsepr_handle h, size_t* bytes);
+sparsepr_status sparsepr_affine_diagnostics(sparsepr_handle h, const void* Os, const void* Od, double* out,
+                                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* Dense softmax attention (scale 1/sqrt(d)) of every query over all keys: the baseline. */
 sparsepr_status sparsepr_dense_attn(sparsepr_handle h, const void* Q, const void* K, const void* V,

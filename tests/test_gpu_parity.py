@@ -376,6 +376,42 @@ def test_head_shards_reproduce_the_call(name):
 
 
 @pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
+def test_affine_diagnostics_match_oracle(name):
+    """Affine diagnostics of the hard-drop residual: on the GPU's own uncorrected sparse output
+    and dense output, the explained fraction and the orthogonal energy equal the oracle's
+    least-squares formula (fp64 on both sides); the sparse output handed to it is the group-major
+    output returned to the original order, and the dense one the dense kernel's."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    with spr.SparsePR.from_workload(w) as h:
+        out, Os, Od = h.affine_diagnostics(q, k, v)
+        part = h.partition(q, k)
+        route = h.route(q, part)
+        Qp, Kp, Vp, Osp = (torch.empty_like(t) for t in (q, k, v, q))
+        h.permute(q, k, v, part, Qp, Kp, Vp)
+        h.blocksparse_attn(Qp, Kp, Vp, part, route, Osp)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0
+        qperm = h.partition_views(part)["qperm"].long()
+        Od2 = h.dense_attn(q, k, v)
+        torch.cuda.synchronize()
+    assert torch.equal(Od, Od2)
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            z = b * w.Hkv + hq // w.g
+            back = torch.empty_like(Osp[b, hq])
+            back[qperm[z]] = Osp[b, hq]
+            assert torch.equal(Os[b, hq], back)
+    o = out.cpu().numpy()
+    Osf, Odf = bf16_to_f64(Os), bf16_to_f64(Od)
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            x = b * w.Hq + hq
+            ex, orth = oracle.affine_diagnostics(Osf[b, hq], Odf[b, hq])
+            assert abs(o[x, 0] - ex) <= 1e-6 and abs(o[x, 1] - orth) <= 1e-6, (x, o[x], ex, orth)
+            assert 0.0 <= o[x, 1] <= 1.0 and o[x, 0] <= 1.0
+
+
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
 def test_semantic_partition_ablation(name):
     """The semantic-partition ablation of [partition] (k-means on the raw keys and the raw mean
     query): the GPU's groups agree with the oracle's where the assignment margin is clear, its
