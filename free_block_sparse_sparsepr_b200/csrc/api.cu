@@ -29,7 +29,21 @@ inline int pad64(int v) { return (v + 63) / 64 * 64; }
 
 enum Stage { kStPartition = 0, kStRoute, kStPermute, kStAttn, kStProbeFit, kStWriteback, kStUnused, kStTotal, kNumStages };
 
+constexpr int kHostChunks = 4;     // KV-head chunks of the host-buffer pipeline
+
 }  // namespace
+
+// Host-buffer pipeline: one sub-handle per contiguous chunk of flattened KV heads (every step is
+// per KV head, so the chunks reproduce the whole call), with the copies in, the chunk calls and
+// the copies out on three streams so that transfers overlap the compute of other chunks.
+struct HostPipe {
+    int nc = 0;
+    int z0[kHostChunks + 1] = {};
+    sparsepr_handle_s* sub[kHostChunks] = {};
+    cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, end_comp = nullptr, end_out = nullptr;
+    cudaEvent_t ev_in[kHostChunks] = {}, ev_done[kHostChunks] = {};
+};
 
 struct sparsepr_handle_s {
     sparsepr_config cfg;
@@ -63,6 +77,7 @@ struct sparsepr_handle_s {
     int* dev_status = nullptr;
     // host-buffer variant staging (allocated on first use)
     bf16 *sQ = nullptr, *sK = nullptr, *sV = nullptr, *sO = nullptr;
+    struct HostPipe* pipe = nullptr;   // host-buffer pipeline over KV-head chunks (first use)
     // timing
     cudaEvent_t ev[kNumStages + 1] = {};
     cudaEvent_t done_ev = nullptr;
@@ -486,9 +501,25 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     return SPARSEPR_OK;
 }
 
+static void destroy_pipe(HostPipe* pp) {
+    if (!pp) return;
+    for (int i = 0; i < pp->nc; ++i)
+        if (pp->sub[i]) sparsepr_destroy(pp->sub[i]);
+    for (cudaStream_t st : {pp->in, pp->comp, pp->out})
+        if (st) cudaStreamDestroy(st);
+    for (cudaEvent_t e : {pp->start, pp->end_comp, pp->end_out})
+        if (e) cudaEventDestroy(e);
+    for (int i = 0; i < kHostChunks; ++i) {
+        if (pp->ev_in[i]) cudaEventDestroy(pp->ev_in[i]);
+        if (pp->ev_done[i]) cudaEventDestroy(pp->ev_done[i]);
+    }
+    delete pp;
+}
+
 sparsepr_status sparsepr_destroy(sparsepr_handle h) {
     if (!h) return SPARSEPR_OK;
     cudaDeviceSynchronize();
+    destroy_pipe(h->pipe);
     if (h->sQ) { cudaFree(h->sQ); cudaFree(h->sK); cudaFree(h->sV); cudaFree(h->sO); }
     free_all(h);
     delete h;
@@ -704,14 +735,92 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
         h->sQ = static_cast<bf16*>(a); h->sK = static_cast<bf16*>(b);
         h->sV = static_cast<bf16*>(cc); h->sO = static_cast<bf16*>(dd);
     }
+    if (!h->pipe) {
+        HostPipe* pp = new (std::nothrow) HostPipe();
+        if (!pp) return SPARSEPR_ERR_WORKSPACE;
+        pp->nc = h->P < kHostChunks ? h->P : kHostChunks;
+        const int base = h->P / pp->nc, extra = h->P % pp->nc;
+        for (int i = 0; i < pp->nc; ++i) pp->z0[i + 1] = pp->z0[i] + base + (i < extra ? 1 : 0);
+        bool ok = true;
+        for (int i = 0; i < pp->nc && ok; ++i) {
+            sparsepr_config sc = c;
+            sc.B = 1;
+            sc.Hkv = pp->z0[i + 1] - pp->z0[i];
+            sc.Hq = sc.Hkv * h->g;
+            sc.flags &= ~SPARSEPR_FLAG_STAGE_TIMING;
+            ok = sparsepr_create(&sc, &pp->sub[i]) == SPARSEPR_OK;
+        }
+        ok = ok && cudaStreamCreateWithFlags(&pp->in, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&pp->comp, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&pp->out, cudaStreamNonBlocking) == cudaSuccess;
+        for (cudaEvent_t* e : {&pp->start, &pp->end_comp, &pp->end_out})
+            ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; i < pp->nc && ok; ++i)
+            ok = cudaEventCreateWithFlags(&pp->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&pp->ev_done[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            destroy_pipe(pp);
+            return SPARSEPR_ERR_WORKSPACE;
+        }
+        h->pipe = pp;
+    }
+    HostPipe* pp = h->pipe;
     cudaStream_t s = as_stream(stream);
-    if (cudaMemcpyAsync(h->sQ, Q, qb, cudaMemcpyHostToDevice, s) || cudaMemcpyAsync(h->sK, K, kb, cudaMemcpyHostToDevice, s) ||
-        cudaMemcpyAsync(h->sV, V, kb, cudaMemcpyHostToDevice, s))
+    const size_t qh = (size_t)h->g * c.N * c.d, kh = (size_t)c.N * c.d;   // elements per KV head
+    const bf16* hQ = static_cast<const bf16*>(Q);
+    const bf16* hK = static_cast<const bf16*>(K);
+    const bf16* hV = static_cast<const bf16*>(V);
+    bf16* hO = static_cast<bf16*>(O);
+    bool ok = cudaEventRecord(pp->start, s) == cudaSuccess;
+    for (cudaStream_t st : {pp->in, pp->comp, pp->out}) ok = ok && cudaStreamWaitEvent(st, pp->start, 0) == cudaSuccess;
+    // every chunk's inputs in order on the copy-in stream
+    for (int i = 0; i < pp->nc && ok; ++i) {
+        const size_t z = pp->z0[i], n = pp->z0[i + 1] - pp->z0[i];
+        ok = cudaMemcpyAsync(h->sQ + z * qh, hQ + z * qh, n * qh * sizeof(bf16), cudaMemcpyHostToDevice, pp->in) ==
+                 cudaSuccess &&
+             cudaMemcpyAsync(h->sK + z * kh, hK + z * kh, n * kh * sizeof(bf16), cudaMemcpyHostToDevice, pp->in) ==
+                 cudaSuccess &&
+             cudaMemcpyAsync(h->sV + z * kh, hV + z * kh, n * kh * sizeof(bf16), cudaMemcpyHostToDevice, pp->in) ==
+                 cudaSuccess &&
+             cudaEventRecord(pp->ev_in[i], pp->in) == cudaSuccess;
+    }
+    // each chunk's call once its inputs have landed, its output copied back behind it
+    int launches = 0;
+    for (int i = 0; i < pp->nc && ok; ++i) {
+        const size_t z = pp->z0[i], n = pp->z0[i + 1] - pp->z0[i];
+        ok = cudaStreamWaitEvent(pp->comp, pp->ev_in[i], 0) == cudaSuccess;
+        if (ok && sparsepr_attention(pp->sub[i], h->sQ + z * qh, h->sK + z * kh, h->sV + z * kh, h->sO + z * qh,
+                                     pp->comp) != SPARSEPR_OK)
+            ok = false;
+        launches += pp->sub[i]->launches;
+        ok = ok && cudaMemcpyAsync(h->pairs + z, pp->sub[i]->pairs, n * sizeof(int64_t), cudaMemcpyDeviceToDevice,
+                                   pp->comp) == cudaSuccess;
+        ok = ok && cudaEventRecord(pp->ev_done[i], pp->comp) == cudaSuccess &&
+             cudaStreamWaitEvent(pp->out, pp->ev_done[i], 0) == cudaSuccess &&
+             cudaMemcpyAsync(hO + z * qh, h->sO + z * qh, n * qh * sizeof(bf16), cudaMemcpyDeviceToHost, pp->out) ==
+                 cudaSuccess;
+    }
+    ok = ok && cudaEventRecord(pp->end_comp, pp->comp) == cudaSuccess &&
+         cudaEventRecord(pp->end_out, pp->out) == cudaSuccess && cudaStreamWaitEvent(s, pp->end_comp, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(s, pp->end_out, 0) == cudaSuccess;
+    // the caller's stream waits for every chunk even after an error, so no copy outlives the call
+    cudaStreamWaitEvent(s, pp->end_comp, 0);
+    if (cudaStreamSynchronize(s) != cudaSuccess || cudaStreamSynchronize(pp->in) != cudaSuccess ||
+        cudaStreamSynchronize(pp->out) != cudaSuccess || !ok)
         return SPARSEPR_ERR_CUDA;
-    sparsepr_status st = sparsepr_attention(h, h->sQ, h->sK, h->sV, h->sO, stream);
-    if (st) return st;
-    if (cudaMemcpyAsync(O, h->sO, qb, cudaMemcpyDeviceToHost, s)) return SPARSEPR_ERR_CUDA;
-    if (cudaStreamSynchronize(s)) return SPARSEPR_ERR_CUDA;
+    // statistics and the device status of the chunk calls on the handle
+    int worst = 0;
+    for (int i = 0; i < pp->nc; ++i) {
+        int ds = 0;
+        if (cudaMemcpy(&ds, pp->sub[i]->dev_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+            return SPARSEPR_ERR_CUDA;
+        if (ds && !worst) worst = ds;
+    }
+    if (worst && cudaMemcpy(h->dev_status, &worst, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return SPARSEPR_ERR_CUDA;
+    cudaEventRecord(h->done_ev, s);
+    h->timed_call = false;
+    h->launches = launches;
     return SPARSEPR_OK;
 }
 

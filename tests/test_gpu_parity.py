@@ -375,6 +375,27 @@ def test_head_shards_reproduce_the_call(name):
     assert torch.equal(torch.cat(parts), O_full)
 
 
+@pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000", "proj_n4096"])
+def test_host_call_matches_device_call(name):
+    """sparsepr_attention_host (host buffers; the KV heads run in chunks whose copies overlap the
+    other chunks' compute) returns the device call's output bit for bit, with the same realised
+    density and a clean device status."""
+    w, (Q, K, V), (q, k, v), res = _setup(name)
+    with spr.SparsePR.from_workload(w) as h:
+        O_dev = h.attention(q, k, v)
+        torch.cuda.synchronize()
+        st_dev = h.stats()
+        pin = [t.cpu().pin_memory() for t in (q, k, v)]
+        Oh = torch.empty_like(pin[0]).pin_memory()
+        for _ in range(2):                                     # the second call reuses the chunk handles
+            Oh.zero_()
+            h.attention_host(*pin, Oh)
+            assert torch.equal(Oh, O_dev.cpu())
+        st = h.stats()
+        assert st["device_status"] == 0 and h.last_launch_count() > 10
+        assert st["rho_exec"] == st_dev["rho_exec"]
+
+
 @pytest.mark.parametrize("name", ["mid_n16384_h4", "ragged_gqa_n1000"])
 def test_affine_diagnostics_match_oracle(name):
     """Affine diagnostics of the hard-drop residual: on the GPU's own uncorrected sparse output
