@@ -40,8 +40,8 @@ struct HostPipe {
     int nc = 0;
     int z0[kHostChunks + 1] = {};
     sparsepr_handle_s* sub[kHostChunks] = {};
-    cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
-    cudaEvent_t start = nullptr, end_comp = nullptr, end_out = nullptr;
+    cudaStream_t in = nullptr, comp[2] = {}, out = nullptr;   // chunks alternate between two compute streams
+    cudaEvent_t start = nullptr, end_comp[2] = {}, end_out = nullptr;
     cudaEvent_t ev_in[kHostChunks] = {}, ev_done[kHostChunks] = {};
 };
 
@@ -505,9 +505,9 @@ static void destroy_pipe(HostPipe* pp) {
     if (!pp) return;
     for (int i = 0; i < pp->nc; ++i)
         if (pp->sub[i]) sparsepr_destroy(pp->sub[i]);
-    for (cudaStream_t st : {pp->in, pp->comp, pp->out})
+    for (cudaStream_t st : {pp->in, pp->comp[0], pp->comp[1], pp->out})
         if (st) cudaStreamDestroy(st);
-    for (cudaEvent_t e : {pp->start, pp->end_comp, pp->end_out})
+    for (cudaEvent_t e : {pp->start, pp->end_comp[0], pp->end_comp[1], pp->end_out})
         if (e) cudaEventDestroy(e);
     for (int i = 0; i < kHostChunks; ++i) {
         if (pp->ev_in[i]) cudaEventDestroy(pp->ev_in[i]);
@@ -751,9 +751,10 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
             ok = sparsepr_create(&sc, &pp->sub[i]) == SPARSEPR_OK;
         }
         ok = ok && cudaStreamCreateWithFlags(&pp->in, cudaStreamNonBlocking) == cudaSuccess &&
-             cudaStreamCreateWithFlags(&pp->comp, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&pp->comp[0], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&pp->comp[1], cudaStreamNonBlocking) == cudaSuccess &&
              cudaStreamCreateWithFlags(&pp->out, cudaStreamNonBlocking) == cudaSuccess;
-        for (cudaEvent_t* e : {&pp->start, &pp->end_comp, &pp->end_out})
+        for (cudaEvent_t* e : {&pp->start, &pp->end_comp[0], &pp->end_comp[1], &pp->end_out})
             ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
         for (int i = 0; i < pp->nc && ok; ++i)
             ok = cudaEventCreateWithFlags(&pp->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
@@ -772,7 +773,8 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
     const bf16* hV = static_cast<const bf16*>(V);
     bf16* hO = static_cast<bf16*>(O);
     bool ok = cudaEventRecord(pp->start, s) == cudaSuccess;
-    for (cudaStream_t st : {pp->in, pp->comp, pp->out}) ok = ok && cudaStreamWaitEvent(st, pp->start, 0) == cudaSuccess;
+    for (cudaStream_t st : {pp->in, pp->comp[0], pp->comp[1], pp->out})
+        ok = ok && cudaStreamWaitEvent(st, pp->start, 0) == cudaSuccess;
     // every chunk's inputs in order on the copy-in stream
     for (int i = 0; i < pp->nc && ok; ++i) {
         const size_t z = pp->z0[i], n = pp->z0[i + 1] - pp->z0[i];
@@ -784,30 +786,34 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
                  cudaSuccess &&
              cudaEventRecord(pp->ev_in[i], pp->in) == cudaSuccess;
     }
-    // each chunk's call once its inputs have landed, its output copied back behind it
+    // each chunk's call once its inputs have landed (consecutive chunks on alternate compute
+    // streams, so one chunk's latency-bound kernels overlap the other's), its output copied back
     int launches = 0;
     for (int i = 0; i < pp->nc && ok; ++i) {
         const size_t z = pp->z0[i], n = pp->z0[i + 1] - pp->z0[i];
-        ok = cudaStreamWaitEvent(pp->comp, pp->ev_in[i], 0) == cudaSuccess;
+        cudaStream_t cs = pp->comp[i & 1];
+        ok = cudaStreamWaitEvent(cs, pp->ev_in[i], 0) == cudaSuccess;
         if (ok && sparsepr_attention(pp->sub[i], h->sQ + z * qh, h->sK + z * kh, h->sV + z * kh, h->sO + z * qh,
-                                     pp->comp) != SPARSEPR_OK)
+                                     cs) != SPARSEPR_OK)
             ok = false;
         launches += pp->sub[i]->launches;
         ok = ok && cudaMemcpyAsync(h->pairs + z, pp->sub[i]->pairs, n * sizeof(int64_t), cudaMemcpyDeviceToDevice,
-                                   pp->comp) == cudaSuccess;
-        ok = ok && cudaEventRecord(pp->ev_done[i], pp->comp) == cudaSuccess &&
+                                   cs) == cudaSuccess;
+        ok = ok && cudaEventRecord(pp->ev_done[i], cs) == cudaSuccess &&
              cudaStreamWaitEvent(pp->out, pp->ev_done[i], 0) == cudaSuccess &&
              cudaMemcpyAsync(hO + z * qh, h->sO + z * qh, n * qh * sizeof(bf16), cudaMemcpyDeviceToHost, pp->out) ==
                  cudaSuccess;
     }
-    ok = ok && cudaEventRecord(pp->end_comp, pp->comp) == cudaSuccess &&
-         cudaEventRecord(pp->end_out, pp->out) == cudaSuccess && cudaStreamWaitEvent(s, pp->end_comp, 0) == cudaSuccess &&
+    for (int k = 0; k < 2; ++k)
+        ok = ok && cudaEventRecord(pp->end_comp[k], pp->comp[k]) == cudaSuccess &&
+             cudaStreamWaitEvent(s, pp->end_comp[k], 0) == cudaSuccess;
+    ok = ok && cudaEventRecord(pp->end_out, pp->out) == cudaSuccess &&
          cudaStreamWaitEvent(s, pp->end_out, 0) == cudaSuccess;
-    // the caller's stream waits for every chunk even after an error, so no copy outlives the call
-    cudaStreamWaitEvent(s, pp->end_comp, 0);
-    if (cudaStreamSynchronize(s) != cudaSuccess || cudaStreamSynchronize(pp->in) != cudaSuccess ||
-        cudaStreamSynchronize(pp->out) != cudaSuccess || !ok)
-        return SPARSEPR_ERR_CUDA;
+    // every internal stream drains before returning, even after an error, so no work outlives the call
+    bool drained = cudaStreamSynchronize(s) == cudaSuccess;
+    for (cudaStream_t st : {pp->in, pp->comp[0], pp->comp[1], pp->out})
+        drained = cudaStreamSynchronize(st) == cudaSuccess && drained;
+    if (!drained || !ok) return SPARSEPR_ERR_CUDA;
     // statistics and the device status of the chunk calls on the handle
     int worst = 0;
     for (int i = 0; i < pp->nc; ++i) {
