@@ -46,12 +46,24 @@ def _cfg(**kw):
     (dict(M=0), 1), (dict(M=65), 2), (dict(r=0), 1), (dict(r=65), 1), (dict(lam=0.0), 1),
     (dict(rho_exec=0.0), 1), (dict(rho_exec=float("nan")), 1), (dict(kmeans_iters=-1), 1),
     (dict(flags=1 << 20), 1),
+    (dict(flags=spr.FLAG_PROBES_UNIFORM | spr.FLAG_PROBES_RANDOM), 1),      # one probe sampler at most
+    (dict(flags=spr.FLAG_SEMANTIC_PARTITION | spr.FLAG_TOPMASS), 1),        # no sampled responses to measure
 ])
 def test_create_rejects_bad_configs_without_gpu(kw, code):
     lib = spr.load_library()
     h = ctypes.c_void_p()
     assert lib.sparsepr_create(ctypes.byref(_cfg(**kw)), ctypes.byref(h)) == code
     assert not h.value
+
+
+def test_diagnostic_entry_points_reject_null_arguments():
+    lib = spr.load_library()
+    n = ctypes.c_size_t()
+    assert lib.sparsepr_shared_support_workspace(None, ctypes.byref(n), None) == 1
+    assert lib.sparsepr_shared_support(None, None, None, None, None, None, None, 0, None) == 1
+    assert lib.sparsepr_affine_diagnostics_workspace(None, ctypes.byref(n)) == 1
+    assert lib.sparsepr_affine_diagnostics(None, None, None, None, None, 0, None) == 1
+    assert lib.sparsepr_attention_host(None, None, None, None, None, None) == 1
 
 
 def test_null_handle_and_pointer_checks():
