@@ -165,50 +165,80 @@ def measured_peaks() -> dict:
 
 # ----------------------------------------------------------------------------- oracle (CPU) sample
 
-def oracle_sample_seconds(w, n_groups: int = 4):
-    """Time the CPU oracle on one KV head of workload w and scale to one whole call.
+CPU_SAMPLE_GROUPS = 8          # query groups of the fixed attention sample
+CPU_WHOLE_HEAD_N = 16384       # up to this length the sample attends every query group (no scaling)
+_SAMPLE_INPUTS = {}
 
-    The sample: the full partition and route of KV head 0 (all N rows), then exact
-    sparse attention for `n_groups` query groups, the M dense probe rows, the
-    ridge fit and the correction of those groups. Per call = Hkv * (partition +
-    route + fit + attention_sample * Gq / n_groups) for each of the g query heads.
+
+def sample_groups(Gq: int, n: int = CPU_SAMPLE_GROUPS) -> np.ndarray:
+    """The fixed, stratified query-group sample: groups floor((2i + 1) Gq / 2n), i < n (group ids
+    follow the k-means seeds, which are spread evenly over the token order)."""
+    n = min(n, Gq)
+    return np.array([((2 * i + 1) * Gq) // (2 * n) for i in range(n)], dtype=np.int64)
+
+
+def oracle_sample(w):
+    """Time the CPU oracle on one fixed sample of workload w and scale it to one whole call.
+
+    The sample is KV head 0 with all its query heads: its whole partition and route (all N rows),
+    exact sparse attention for the rows of CPU_SAMPLE_GROUPS fixed query groups (sample_groups;
+    every query group, so no scaling, when N <= CPU_WHOLE_HEAD_N),
+    the sparse output at the M probe rows, the probe fit (dense probe rows, ridge, subspace) and
+    the correction of an N x d output. Only the sampled attention is scaled, by routed pairs (the
+    head's routed pairs over the sampled groups' routed pairs: the attention work is proportional
+    to pairs, not rows); every other stage is timed whole. One call = B*Hkv such KV heads.
+    Returns (seconds per call, per-stage seconds of the sample, sample description).
     """
     import oracle
     from synthetic import bf16_bits_to_f64, video_qkv
 
     one = w.replace(B=1, Hq=w.g, Hkv=1)
-    Qb, Kb, Vb = video_qkv(one)
-    Q, K, V = (bf16_bits_to_f64(x) for x in (Qb, Kb, Vb))
+    if one not in _SAMPLE_INPUTS:
+        _SAMPLE_INPUTS.clear()
+        _SAMPLE_INPUTS[one] = tuple(bf16_bits_to_f64(x) for x in video_qkv(one))
+    Q, K, V = _SAMPLE_INPUTS[one]
     Qg, Kh, Vh = Q[0], K[0, 0], V[0, 0]
+    st = dict.fromkeys(("partition", "route", "attention_sample", "probe_rows_sparse", "fit", "correction"), 0.0)
     t0 = time.perf_counter()
     part = oracle.partition_head(Qg, Kh, one)
     t1 = time.perf_counter()
     rt = oracle.route_head(Qg, part, one)
     t2 = time.perf_counter()
-    groups = np.unique(part.qgroup)[:n_groups]
+    st["partition"], st["route"] = t1 - t0, t2 - t1
+    groups = np.arange(w.Gq) if w.N <= CPU_WHOLE_HEAD_N else sample_groups(w.Gq)
     rows = np.nonzero(np.isin(part.qgroup, groups))[0]
-    t_attn = t_fit = 0.0
+    qsize, ksize = np.diff(part.qoff), np.diff(part.koff)
+    sampled_pairs = int((qsize[groups] * (rt.sel[groups] * ksize[None, :]).sum(axis=1)).sum())
     for j in range(w.g):
         ta = time.perf_counter()
-        o, _ = oracle.sparse_attention(Qg[j], Kh, Vh, part.qgroup, part.kgroup, rt.sel,
-                                       rows=np.union1d(rows, part.probe))
+        o_rows, _ = oracle.sparse_attention(Qg[j], Kh, Vh, part.qgroup, part.kgroup, rt.sel, rows=rows)
         tb = time.perf_counter()
-        fit = oracle.fit_head(Qg[j], Kh, Vh, o[part.probe], part, one)
-        oracle.correction(o[rows], fit.U, fit.A, fit.obar, fit.Rbar)
+        o_probe, _ = oracle.sparse_attention(Qg[j], Kh, Vh, part.qgroup, part.kgroup, rt.sel, rows=part.probe)
         tc = time.perf_counter()
-        t_attn += tb - ta
-        t_fit += tc - tb
-    sample_s = tc - t0
-    frac = len(rows) / float(w.N)
-    per_head = (t1 - t0) + (t2 - t1) + t_fit + t_attn / max(frac, 1e-12)
+        fit = oracle.fit_head(Qg[j], Kh, Vh, o_probe[part.probe], part, one)
+        td = time.perf_counter()
+        o_full = np.resize(o_rows[rows], (w.N, w.d))       # an N x d output: the correction's cost
+        oracle.correction(o_full, fit.U, fit.A, fit.obar, fit.Rbar)
+        te = time.perf_counter()
+        st["attention_sample"] += tb - ta
+        st["probe_rows_sparse"] += tc - tb
+        st["fit"] += td - tc
+        st["correction"] += te - td
+    scale = rt.pairs / max(sampled_pairs, 1)
+    per_head = (st["partition"] + st["route"] + st["attention_sample"] * scale + st["probe_rows_sparse"]
+                + st["fit"] + st["correction"])
     per_call = per_head * w.Hkv * w.B
-    desc = (f"KV head 0 of {w.name}: full partition + route, exact attention/fit/correction for "
-            f"{len(groups)} of {w.Gq} query groups ({len(rows)} rows) on each of its {w.g} query heads; "
-            f"scaled by rows and by {w.B * w.Hkv} KV heads")
-    return per_call, sample_s, desc
+    which = ("every query group" if len(groups) == w.Gq else
+             f"query groups {groups.tolist()} of {w.Gq} ({len(rows)} rows, {sampled_pairs} of {rt.pairs} routed pairs), "
+             "scaled by routed pairs")
+    desc = (f"KV head 0 of {w.name} with its {w.g} query head(s): whole partition, route, probe rows, fit and "
+            f"correction; exact sparse attention for {which}; x {w.B * w.Hkv} KV heads")
+    stages = dict(st, attention_scale=scale, sampled_pairs=sampled_pairs, routed_pairs=int(rt.pairs))
+    return per_call, stages, desc
 
 
 def cpu_cores_used() -> int:
+    """Threads the oracle's BLAS actually uses (its matrix products dominate), else the core count."""
     try:
         from threadpoolctl import threadpool_info
 
@@ -230,21 +260,27 @@ def run_reference(args):
     from synthetic import get_workload
 
     w = get_workload(args.workload)
-    vals = []
+    # warm-up: the same code paths on the smallest configuration (imports, BLAS thread pools)
+    for _ in range(args.warmup):
+        oracle_sample(get_workload("tiny_n1024"))
+    vals, stages = [], []
     sample_desc = ""
-    for i in range(args.warmup + args.steps):
-        per_call, sample_s, sample_desc = oracle_sample_seconds(w, n_groups=2)
-        if i >= args.warmup:
-            vals.append(per_call)
+    for _ in range(args.steps):
+        per_call, st, sample_desc = oracle_sample(w)
+        vals.append(per_call)
+        stages.append(st)
     per_call = statistics.mean(vals)
     value = w.dense_equiv_flops() / per_call / 1e12
     cores = cpu_cores_used()
+    stage_s = {k: statistics.mean(x[k] for x in stages) for k in stages[0]}
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_call * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, world=1),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample_desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu_count": os.cpu_count(),
+                         "kind": "oracle", "sample": sample_desc, "sample_stage_seconds": stage_s,
+                         "ms_per_call_scaled": per_call * 1e3},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -330,7 +366,7 @@ def run_ours(args):
         Oh = torch.empty_like(pin[0]).pin_memory()
         h.attention_host(*pin, Oh)
         e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        nsteps = max(1, min(args.steps, 3))
+        nsteps = max(1, args.steps)
         barrier()
         torch.cuda.synchronize()
         e_start.record(stream)
@@ -341,30 +377,36 @@ def run_ours(args):
         barrier()
         e_ms = reduce_max(e_start.elapsed_time(e_end) / nsteps, dev)
         h2d = sum(t.numel() * t.element_size() for t in pin)
-        e2e = {"value": whole_job_value(flops, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": whole_job_value(flops, world, e_ms), "unit": UNIT, "ms_per_step": e_ms, "steps": nsteps,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": Oh.numel() * Oh.element_size()}
 
     # dense baseline of the same library on the same shapes
     dense = None
     if not args.no_dense:
         Od = torch.empty_like(q)
-        h.dense_attn(q, k, v, Od)
+        for _ in range(max(1, args.warmup)):
+            h.dense_attn(q, k, v, Od)
         torch.cuda.synchronize()
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dsteps = max(1, args.steps)
+        barrier()
+        torch.cuda.synchronize()
         d0.record(stream)
-        h.dense_attn(q, k, v, Od)
-        h.dense_attn(q, k, v, Od)
+        for _ in range(dsteps):
+            h.dense_attn(q, k, v, Od)
         d1.record(stream)
         torch.cuda.synchronize()
-        dms = reduce_max(d0.elapsed_time(d1) / 2.0, dev)
-        dense = {"ms_per_call": dms, "tflops": flops / (dms * 1e-3) / 1e12, "speedup_vs_dense": dms / ms_max,
+        barrier()
+        dms = reduce_max(d0.elapsed_time(d1) / dsteps, dev)
+        dense = {"ms_per_call": dms, "steps": dsteps, "tflops": flops / (dms * 1e-3) / 1e12,
+                 "speedup_vs_dense": dms / ms_max,
                  "frac_of_peak": flops / (dms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        per_call, sample_s, desc = oracle_sample_seconds(w)
-        cpu = {"value": flops / per_call / 1e12, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
-               "sample": desc, "sample_seconds": sample_s, "ms_per_call_extrapolated": per_call * 1e3}
+        per_call, stages, desc = oracle_sample(w)
+        cpu = {"value": flops / per_call / 1e12, "unit": UNIT, "cores": cpu_cores_used(), "cpu_count": os.cpu_count(),
+               "kind": "oracle", "sample": desc, "sample_stage_seconds": stages, "ms_per_call_scaled": per_call * 1e3}
 
     if rank == 0:
         line = {

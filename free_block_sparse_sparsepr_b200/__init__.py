@@ -24,6 +24,7 @@ FLAG_PROBES_UNIFORM = 1 << 5     # ablation: probes on a uniform grid of the ori
 FLAG_PROBES_RANDOM = 1 << 6      # ablation: probes drawn at random (seeded SplitMix64)
 FLAG_SEMANTIC_PARTITION = 1 << 7  # ablation: k-means on the raw keys and the raw mean query
 FLAG_STAGE_TIMING = 1 << 8
+FLAG_TEST_STALL = 1 << 9          # test only: the dense kernel's first bounded wait runs out
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace allocation failed",
           4: "CUDA error", 5: "device wait timed out", 6: "device-side check failed"}

@@ -22,7 +22,8 @@ constexpr int kSortChunk = 2048;   // rows per counting-sort chunk (matches the 
 constexpr unsigned kSupportedFlags =
     SPARSEPR_FLAG_HARD_DROP_ONLY | SPARSEPR_FLAG_RIDGE_ONLY | SPARSEPR_FLAG_RBAR_UNPROJECTED |
     SPARSEPR_FLAG_UNIFORM_WEIGHTS | SPARSEPR_FLAG_TOPMASS | SPARSEPR_FLAG_STAGE_TIMING |
-    SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM | SPARSEPR_FLAG_SEMANTIC_PARTITION;
+    SPARSEPR_FLAG_PROBES_UNIFORM | SPARSEPR_FLAG_PROBES_RANDOM | SPARSEPR_FLAG_SEMANTIC_PARTITION |
+    SPARSEPR_FLAG_TEST_STALL;
 
 inline int pad16(int v) { return (v + 15) / 16 * 16; }
 inline int pad64(int v) { return (v + 63) / 64 * 64; }
@@ -143,6 +144,7 @@ sparsepr_status validate(const sparsepr_config* c) {
         return SPARSEPR_ERR_INVALID_ARG;
     if ((c->flags & SPARSEPR_FLAG_SEMANTIC_PARTITION) && (c->flags & SPARSEPR_FLAG_TOPMASS))
         return SPARSEPR_ERR_INVALID_ARG;
+    if ((c->flags & SPARSEPR_FLAG_TEST_STALL) && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
     if (!(c->flags & SPARSEPR_FLAG_HARD_DROP_ONLY)) {
         if (c->M < 1 || c->M > c->N) return SPARSEPR_ERR_INVALID_ARG;
         if (c->M > 64) return SPARSEPR_ERR_UNSUPPORTED;
@@ -838,7 +840,8 @@ sparsepr_status sparsepr_dense_attn(sparsepr_handle h, const void* Q, const void
     if (spr::attn_tc_supported(c.d)) {
         SPR_TRY(spr::launch_attn_dense_tc(static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
                                           static_cast<const bf16*>(V), static_cast<bf16*>(O), nullptr, c.B, c.Hq,
-                                          c.Hkv, c.N, h->dev_status, as_stream(stream)));
+                                          c.Hkv, c.N, h->dev_status, (c.flags & SPARSEPR_FLAG_TEST_STALL) != 0,
+                                          as_stream(stream)));
         return SPARSEPR_OK;
     }
     SPR_TRY(spr::launch_attn_dense(static_cast<const bf16*>(Q), static_cast<const bf16*>(K),

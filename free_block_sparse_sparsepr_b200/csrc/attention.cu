@@ -99,10 +99,16 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
     // Query tile (zero rows past the tile's end).
     for (int c = tid; c < kBM * VPR; c += 128) {
         const int r = c / VPR, v = c % VPR;
-        const bool valid = r < qn;
+        bool valid = r < qn;
         long long row;
-        if (MODE == kProbe) row = valid ? p.qidx[(long long)z * p.M + m0 + r] : 0;
-        else row = valid ? qlo + r : 0;
+        if (MODE == kProbe) {
+            // a row index outside [0, N) reads nothing: its query is zero-filled
+            const int32_t ri = valid ? p.qidx[(long long)z * p.M + m0 + r] : 0;
+            valid = valid && ri >= 0 && ri < p.N;
+            row = valid ? ri : 0;
+        } else {
+            row = valid ? qlo + r : 0;
+        }
         cp_async16(sQ + r * LD + v * 8, Qh + row * D + v * 8, valid);
     }
     cp_async_commit();

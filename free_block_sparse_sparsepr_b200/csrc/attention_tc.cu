@@ -68,6 +68,7 @@ struct TcParams {
     const int32_t* klist_off;     // [P][Gq+1] offsets into klist
     int* status;
     int N, g, Gq;
+    int stall;                    // test only: issue no loads (the first bounded wait runs out)
     float scale_log2;
 };
 
@@ -233,8 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 8) {
-        // ================= TMA producer
-        if (lane == 0) {
+        // ================= TMA producer (with p.stall set it issues nothing, so the MMA warp's
+        // wait for Q gives up after its bound and raises the abort flag; no copy is in flight)
+        if (lane == 0 && !p.stall) {
             const int qrow = x * p.N + qlo;
             tc::mbar_arrive_expect_tx(bar(kBarQ), (two ? 4 : 2) * kRegion);
             tc::tma_load_2d(sQ, &tmQ, bar(kBarQ), 0, qrow);
@@ -723,8 +725,9 @@ cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp
 }
 
 cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
-                                 int Hkv, int N, int* status, cudaStream_t s) {
+                                 int Hkv, int N, int* status, bool stall, cudaStream_t s) {
     TcParams p = params(O, lse, N, Hq / Hkv, status);
+    p.stall = stall ? 1 : 0;
     dim3 grid((N + 2 * kBM - 1) / (2 * kBM), B * Hq);
     return launch_tc<kModeDense>(Q, K, V, p, B, Hq, Hkv, grid, s);
 }

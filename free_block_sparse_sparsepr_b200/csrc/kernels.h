@@ -153,8 +153,9 @@ cudaError_t launch_key_tiles(const int32_t* rowptr, const int32_t* kg, const int
 cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp, const int32_t* qoff,
                                   const int32_t* tile_off, const int2* klist, const int32_t* klist_off, bf16* O,
                                   float* lse, int B, int Hq, int Hkv, int N, int Gq, int* status, cudaStream_t s);
+// stall: test only -- the producer issues no loads, so the first bounded wait runs out.
 cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
-                                 int Hkv, int N, int* status, cudaStream_t s);
+                                 int Hkv, int N, int* status, bool stall, cudaStream_t s);
 // Dense attention of gathered probe rows, split over ns key chunks, then combined.
 cudaError_t launch_attn_probe(const bf16* Q, const bf16* K, const bf16* V, const int32_t* probe,
                               float* Opart, float* mpart, float* lpart, float* Odense, int B,

@@ -8,8 +8,6 @@
 // of sparsepr_probe_fit). Its only scratch -- the per-split partial outputs,
 // maxima and sums of the split-key pass -- lives in one fixed-size array that
 // is compiled into the library, so the call allocates nothing.
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sparsepr.h"
@@ -19,32 +17,22 @@ namespace {
 constexpr size_t kScratchBytes = size_t(8) << 20;               // 8 MiB per GPU
 constexpr size_t kScratchFloats = kScratchBytes / sizeof(float);
 constexpr int kMaxSplits = 32;
-constexpr int kMaxDevices = 64;
 constexpr int kKeyTile = 64;
 
 // Split-key partials: Opart [B*Hq][ns][M][d], then mpart and lpart [B*Hq][ns][M].
 // Every GPU that loads the library keeps these 8 MiB until the process exits.
 static __device__ __align__(256) float g_probe_scratch[kScratchFloats];
 
-std::mutex g_scratch_mu;
-float* g_scratch_ptr[kMaxDevices] = {};
-
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Device address of the scratch array on the current device. The host-side name of
-// the array is only a stand-in, so the address is looked up once per device (with that
-// device current) and cached.
-sparsepr_status scratch_on_current_device(float** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SPARSEPR_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SPARSEPR_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_probe_scratch) != cudaSuccess || p == nullptr) return SPARSEPR_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<float*>(p);
-    }
-    *out = g_scratch_ptr[dev];
+// Device address of the scratch array in the current context. The host-side name of the array
+// is only a stand-in, so the address is looked up on every call, with the caller's device and
+// context current: a cached address would go stale after cudaDeviceReset or point into another
+// context when the caller switches contexts through the driver API.
+sparsepr_status scratch_in_current_context(float** out) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_probe_scratch) != cudaSuccess || p == nullptr) return SPARSEPR_ERR_CUDA;
+    *out = static_cast<float*>(p);
     return SPARSEPR_OK;
 }
 
@@ -54,6 +42,7 @@ extern "C" sparsepr_status sparsepr_probe_attention_noalloc(const void* Q, const
                                                             const int32_t* rows, float* O, int B, int Hq,
                                                             int Hkv, int N, int d, int M, void* stream) {
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !rows || !aligned16(O)) return SPARSEPR_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(rows) & 3u) != 0) return SPARSEPR_ERR_INVALID_ARG;
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || N < 1 || M < 1 || M > N) return SPARSEPR_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SPARSEPR_ERR_UNSUPPORTED;
     if (M > 64) return SPARSEPR_ERR_UNSUPPORTED;
@@ -64,7 +53,7 @@ extern "C" sparsepr_status sparsepr_probe_attention_noalloc(const void* Q, const
     const int tiles = (N + kKeyTile - 1) / kKeyTile;
     if (ns > tiles) ns = tiles;
     float* scratch = nullptr;
-    sparsepr_status st = scratch_on_current_device(&scratch);
+    sparsepr_status st = scratch_in_current_context(&scratch);
     if (st != SPARSEPR_OK) return st;
     const size_t hp = (size_t)B * Hq;
     float* Opart = scratch;

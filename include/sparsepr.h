@@ -69,6 +69,12 @@ typedef enum sparsepr_status {
                                                       of width d; `features` then holds the keys); not with
                                                       SPARSEPR_FLAG_TOPMASS */
 #define SPARSEPR_FLAG_STAGE_TIMING      (1u << 8)  /* record per-stage CUDA events (sparsepr_get_stats) */
+#define SPARSEPR_FLAG_TEST_STALL        (1u << 9)  /* TEST ONLY (d = 128): the kernel of sparsepr_dense_attn issues
+                                                      no loads, so its first bounded wait runs out (about 2 s of SM
+                                                      clock), every CTA returns with its TMEM freed and nothing in
+                                                      flight, the output rows are written as zeros and the device
+                                                      status word reads SPARSEPR_ERR_TIMEOUT; it exercises the
+                                                      bounded waits without a fault or a hang */
 
 /*
  * Shape and hyper-parameters of one call. Defaults used by the page: rK=48,
@@ -372,14 +378,18 @@ sparsepr_status sparsepr_set_stage_events(sparsepr_handle h, void* const* events
  * and the split-key partial results go to a fixed 8 MiB array compiled into the
  * library (every GPU that loads the library holds it until the process exits).
  *   Q        bf16 [B][Hq][N][d], K and V bf16 [B][Hkv][N][d] (device, 16-byte aligned)
- *   rows     int32 [B*Hkv][M]: original query rows, shared by the KV head's query heads
+ *   rows     int32 [B*Hkv][M] (device, 4-byte aligned): original query rows, shared by the KV
+ *            head's query heads; each must satisfy 0 <= row < N. A row outside that range reads
+ *            no memory: its query is taken as zero, so its output row is the mean of V.
  *   O        fp32 [B*Hq][M][d] (device, caller-owned): softmax(q K^T / sqrt(d)) V per row
  *   d in {64, 128}, 1 <= M <= min(N, 64)
  * Limit: B*Hq*M*(d+2)*4 bytes must fit in the 8 MiB array (e.g. 24 heads x 64
  * rows x d=128 uses 0.8 MB per key split, so 10 splits); larger requests return
- * SPARSEPR_ERR_UNSUPPORTED without touching the device. The first call on a
- * device looks up the array's device address on that device (cudaGetSymbolAddress,
- * with the device current), so make that first call before any stream capture.
+ * SPARSEPR_ERR_UNSUPPORTED without touching the device. Every call looks up the
+ * array's device address in the current context (cudaGetSymbolAddress, with the
+ * caller's device current), so the address stays right after cudaDeviceReset or a
+ * context switch; the first call on a device may load the library's device code, so
+ * make that first call before any stream capture.
  * Every call uses the same array: calls whose work overlaps on a GPU (two streams,
  * two threads) race on it and must be serialised by the caller. No part of the
  * array needs to start at zero: each call writes every slot it later reads.

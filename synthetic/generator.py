@@ -7,11 +7,14 @@ Recipe (per batch element b and KV head h, one independent random stream each):
   * one Gaussian matrix G ~ N(0, 1/8) of shape 8 x d shared by Q and K, so
     q.k reflects positional similarity;
   * K = a*phi(p)G + s*eps_K and, for every query head of the KV group,
-    Q = a*phi(p)G + s*eps_Q, with s = noise and a = 0.8*sqrt(2)*locality**0.4.
-    The locality scale enters the amplitude through that power law, fitted
-    so that one law meets both stated targets: at locality 1.2, noise 0.3 and
-    N=118800 a single query row needs a median 5-10% of the keys for 90% of
-    its softmax mass; at locality 0.4, noise 0.6 and N=75600 about 50%;
+    Q = a*phi(p)G + s*eps_Q, with s = noise. Workloads that state a locality
+    target (the 720p, world-model, sweep and stack calls) use
+    a = 0.8*sqrt(2)*locality**0.4: the locality scale enters the amplitude
+    through that power law, fitted so that one law meets both stated targets
+    (at locality 1.2, noise 0.3 and N=118800 a single query row needs a
+    median 5-10% of the keys for 90% of its softmax mass; at locality 0.4,
+    noise 0.6 and N=75600 about 50%). The tiny and mid calls, which state the
+    amplitude 0.8 and no target, use a = 0.8*locality;
   * V ~ N(0, 1);
   * everything rounded to bf16 (round to nearest even) and returned as the
     16-bit patterns, so both consumers see identical bits.
@@ -45,6 +48,14 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f32(b).astype(np.float64)
 
 
+def amplitude(w, locality: float | None = None) -> float:
+    """Amplitude a of the positional part of Q and K for workload w (locality override optional)."""
+    loc = w.locality if locality is None else locality
+    if getattr(w, "calibrated", True):
+        return AMPLITUDE * LOCALITY_GAIN * loc ** LOCALITY_EXPONENT
+    return AMPLITUDE * loc
+
+
 def _positions(T: int, Hg: int, Wg: int) -> np.ndarray:
     t, y, x = np.meshgrid(np.arange(T), np.arange(Hg), np.arange(Wg), indexing="ij")
     return np.stack([t.ravel() / T, y.ravel() / Hg, x.ravel() / Wg], axis=1)  # [N, 3]
@@ -71,8 +82,7 @@ def video_qkv(w, layer: int = 0, locality: float | None = None, threads: int | N
     Shapes: Q [B, Hq, N, d], K and V [B, Hkv, N, d]. Query head hq belongs to
     KV head hq // (Hq // Hkv).
     """
-    loc = w.locality if locality is None else locality
-    amp = AMPLITUDE * LOCALITY_GAIN * loc ** LOCALITY_EXPONENT
+    amp = amplitude(w, locality)
     pos = _positions(w.T, w.Hg, w.Wg)
     N, d, g = w.N, w.d, w.g
     Q = np.empty((w.B, w.Hq, N, d), dtype=np.uint16)
@@ -95,8 +105,7 @@ def video_qkv_device(w, layer: int = 0, locality: float | None = None, device: s
     values); it serves stacks of many layers, whose inputs would take minutes on the host."""
     import torch
 
-    loc = w.locality if locality is None else locality
-    amp = AMPLITUDE * LOCALITY_GAIN * loc ** LOCALITY_EXPONENT
+    amp = amplitude(w, locality)
     pos = torch.from_numpy(_positions(w.T, w.Hg, w.Wg)).to(device=device, dtype=torch.float64)
     N, d, g = w.N, w.d, w.g
     Q = torch.empty((w.B, w.Hq, N, d), dtype=torch.bfloat16, device=device)

@@ -34,6 +34,7 @@ class Workload:
     lam: float = 0.1
     kmeans_iters: int = 10
     seed: int = 0
+    calibrated: bool = True  # amplitude 0.8*sqrt(2)*locality**0.4 (locality targets); else 0.8*locality
 
     @property
     def N(self) -> int:
@@ -53,11 +54,15 @@ class Workload:
 
 WORKLOADS = {
     # Tiny single call: 2 heads, d=64, grid 4x16x16.
+    # Amplitude 0.8 as stated for this call (no locality target to calibrate to).
     "tiny_n1024": Workload("tiny_n1024", B=1, Hq=2, Hkv=2, T=4, Hg=16, Wg=16, d=64,
-                           Gk=16, Gq=16, block=64, rho=0.25, locality=1.0, noise=0.3),
+                           Gk=16, Gq=16, block=64, rho=0.25, locality=1.0, noise=0.3,
+                           calibrated=False),
     # Mid call: 12 heads MHA, d=128, grid 16x32x32.
+    # Amplitude 0.8 as stated for this call (no locality target to calibrate to).
     "mid_n16384": Workload("mid_n16384", B=1, Hq=12, Hkv=12, T=16, Hg=32, Wg=32, d=128,
-                           Gk=64, Gq=64, block=64, rho=0.22, locality=1.0, noise=0.3),
+                           Gk=64, Gq=64, block=64, rho=0.22, locality=1.0, noise=0.3,
+                           calibrated=False),
     # HunyuanVideo-shaped 720p call: 24 heads MHA, d=128, latent grid 33x45x80.
     "hunyuan720p_n118800": Workload("hunyuan720p_n118800", B=1, Hq=24, Hkv=24, T=33, Hg=45,
                                     Wg=80, d=128, Gk=256, Gq=256, block=128, rho=0.22,
