@@ -57,6 +57,7 @@ struct sparsepr_handle_s {
     int32_t *kgroup = nullptr, *qgroup = nullptr, *kperm = nullptr, *koff = nullptr, *qperm = nullptr,
             *qoff = nullptr, *probe = nullptr, *probe_pos = nullptr, *probe_seq = nullptr;
     float* topmass = nullptr;
+    unsigned* colmax = nullptr;          // column maxima of the responses (support diagnostic)
     float *kcent = nullptr, *radial = nullptr, *weights = nullptr, *features = nullptr, *ycoord = nullptr,
           *kdist = nullptr, *kmC = nullptr;
     int *counts = nullptr, *bases = nullptr, *km_changed = nullptr, *km_done = nullptr;
@@ -69,6 +70,8 @@ struct sparsepr_handle_s {
     int64_t* pairs = nullptr;
     // permuted tensors and sparse output
     bf16 *Qp = nullptr, *Kp = nullptr, *Vp = nullptr, *Osp = nullptr;
+    bf16* Qpr = nullptr;                 // gathered probe rows [Hp][128][d] (tensor-core probe pass)
+    bf16* wbparts = nullptr;             // bf16 parts of Bm and U^T (tensor-core write-back)
     float* lse = nullptr;
     // probes and fit
     float *Opart = nullptr, *mpart = nullptr, *lpart = nullptr, *Odense = nullptr, *R = nullptr,
@@ -89,7 +92,6 @@ struct sparsepr_handle_s {
     bf16 *kmX2 = nullptr, *kmC2 = nullptr;
     float *kmxx = nullptr, *kmcc = nullptr;
     int4* kmfix = nullptr;
-    int* kmfix_count = nullptr;
     bool semantic = false;   // ablation: k-means on the raw activations
     int launches = 0;
     int device = 0;
@@ -144,7 +146,7 @@ sparsepr_status validate(const sparsepr_config* c) {
         return SPARSEPR_ERR_INVALID_ARG;
     if ((c->flags & SPARSEPR_FLAG_SEMANTIC_PARTITION) && (c->flags & SPARSEPR_FLAG_TOPMASS))
         return SPARSEPR_ERR_INVALID_ARG;
-    if ((c->flags & SPARSEPR_FLAG_TEST_STALL) && c->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
+    if ((c->flags & SPARSEPR_FLAG_TEST_STALL) && !spr::attn_tc_supported(c->d)) return SPARSEPR_ERR_UNSUPPORTED;
     if (!(c->flags & SPARSEPR_FLAG_HARD_DROP_ONLY)) {
         if (c->M < 1 || c->M > c->N) return SPARSEPR_ERR_INVALID_ARG;
         if (c->M > 64) return SPARSEPR_ERR_UNSUPPORTED;
@@ -170,8 +172,9 @@ long long budget_pairs(const sparsepr_config& c, int M) {
 // Lloyd k-means on X [P][n][DP] into G groups, then the stable group-major order. With
 // G <= 256 the assignment runs on tensor cores (bf16 split operands, near ties settled in fp64)
 // and the radial distances come from one exact pass after the last assignment.
+// rows_split: the caller already wrote the rows' bf16 parts and squared norms (kmX2, kmxx).
 sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t* labels, float* dist,
-                       int32_t* perm, int32_t* off, cudaStream_t s) {
+                       int32_t* perm, int32_t* off, cudaStream_t s, bool rows_split = false) {
     const int P = h->P, n = h->cfg.N;
     const bool tc = spr::km_tc_supported(G) && DP <= 64;
     auto assign = [&](bool first, const int* done) -> cudaError_t {
@@ -179,15 +182,11 @@ sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t
         cudaError_t e = spr::launch_km_split_cent(h->kmC, h->kmC2, h->kmcc, P, G, DP, s);
         if (e != cudaSuccess) return e;
         ++h->launches;
-        e = spr::launch_km_assign_tc(X, h->kmX2, h->kmxx, h->kmC, h->kmC2, h->kmcc, labels, h->km_changed, done,
-                                     h->kmfix, h->kmfix_count, h->dev_status, P, n, G, DP, first, h->num_sms, s);
-        if (e != cudaSuccess) return e;
-        ++h->launches;
-        return spr::launch_km_fixup(h->kmfix, h->kmfix_count, X, h->kmC, h->kmcc, labels, h->km_changed, done, P, n,
-                                    G, DP, h->num_sms, s);
+        return spr::launch_km_assign_tc(X, h->kmX2, h->kmxx, h->kmC, h->kmC2, h->kmcc, labels, h->km_changed, done,
+                                        h->kmfix, h->dev_status, P, n, G, DP, first, h->num_sms, s);
     };
     SPR_TRY(spr::launch_km_reset(h->km_changed, h->km_done, P, s));
-    if (tc) SPR_TRY(spr::launch_km_split_rows(X, h->kmX2, h->kmxx, P, n, DP, s));
+    if (tc && !rows_split) SPR_TRY(spr::launch_km_split_rows(X, h->kmX2, h->kmxx, P, n, DP, s));
     SPR_TRY(spr::launch_km_seed(X, h->kmC, P, n, G, DP, s));
     SPR_TRY(assign(true, nullptr));
     for (int it = 0; it < h->cfg.kmeans_iters; ++it) {
@@ -249,19 +248,31 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     const sparsepr_config& c = h->cfg;
     const int P = h->P, N = c.N, d = c.d;
     if (h->semantic) return partition_semantic(h, Q, K, s);
-    // (1) sampled responses: F[z] = K[z] . Qs[z]^T / sqrt(d)
+    // (1) sampled responses: F[z] = K[z] . Qs[z]^T / sqrt(d); on the tensor cores the same pass
+    // writes the key k-means operands and (support diagnostic) the column maxima
+    const bool topmass = (c.flags & SPARSEPR_FLAG_TOPMASS) != 0;
     SPR_TRY(spr::launch_gather_samples(Q, h->Qs, c.B, c.Hq, c.Hkv, N, d, c.rK, h->DPk, s));
-    spr::GemmArgs a;
-    memset(&a, 0, sizeof(a));
-    a.A1 = K; a.sA = (long long)N * d; a.lda = d;
-    a.B1 = h->Qs; a.sB = (long long)h->DPk * d; a.ldb = d; a.bdiv = 1;
-    a.C = h->features; a.sC = (long long)N * h->DPk; a.ldc = h->DPk;
-    a.M = N; a.N = h->DPk; a.K = d; a.batch = P;
-    a.alpha = (float)(1.0 / sqrt((double)d));
-    SPR_TRY(spr::launch_gemm_bf16(a, s));
-    if (c.flags & SPARSEPR_FLAG_TOPMASS) SPR_TRY(spr::launch_topmass(h->features, h->topmass, P, N, h->DPk, c.rK, s));
+    const bool resp_tc = spr::resp_tc_supported(d, h->DPk);
+    if (resp_tc) {
+        SPR_TRY(spr::launch_resp_tc(K, h->Qs, h->features, h->kmX2, h->kmxx, topmass ? h->colmax : nullptr, P, N, d,
+                                    h->DPk, c.rK, h->num_sms, h->dev_status, s));
+        if (topmass) ++h->launches;   // the memset of the maxima
+    } else {
+        spr::GemmArgs a;
+        memset(&a, 0, sizeof(a));
+        a.A1 = K; a.sA = (long long)N * d; a.lda = d;
+        a.B1 = h->Qs; a.sB = (long long)h->DPk * d; a.ldb = d; a.bdiv = 1;
+        a.C = h->features; a.sC = (long long)N * h->DPk; a.ldc = h->DPk;
+        a.M = N; a.N = h->DPk; a.K = d; a.batch = P;
+        a.alpha = (float)(1.0 / sqrt((double)d));
+        SPR_TRY(spr::launch_gemm_bf16(a, s));
+    }
+    if (topmass)
+        SPR_TRY(spr::launch_topmass(h->features, h->topmass, resp_tc ? h->colmax : nullptr, P, N, h->DPk, c.rK, s));
     // (2a) key groups and their means in the original key space
-    sparsepr_status st = kmeans(h, h->features, h->DPk, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s);
+    const bool key_rows_split = resp_tc && spr::km_tc_supported(c.Gk);
+    sparsepr_status st = kmeans(h, h->features, h->DPk, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s,
+                                key_rows_split);
     if (st) return st;
     SPR_TRY(spr::launch_group_mean_bf16(K, h->kperm, h->koff, h->kcent, h->chi, h->clo, P, N, c.Gk, d, s));
     // (2b) query coordinates and query groups
@@ -358,12 +369,12 @@ sparsepr_status attn_impl(sparsepr_handle h, const bf16* Qp, const bf16* Kp, con
                           cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
     if (spr::attn_tc_supported(c.d)) {
-        SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, spr::attn_tc_rows_per_cta(), s));
+        SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, spr::attn_tc_rows_per_cta(h->g), s));
         SPR_TRY(spr::launch_key_tiles(r->rowptr, r->kg, p->koff, h->ktile_cnt, h->ktile_off, h->ktile_list, h->P, c.N,
                                       c.Gq, c.Gk, s));
         h->launches += 2;  // count, scan and write kernels
         SPR_TRY(spr::launch_attn_sparse_tc(Qp, Kp, Vp, p->qoff, h->tile_off, h->ktile_list, h->ktile_off, Osp, lse,
-                                           c.B, c.Hq, c.Hkv, c.N, c.Gq, h->dev_status, s));
+                                           c.B, c.Hq, c.Hkv, c.N, c.d, c.Gq, h->dev_status, s));
         return SPARSEPR_OK;
     }
     SPR_TRY(spr::launch_tile_offsets(p->qoff, h->tile_off, h->P, c.Gq, 64, s));
@@ -376,9 +387,18 @@ sparsepr_status probe_fit_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
                                const sparsepr_partition_t* p, const bf16* Osp, cudaStream_t s) {
     const sparsepr_config& c = h->cfg;
     if (!h->M) return SPARSEPR_OK;
-    SPR_TRY(spr::launch_attn_probe(Q, K, V, p->probe, h->Opart, h->mpart, h->lpart, h->Odense, c.B, c.Hq, c.Hkv,
-                                   c.N, c.d, h->M, kProbeSplits, s));
-    ++h->launches;  // combine kernel
+    if (spr::attn_tc_supported(c.d)) {
+        // dense attention of the probe rows on the tensor cores, split over the keys
+        SPR_TRY(spr::launch_gather_probe_rows(Q, p->probe, h->Qpr, c.B, c.Hq, c.Hkv, c.N, h->M, c.d, 128, s));
+        SPR_TRY(spr::launch_attn_probe_tc(h->Qpr, K, V, h->Opart, h->mpart, h->lpart, c.B, c.Hq, c.Hkv, c.N, c.d,
+                                          h->M, kProbeSplits, h->dev_status, s));
+        SPR_TRY(spr::launch_probe_combine(h->Opart, h->mpart, h->lpart, h->Odense, h->Hp, h->M,
+                                          spr::probe_tc_splits(c.N, kProbeSplits), c.d, s));
+    } else {
+        SPR_TRY(spr::launch_attn_probe(Q, K, V, p->probe, h->Opart, h->mpart, h->lpart, h->Odense, c.B, c.Hq, c.Hkv,
+                                       c.N, c.d, h->M, kProbeSplits, s));
+        ++h->launches;  // combine kernel
+    }
     SPR_TRY(spr::launch_probe_residual(h->Odense, Osp, p->probe_pos, h->R, h->Xprobe, h->Hp, h->g, c.N, c.d,
                                        h->M, s));
     SPR_TRY(spr::launch_fit(h->R, h->Xprobe, p->weights, c.lambda, h->obar, h->Rbar, h->A, h->U, h->Bm, h->c0,
@@ -394,6 +414,11 @@ sparsepr_status writeback_impl(sparsepr_handle h, const sparsepr_partition_t* p,
     if (correct && (c.flags & SPARSEPR_FLAG_RIDGE_ONLY)) {
         SPR_TRY(spr::launch_writeback_ridge(Osp, p->qperm, f->A, f->obar, f->Rbar, O, h->Hp, h->g, c.N, c.d,
                                             h->num_sms, s));
+    } else if (correct && h->wbparts && spr::wb_tc_supported(c.d, c.r)) {
+        const float* radd = (c.flags & SPARSEPR_FLAG_RBAR_UNPROJECTED) ? f->Rbar : nullptr;
+        SPR_TRY(spr::launch_writeback_tc(Osp, p->qperm, f->U, f->Bm, f->c0, radd, h->wbparts, O, h->Hp, h->g, c.N, c.r,
+                                         h->dev_status, h->num_sms, s));
+        ++h->launches;   // the split of Bm and U^T into bf16 parts
     } else {
         const float* radd = (correct && (c.flags & SPARSEPR_FLAG_RBAR_UNPROJECTED)) ? f->Rbar : nullptr;
         SPR_TRY(spr::launch_writeback(Osp, p->qperm, correct ? f->U : nullptr, correct ? f->Bm : nullptr,
@@ -461,6 +486,7 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     A_(kgroup, P * N); A_(qgroup, P * N); A_(kperm, P * N); A_(koff, P * (Gk + 1));
     A_(qperm, P * N); A_(qoff, P * (Gq + 1)); A_(probe, P * M); A_(probe_pos, P * M); A_(probe_seq, P * M);
     A_(kcent, P * Gk * d); A_(radial, P * N); A_(weights, P * M); A_(features, P * N * h->DPk); A_(topmass, P * c.rK);
+    A_(colmax, P * h->DPk);
     A_(ycoord, P * N * h->DPy); A_(kdist, P * N); A_(kmC, P * h->Gmax * (size_t)(h->DPk > 64 || h->DPy > 64 ? (h->DPk > h->DPy ? h->DPk : h->DPy) : 64));
     A_(counts, P * h->nch * h->Gmax); A_(bases, P * h->nch * h->Gmax); A_(km_changed, P); A_(km_done, P);
     A_(Qs, P * h->DPk * d); A_(chi, P * Gk * d); A_(clo, P * Gk * d);
@@ -475,13 +501,16 @@ sparsepr_status sparsepr_create(const sparsepr_config* cfg, sparsepr_handle* out
     A_(Qp, Hp * N * d); A_(Kp, P * N * d); A_(Vp, P * N * d); A_(Osp, Hp * N * d); A_(lse, Hp * N);
     A_(Opart, Hp * kProbeSplits * M * d); A_(mpart, Hp * kProbeSplits * M); A_(lpart, Hp * kProbeSplits * M);
     A_(Odense, Hp * M * d); A_(R, Hp * M * d); A_(Xprobe, Hp * M * d);
+    if (spr::attn_tc_supported(c.d)) A_(Qpr, Hp * 128 * d);
+    if (spr::wb_tc_supported(c.d, (int)r)) A_(wbparts, spr::wb_tc_parts_elems((int)Hp));
     A_(obar, Hp * d); A_(Rbar, Hp * d); A_(A, Hp * d * d); A_(U, Hp * d * r); A_(Bm, Hp * r * d); A_(c0, Hp * r);
     A_(rank, Hp); A_(dev_status, 1);
     {
         const size_t G16 = (size_t)((h->Gmax + 15) / 16 * 16), G32 = (size_t)((h->Gmax + 31) / 32 * 32);
         A_(kmX2, 2 * P * N * 64); A_(kmxx, P * N);
         A_(kmC2, 2 * P * G16 * 64); A_(kmcc, P * G32);
-        A_(kmfix, spr::km_fix_slots(P, N, h->num_sms)); A_(kmfix_count, P * h->num_sms);
+        A_(kmfix, spr::km_fix_slots(P, N, h->num_sms));
+
     }
 #undef A_
     bool ok = cudaMemset(h->dev_status, 0, sizeof(int)) == cudaSuccess;
@@ -840,7 +869,7 @@ sparsepr_status sparsepr_dense_attn(sparsepr_handle h, const void* Q, const void
     if (spr::attn_tc_supported(c.d)) {
         SPR_TRY(spr::launch_attn_dense_tc(static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
                                           static_cast<const bf16*>(V), static_cast<bf16*>(O), nullptr, c.B, c.Hq,
-                                          c.Hkv, c.N, h->dev_status, (c.flags & SPARSEPR_FLAG_TEST_STALL) != 0,
+                                          c.Hkv, c.N, c.d, h->dev_status, (c.flags & SPARSEPR_FLAG_TEST_STALL) != 0,
                                           as_stream(stream)));
         return SPARSEPR_OK;
     }

@@ -280,6 +280,23 @@ __global__ void probe_combine_kernel(const float* __restrict__ Opart, const floa
     Od[((long long)x * M + m) * D + c] = L > 0.f ? acc / L : 0.f;
 }
 
+// Qpr[x][r] = Q[x][probe[z][r]] for r < M, zero for M <= r < rows (one 16-byte vector per thread
+// step); a probe index outside [0, N) gives a zero row.
+__global__ void gather_probe_rows_kernel(const bf16* __restrict__ Q, const int32_t* __restrict__ probe, bf16* Qpr,
+                                         int g, int N, int M, int d, int rows) {
+    const int x = blockIdx.x, z = x / g;
+    const int vpr = d / 8;
+    for (int t = threadIdx.x; t < rows * vpr; t += blockDim.x) {
+        const int r = t / vpr, c = t % vpr;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < M) {
+            const int row = probe[(long long)z * M + r];
+            if (row >= 0 && row < N) v = reinterpret_cast<const uint4*>(Q + ((long long)x * N + row) * d)[c];
+        }
+        reinterpret_cast<uint4*>(Qpr + ((long long)x * rows + r) * d)[c] = v;
+    }
+}
+
 __global__ void tile_offsets_kernel(const int32_t* __restrict__ qoff, int32_t* tile_off, int P, int Gq, int bm) {
     const int z = blockIdx.x * blockDim.x + threadIdx.x;
     if (z >= P) return;
@@ -343,6 +360,18 @@ cudaError_t launch_attn_dense(const bf16* Q, const bf16* K, const bf16* V, bf16*
     p.Q = Q; p.K = K; p.V = V; p.O = O; p.lse = lse;
     dim3 grid((N + kBM - 1) / kBM, B * Hq);
     return launch_attn_d<kDense>(d, p, grid, s);
+}
+
+cudaError_t launch_gather_probe_rows(const bf16* Q, const int32_t* probe, bf16* Qpr, int B, int Hq, int Hkv, int N,
+                                    int M, int d, int rows, cudaStream_t s) {
+    gather_probe_rows_kernel<<<B * Hq, 256, 0, s>>>(Q, probe, Qpr, Hq / Hkv, N, M, d, rows);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_probe_combine(const float* Opart, const float* mpart, const float* lpart, float* Odense, int Hp,
+                                 int M, int ns, int d, cudaStream_t s) {
+    probe_combine_kernel<<<dim3(M, Hp), d, 0, s>>>(Opart, mpart, lpart, Odense, M, ns, d);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_attn_probe(const bf16* Q, const bf16* K, const bf16* V, const int32_t* probe,

@@ -35,7 +35,6 @@ namespace {
 
 constexpr int kBM = 128;            // rows per query tile (two tiles per CTA)
 constexpr int kBN = 128;            // keys per tile
-constexpr int kD = 128;             // head dimension
 constexpr int kStages = 2;          // K/V ring depth
 constexpr int kRegion = 16384;      // one [128 rows][64 bf16] 128B-swizzled region
 constexpr int kThreads = 320;
@@ -57,7 +56,7 @@ constexpr int kOffMisc = kOffBar + 8 * kNumBars;          // tmem base (u32), ab
 constexpr int kOffML = kOffMisc + 16;                      // split mode: tile 1's running max and sum [2][128]
 constexpr int kSmemBytes = kOffML + 2 * kBM * 4 + 1024;   // + slack to align the base to 1024
 
-enum { kModeSparse = 0, kModeDense = 1 };
+enum { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 
 struct TcParams {
     bf16* O;
@@ -68,7 +67,14 @@ struct TcParams {
     const int32_t* klist_off;     // [P][Gq+1] offsets into klist
     int* status;
     int N, g, Gq;
+    int head_pairs;               // sparse mode, g even: one CTA = the same query tile of two query heads
     int stall;                    // test only: issue no loads (the first bounded wait runs out)
+    // probe mode: M gathered rows per query head against key split blockIdx.x (chunk keys each);
+    // unnormalised partial outputs [x][ns][M][d], running maxima (log2 units) and sums [x][ns][M]
+    float* Opart;
+    float* mpart;
+    float* lpart;
+    int M, ns, chunk;
     float scale_log2;
 };
 
@@ -154,14 +160,20 @@ __device__ __forceinline__ int2 key_tile(const TcParams& p, int mode, const int2
         const int st = j * kBN;
         return make_int2(st, min(kBN, p.N - st));
     }
+    if (mode == kModeProbe) {
+        const int st = blockIdx.x * p.chunk + j * kBN;
+        return make_int2(st, min(kBN, min(p.N, (blockIdx.x + 1) * p.chunk) - st));
+    }
     return list[j];
 }
 
-template <int MODE>
+template <int MODE, int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                               const __grid_constant__ CUtensorMap tmK,
                                                               const __grid_constant__ CUtensorMap tmV,
                                                               const TcParams p) {
+    static_assert(D == 64 || D == 128, "head dimension");
+    constexpr int kNR = D / 64;          // 128-byte swizzle regions per row of a tile
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = tc::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -173,12 +185,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int x = blockIdx.y, z = x / p.g;
+    // Query tile t covers rows [qrow[t], qrow[t] + qn_t) of the flattened [B*Hq*N] query rows:
+    // either two consecutive 128-row tiles of query head x, or (head pairs, grouped-query
+    // attention with an even group) the same 128 rows of query heads x and x + 1, which share
+    // the KV head, the query group and therefore every key tile.
+    const int hp = p.head_pairs ? p.g / 2 : 1;
+    const int z = p.head_pairs ? (int)blockIdx.y / hp : (int)blockIdx.y / p.g;
+    const int x = p.head_pairs ? z * p.g + 2 * ((int)blockIdx.y % hp) : (int)blockIdx.y;
     // a CTA that timed out earlier in this launch (or call) makes the rest return at once
     if (p.status && *reinterpret_cast<volatile int*>(p.status) == kDevTimeout) return;
 
-    // ---- which query tiles: rows [qlo, qlo + qn0) and [qlo + 128, qlo + 128 + qn1)
+    // ---- which query tiles
     int qlo, qn0, qn1, a = 0, ntk = 0;
+    long long qrow[2];
     const int2* klist = nullptr;
     if (MODE == kModeSparse) {
         const int32_t* toff = p.tile_off + (long long)z * (p.Gq + 1);
@@ -189,16 +208,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         klist = p.klist + lo[a];
         ntk = lo[a + 1] - lo[a];
         const int32_t* qo = p.qoff + (long long)z * (p.Gq + 1);
-        qlo = qo[a] + (pair - toff[a]) * 2 * kBM;
-        const int rows = qo[a + 1] - qlo;
-        qn0 = min(kBM, rows);
-        qn1 = min(kBM, rows - kBM);
+        if (p.head_pairs) {
+            qlo = qo[a] + (pair - toff[a]) * kBM;
+            qn0 = qn1 = min(kBM, qo[a + 1] - qlo);
+            qrow[0] = (long long)x * p.N + qlo;
+            qrow[1] = (long long)(x + 1) * p.N + qlo;
+        } else {
+            qlo = qo[a] + (pair - toff[a]) * 2 * kBM;
+            const int rows = qo[a + 1] - qlo;
+            qn0 = min(kBM, rows);
+            qn1 = min(kBM, rows - kBM);
+            qrow[0] = (long long)x * p.N + qlo;
+            qrow[1] = qrow[0] + kBM;
+        }
+    } else if (MODE == kModeProbe) {
+        // the head's gathered probe rows (one tile, rows >= M zero) against keys of split blockIdx.x
+        qlo = 0;
+        qn0 = p.M;
+        qn1 = 0;
+        const int klo = blockIdx.x * p.chunk, khi = min(p.N, klo + p.chunk);
+        ntk = khi > klo ? (khi - klo + kBN - 1) / kBN : 0;
+        qrow[0] = (long long)x * kBM;
+        qrow[1] = qrow[0];
     } else {
         qlo = blockIdx.x * 2 * kBM;
         if (qlo >= p.N) return;
         qn0 = min(kBM, p.N - qlo);
         qn1 = min(kBM, p.N - qlo - kBM);
         ntk = (p.N + kBN - 1) / kBN;
+        qrow[0] = (long long)x * p.N + qlo;
+        qrow[1] = qrow[0] + kBM;
     }
     const bool two = qn1 > 0;
     // split mode: a lone query tile with two or more key tiles. Both softmax warpgroups take
@@ -237,14 +276,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // ================= TMA producer (with p.stall set it issues nothing, so the MMA warp's
         // wait for Q gives up after its bound and raises the abort flag; no copy is in flight)
         if (lane == 0 && !p.stall) {
-            const int qrow = x * p.N + qlo;
-            tc::mbar_arrive_expect_tx(bar(kBarQ), (two ? 4 : 2) * kRegion);
-            tc::tma_load_2d(sQ, &tmQ, bar(kBarQ), 0, qrow);
-            tc::tma_load_2d(sQ + kRegion, &tmQ, bar(kBarQ), 64, qrow);
-            if (two) {
-                tc::tma_load_2d(sQ + 2 * kRegion, &tmQ, bar(kBarQ), 0, qrow + kBM);
-                tc::tma_load_2d(sQ + 3 * kRegion, &tmQ, bar(kBarQ), 64, qrow + kBM);
-            }
+            tc::mbar_arrive_expect_tx(bar(kBarQ), (two ? 2 : 1) * kNR * kRegion);
+            for (int h = 0; h < kNR; ++h) tc::tma_load_2d(sQ + h * kRegion, &tmQ, bar(kBarQ), 64 * h, (int)qrow[0]);
+            if (two)
+                for (int h = 0; h < kNR; ++h)
+                    tc::tma_load_2d(sQ + (2 + h) * kRegion, &tmQ, bar(kBarQ), 64 * h, (int)qrow[1]);
             // K runs one tile ahead of V: K(0), then K(j+1) before V(j).
             auto load = [&](int m, bool isv) -> bool {
                 const int s = m % kStages;
@@ -253,9 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 const int krow = z * p.N + key_tile(p, MODE, klist, m).x;
                 const uint32_t d = (isv ? sV : sK) + s * 2 * kRegion;
                 const uint32_t b = bar((isv ? kBarV : kBarK) + s);
-                tc::mbar_arrive_expect_tx(b, 2 * kRegion);
-                tc::tma_load_2d(d, isv ? &tmV : &tmK, b, 0, krow);
-                tc::tma_load_2d(d + kRegion, isv ? &tmV : &tmK, b, 64, krow);
+                tc::mbar_arrive_expect_tx(b, kNR * kRegion);
+                for (int h = 0; h < kNR; ++h) tc::tma_load_2d(d + h * kRegion, isv ? &tmV : &tmK, b, 64 * h, krow);
                 return true;
             };
             int nk = 0, nv = 0;   // K and V tiles issued
@@ -280,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // ================= MMA issuer
         const uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0);
         const uint32_t idS64 = tc::idesc_bf16_f32(kBM, 64, 0);   // half tile: at most 64 valid keys
-        const uint32_t idO = tc::idesc_bf16_f32(kBM, kD, 1);
+        const uint32_t idO = tc::idesc_bf16_f32(kBM, D, 1);
         // PV k-steps of key tile j (16 keys each): 4 for a half tile, else 8
         auto pv_steps = [&](int j) { return key_tile(p, MODE, klist, j).y <= 64 ? 4 : kBN / 16; };
         const int ntiles = two ? 2 : 1;
@@ -291,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const uint32_t qb = sQ + (split ? 0 : t) * 2 * kRegion;
             const uint32_t id = key_tile(p, MODE, klist, j).y <= 64 ? idS64 : idS;
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k) {
+            for (int k = 0; k < D / 16; ++k) {
                 const uint32_t off = (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
                 tc::mma_f16_ss(tmem + (uint32_t)(t * 128), tc::smem_desc_sw128(qb + off, 16, 1024),
                                tc::smem_desc_sw128(kb + off, 16, 1024), id, k > 0 ? 1u : 0u);
@@ -397,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // ================= softmax warpgroup t: thread r <-> row r of tile t <-> TMEM lane r
         const int t = warp >> 2;
         const int r = threadIdx.x & 127;
+        const long long qrow_t = t ? qrow[1] : qrow[0];   // first flattened query row of tile t
         const int qn = (t == 0 || split) ? qn0 : qn1;
         float* sML = reinterpret_cast<float*>(sbase + kOffML);   // split mode: [0][r] max, [1][r] sum of tile 1
         if (qn > 0) {
@@ -459,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         // S_t(j) complete => PV_t(j-1) complete: O_t may be rescaled now
                         const float f = rescale ? exp2f(m_run - m_new) : 1.f;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < D / 32; ++c) {
                             uint32_t ov[32];
                             tc::tmem_ld32(tO + 32 * c, ov);
                             tc::tmem_wait_ld();
@@ -524,17 +560,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         const float f1 = mm == -INFINITY ? 0.f : exp2f(m1 - mm);
                         const float l = l_run * f0 + l1 * f1;
                         const float inv = l > 0.f ? 1.f / l : 0.f;
-                        const float a0 = f0 * inv, a1 = f1 * inv;
-                        bf16* orow = p.O + ((long long)x * p.N + qlo + r) * kD;
+                        // probe mode keeps the merged partial state unnormalised (scaled to mm)
+                        const float a0 = MODE == kModeProbe ? f0 : f0 * inv, a1 = MODE == kModeProbe ? f1 : f1 * inv;
+                        bf16* orow = p.O + (qrow[0] + r) * D;
+                        const long long pb = ((long long)x * p.ns + blockIdx.x) * p.M + r;
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < D / 32; ++c) {
                             uint32_t o0[32], o1[32];
                             tc::tmem_ld32(tO + 32 * c, o0);
                             tc::tmem_ld32(tO + 128 + 32 * c, o1);
                             tc::tmem_wait_ld();
                             tc::regs_after_wait(o0);
                             tc::regs_after_wait(o1);
-                            if (r < qn) {
+                            if (MODE == kModeProbe) {
+                                if (r < qn) {
+                                    float4* prow = reinterpret_cast<float4*>(p.Opart + pb * D + 32 * c);
+#pragma unroll
+                                    for (int q = 0; q < 8; ++q)
+                                        prow[q] = make_float4(
+                                            fmaf(__uint_as_float(o0[4 * q]), a0, __uint_as_float(o1[4 * q]) * a1),
+                                            fmaf(__uint_as_float(o0[4 * q + 1]), a0, __uint_as_float(o1[4 * q + 1]) * a1),
+                                            fmaf(__uint_as_float(o0[4 * q + 2]), a0, __uint_as_float(o1[4 * q + 2]) * a1),
+                                            fmaf(__uint_as_float(o0[4 * q + 3]), a0, __uint_as_float(o1[4 * q + 3]) * a1));
+                                }
+                            } else if (r < qn) {
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) {
                                     uint32_t w[4];
@@ -550,18 +599,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                 }
                             }
                         }
-                        if (r < qn && p.lse) p.lse[(long long)x * p.N + qlo + r] = (mm + log2f(l)) * kLn2;
+                        if (MODE == kModeProbe) {
+                            if (r < qn) {
+                                p.mpart[pb] = mm;
+                                p.lpart[pb] = l;
+                            }
+                        } else if (r < qn && p.lse) {
+                            p.lse[qrow[0] + r] = (mm + log2f(l)) * kLn2;
+                        }
                     }
                 }
             } else {
             bool got_last = false;
             if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO + t), 0, abort_flag);
-            if (j > 0 && __all_sync(kFull, got_last)) {
+            const long long pb = ((long long)x * p.ns + blockIdx.x) * p.M + r;   // probe mode
+            if (MODE == kModeProbe && j > 0 && __all_sync(kFull, got_last)) {
+                // a single key tile: the unnormalised state as it stands
+                tc::fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t ov[32];
+                    tc::tmem_ld32(tO + 32 * c, ov);
+                    tc::tmem_wait_ld();
+                    tc::regs_after_wait(ov);
+                    if (r < qn) {
+                        float4* prow = reinterpret_cast<float4*>(p.Opart + pb * D + 32 * c);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            prow[q] = make_float4(__uint_as_float(ov[4 * q]), __uint_as_float(ov[4 * q + 1]),
+                                                  __uint_as_float(ov[4 * q + 2]), __uint_as_float(ov[4 * q + 3]));
+                    }
+                }
+                if (r < qn) {
+                    p.mpart[pb] = m_run;
+                    p.lpart[pb] = l_run;
+                }
+            } else if (MODE == kModeProbe) {
+                if (j == 0 && r < qn) {
+                    // an empty key split: no mass
+                    float4* prow = reinterpret_cast<float4*>(p.Opart + pb * D);
+                    for (int c = 0; c < D / 4; ++c) prow[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    p.mpart[pb] = -INFINITY;
+                    p.lpart[pb] = 0.f;
+                }
+            } else if (j > 0 && __all_sync(kFull, got_last)) {
                 tc::fence_after_sync();
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-                bf16* orow = p.O + ((long long)x * p.N + qlo + t * kBM + r) * kD;
+                bf16* orow = p.O + (qrow_t + r) * D;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t ov[32];
                     tc::tmem_ld32(tO + 32 * c, ov);
                     tc::tmem_wait_ld();
@@ -581,11 +667,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     }
                 }
                 if (r < qn && p.lse)
-                    p.lse[(long long)x * p.N + qlo + t * kBM + r] = (m_run + log2f(l_run)) * kLn2;
+                    p.lse[qrow_t + r] = (m_run + log2f(l_run)) * kLn2;
             } else if (j == 0 && r < qn) {
-                bf16* orow = p.O + ((long long)x * p.N + qlo + t * kBM + r) * kD;
-                for (int c = 0; c < kD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[(long long)x * p.N + qlo + t * kBM + r] = -INFINITY;
+                bf16* orow = p.O + (qrow_t + r) * D;
+                for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+                if (p.lse) p.lse[qrow_t + r] = -INFINITY;
             }
             }
         }
@@ -666,21 +752,30 @@ __global__ void key_tiles_scan_kernel(const int32_t* __restrict__ cnt, int32_t* 
 
 // ---------------------------------------------------------------- host side
 
-template <int MODE>
-cudaError_t launch_tc(const bf16* Q, const bf16* K, const bf16* V, const TcParams& p, int B, int Hq, int Hkv,
+template <int MODE, int D>
+cudaError_t launch_tc(const bf16* Q, const bf16* K, const bf16* V, const TcParams& p, long long qrows, int B, int Hkv,
                       dim3 grid, cudaStream_t s) {
     CUtensorMap mq, mk, mv;
-    if (!make_tmap_bf16_sw128(&mq, Q, (long long)B * Hq * p.N, kD, kBM, 64) ||
-        !make_tmap_bf16_sw128(&mk, K, (long long)B * Hkv * p.N, kD, kBN, 64) ||
-        !make_tmap_bf16_sw128(&mv, V, (long long)B * Hkv * p.N, kD, kBN, 64))
+    if (!make_tmap_bf16_sw128(&mq, Q, qrows, D, kBM, 64) ||
+        !make_tmap_bf16_sw128(&mk, K, (long long)B * Hkv * p.N, D, kBN, 64) ||
+        !make_tmap_bf16_sw128(&mv, V, (long long)B * Hkv * p.N, D, kBN, 64))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<MODE, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
+    attn_tc_kernel<MODE, D><<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
-TcParams params(bf16* O, float* lse, int N, int g, int* status) {
+template <int MODE>
+cudaError_t launch_tc_d(int d, const bf16* Q, const bf16* K, const bf16* V, const TcParams& p, long long qrows, int B,
+                        int Hkv, dim3 grid, cudaStream_t s) {
+    if (d == 128) return launch_tc<MODE, 128>(Q, K, V, p, qrows, B, Hkv, grid, s);
+    if (d == 64) return launch_tc<MODE, 64>(Q, K, V, p, qrows, B, Hkv, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+TcParams params(bf16* O, float* lse, int N, int g, int d, int* status) {
     TcParams p;
     memset(&p, 0, sizeof(p));
     p.O = O;
@@ -688,15 +783,21 @@ TcParams params(bf16* O, float* lse, int N, int g, int* status) {
     p.N = N;
     p.g = g;
     p.status = status;
-    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kD));
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
     return p;
 }
 
 }  // namespace
 
-bool attn_tc_supported(int d) { return d == kD; }
+bool attn_tc_supported(int d) { return d == 64 || d == 128; }
 
-int attn_tc_rows_per_cta() { return 2 * kBM; }
+// Keys per probe split (whole 128-key tiles) and the number of non-empty splits.
+int probe_tc_chunk(int N, int ns) { return ((N + ns - 1) / ns + kBN - 1) / kBN * kBN; }
+int probe_tc_splits(int N, int ns) { return (N + probe_tc_chunk(N, ns) - 1) / probe_tc_chunk(N, ns); }
+
+bool attn_tc_head_pairs(int g) { return g % 2 == 0; }
+
+int attn_tc_rows_per_cta(int g) { return attn_tc_head_pairs(g) ? kBM : 2 * kBM; }
 
 long long key_tiles_capacity(int N, int Gq, int Gk) { return (long long)Gq * ((N + kBN - 1) / kBN + Gk); }
 
@@ -716,20 +817,35 @@ cudaError_t launch_key_tiles(const int32_t* rowptr, const int32_t* kg, const int
 
 cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp, const int32_t* qoff,
                                   const int32_t* tile_off, const int2* klist, const int32_t* klist_off, bf16* O,
-                                  float* lse, int B, int Hq, int Hkv, int N, int Gq, int* status, cudaStream_t s) {
-    TcParams p = params(O, lse, N, Hq / Hkv, status);
+                                  float* lse, int B, int Hq, int Hkv, int N, int d, int Gq, int* status, cudaStream_t s) {
+    const int g = Hq / Hkv;
+    TcParams p = params(O, lse, N, g, d, status);
     p.qoff = qoff; p.tile_off = tile_off; p.klist = klist; p.klist_off = klist_off;
     p.Gq = Gq;
-    dim3 grid((N + 2 * kBM - 1) / (2 * kBM) + Gq, B * Hq);
-    return launch_tc<kModeSparse>(Qp, Kp, Vp, p, B, Hq, Hkv, grid, s);
+    p.head_pairs = attn_tc_head_pairs(g) ? 1 : 0;
+    const int rows = attn_tc_rows_per_cta(g);
+    dim3 grid((N + rows - 1) / rows + Gq, p.head_pairs ? B * Hq / 2 : B * Hq);
+    return launch_tc_d<kModeSparse>(d, Qp, Kp, Vp, p, (long long)B * Hq * N, B, Hkv, grid, s);
+}
+
+cudaError_t launch_attn_probe_tc(const bf16* Qpr, const bf16* K, const bf16* V, float* Opart, float* mpart,
+                                 float* lpart, int B, int Hq, int Hkv, int N, int d, int M, int ns, int* status,
+                                 cudaStream_t s) {
+    if (M < 1 || M > kBM || ns < 1) return cudaErrorInvalidValue;
+    TcParams p = params(nullptr, nullptr, N, Hq / Hkv, d, status);
+    p.Opart = Opart; p.mpart = mpart; p.lpart = lpart;
+    p.M = M;
+    p.chunk = probe_tc_chunk(N, ns);
+    p.ns = probe_tc_splits(N, ns);      // splits launched = the stride of the partial outputs
+    return launch_tc_d<kModeProbe>(d, Qpr, K, V, p, (long long)B * Hq * kBM, B, Hkv, dim3(p.ns, B * Hq), s);
 }
 
 cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
-                                 int Hkv, int N, int* status, bool stall, cudaStream_t s) {
-    TcParams p = params(O, lse, N, Hq / Hkv, status);
+                                 int Hkv, int N, int d, int* status, bool stall, cudaStream_t s) {
+    TcParams p = params(O, lse, N, Hq / Hkv, d, status);
     p.stall = stall ? 1 : 0;
     dim3 grid((N + 2 * kBM - 1) / (2 * kBM), B * Hq);
-    return launch_tc<kModeDense>(Q, K, V, p, B, Hq, Hkv, grid, s);
+    return launch_tc_d<kModeDense>(d, Q, K, V, p, (long long)B * Hq * N, B, Hkv, grid, s);
 }
 
 }  // namespace spr

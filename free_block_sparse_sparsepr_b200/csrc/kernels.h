@@ -49,17 +49,12 @@ cudaError_t launch_group_mean_bf16(const bf16* Y, const int32_t* perm, const int
 bool km_tc_supported(int G);
 cudaError_t launch_km_split_rows(const float* X, bf16* X2, float* xx, int P, int n, int DP, cudaStream_t s);
 cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int P, int G, int DP, cudaStream_t s);
-// fix: km_fix_slots(P, n, num_sms) int4 slots (each CTA owns a region); fix_count: one int per
-// CTA (P * num_sms at most).
+// fix: km_fix_slots(P, n, num_sms) int4 slots (each CTA owns a region for the rows it flags and
+// settles exactly in fp64 at its end, correcting labels and moved counts).
 size_t km_fix_slots(int P, int n, int num_sms);
 cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx, const float* C, const bf16* C2,
                                 const float* cc, int32_t* labels, int* changed, const int* done, int4* fix,
-                                int* fix_count, int* status, int P, int n, int G, int DP, bool first, int num_sms,
-                                cudaStream_t s);
-// Exact fp64 resolution of the rows the assignment flagged (labels and moved counts corrected).
-cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, const float* cc,
-                            int32_t* labels, int* changed, const int* done, int P, int n, int G, int DP, int num_sms,
-                            cudaStream_t s);
+                                int* status, int P, int n, int G, int DP, bool first, int num_sms, cudaStream_t s);
 // dist[z][i] = fp32 of the fp64 squared distance of row i to its own centroid.
 cudaError_t launch_km_dist(const float* X, const float* C, const int32_t* labels, float* dist, int P, int n, int G,
                            int DP, cudaStream_t s);
@@ -71,8 +66,17 @@ cudaError_t launch_logits_tc(const bf16* Q, const bf16* chi, const bf16* clo, co
 cudaError_t launch_split_bf16(const float* x, bf16* hi, bf16* lo, long long count, cudaStream_t s);
 
 // Support diagnostic: out[z][s] = (smallest k whose k largest exp(F[.][s] - max) hold 90% of the
-// row's softmax mass) / N, for s < S; F [P][N][DP] fp32 (DP a multiple of 8, S <= DP).
-cudaError_t launch_topmass(const float* F, float* out, int P, int N, int DP, int S, cudaStream_t s);
+// row's softmax mass) / N, for s < S; F [P][N][DP] fp32 (DP a multiple of 8, S <= DP). colmax
+// (optional, [P][DP]): the column maxima as written by launch_resp_tc, which saves one pass.
+cudaError_t launch_topmass(const float* F, float* out, const unsigned* colmax, int P, int N, int DP, int S,
+                           cudaStream_t s);
+// Sampled responses on the tensor cores (d in {64, 128}, DP a multiple of 16 up to 64):
+// F[z][j][s] = K[z][j] . Qs[z][s] / sqrt(d) for every key j, with the two bf16 parts of F in X2
+// ([2][P*N][DP]) and ||F[z][j]||^2 in xx; colmax (optional, [P][DP]) receives order-preserving
+// keys of the maxima of the first S columns over all keys. Qs [P][DP][d], rows >= S zero.
+bool resp_tc_supported(int d, int DP);
+cudaError_t launch_resp_tc(const bf16* K, const bf16* Qs, float* F, bf16* X2, float* xx, unsigned* colmax, int P,
+                           int N, int d, int DP, int S, int num_sms, int* status, cudaStream_t s);
 // Affine diagnostics: per query head, [explained fraction, orthogonal energy] of R = Od - Os.
 size_t affine_diag_workspace(int Hp, int d);
 cudaError_t launch_affine_diag(const bf16* Os, const bf16* Od, double* out, void* ws, int Hp, int N, int d,
@@ -144,7 +148,9 @@ cudaError_t launch_attn_dense(const bf16* Q, const bf16* K, const bf16* V, bf16*
                               int B, int Hq, int Hkv, int N, int d, cudaStream_t s);
 // tcgen05/TMEM versions (head dimension 128): two 128-row query tiles per CTA, 128-key tiles.
 bool attn_tc_supported(int d);
-int attn_tc_rows_per_cta();
+// Query rows one CTA covers: two 128-row tiles of one head, or (g even) one tile of two heads.
+bool attn_tc_head_pairs(int g);
+int attn_tc_rows_per_cta(int g);
 // Key tiles (start row, valid keys) of every query group's merged kept runs: cnt [P][Gq]
 // scratch, off [P][Gq+1] absolute offsets, list of key_tiles_capacity(N, Gq, Gk) * P entries.
 long long key_tiles_capacity(int N, int Gq, int Gk);
@@ -152,10 +158,24 @@ cudaError_t launch_key_tiles(const int32_t* rowptr, const int32_t* kg, const int
                              int32_t* off, int2* list, int P, int N, int Gq, int Gk, cudaStream_t s);
 cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp, const int32_t* qoff,
                                   const int32_t* tile_off, const int2* klist, const int32_t* klist_off, bf16* O,
-                                  float* lse, int B, int Hq, int Hkv, int N, int Gq, int* status, cudaStream_t s);
+                                  float* lse, int B, int Hq, int Hkv, int N, int d, int Gq, int* status,
+                                  cudaStream_t s);
 // stall: test only -- the producer issues no loads, so the first bounded wait runs out.
 cudaError_t launch_attn_dense_tc(const bf16* Q, const bf16* K, const bf16* V, bf16* O, float* lse, int B, int Hq,
-                                 int Hkv, int N, int* status, bool stall, cudaStream_t s);
+                                 int Hkv, int N, int d, int* status, bool stall, cudaStream_t s);
+// Probe rows on the tensor cores (d = 128): the M (<= 128) probe rows of every query head
+// gathered into Qpr [B*Hq][128][d] (rows >= M zero), attended against all keys in
+// probe_tc_splits(N, ns) splits of probe_tc_chunk(N, ns) keys; partial outputs, maxima and
+// sums in the layout of launch_attn_probe, merged by launch_probe_combine.
+cudaError_t launch_gather_probe_rows(const bf16* Q, const int32_t* probe, bf16* Qpr, int B, int Hq, int Hkv, int N,
+                                    int M, int d, int rows, cudaStream_t s);
+int probe_tc_chunk(int N, int ns);
+int probe_tc_splits(int N, int ns);
+cudaError_t launch_attn_probe_tc(const bf16* Qpr, const bf16* K, const bf16* V, float* Opart, float* mpart,
+                                 float* lpart, int B, int Hq, int Hkv, int N, int d, int M, int ns, int* status,
+                                 cudaStream_t s);
+cudaError_t launch_probe_combine(const float* Opart, const float* mpart, const float* lpart, float* Odense, int Hp,
+                                 int M, int ns, int d, cudaStream_t s);
 // Dense attention of gathered probe rows, split over ns key chunks, then combined.
 cudaError_t launch_attn_probe(const bf16* Q, const bf16* K, const bf16* V, const int32_t* probe,
                               float* Opart, float* mpart, float* lpart, float* Odense, int B,
@@ -176,6 +196,14 @@ cudaError_t launch_writeback(const bf16* Osp, const int32_t* qperm, const float*
 cudaError_t launch_writeback_ridge(const bf16* Osp, const int32_t* qperm, const float* A, const float* obar,
                                    const float* Rbar, bf16* O, int Hp, int g, int N, int d, int num_sms,
                                    cudaStream_t s);
+// Correction and write-back on the tensor cores (d = 128, r <= 32): O[qperm[p]] = o + U (c0 + Bm o)
+// (+ Radd) for every group-major row o of Osp; parts: wb_tc_parts_elems(Hp) bf16 of scratch for the
+// bf16 parts of Bm and U^T.
+bool wb_tc_supported(int d, int r);
+size_t wb_tc_parts_elems(int Hp);
+cudaError_t launch_writeback_tc(const bf16* Osp, const int32_t* qperm, const float* U, const float* Bm,
+                                const float* c0, const float* Radd, bf16* parts, bf16* O, int Hp, int g, int N, int r,
+                                int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_probe_override(const float* Odense, const int32_t* probe, bf16* O, int Hp,
                                   int g, int N, int d, int M, cudaStream_t s);
 

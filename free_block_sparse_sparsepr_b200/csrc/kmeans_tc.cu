@@ -5,16 +5,20 @@
 // Rows and centroids are split into two bf16 parts (x = x0 + x1 + e, |e| <= 2^-16 |x|
 // elementwise) and the three terms x0 c0 + x0 c1 + x1 c0 are accumulated in fp32 TMEM, so
 // each dot product is known to within about 2^-14 ||x|| ||c||. One epilogue thread per row
-// takes the best and second-best of dd_g = ||c_g||^2 - 2 x.c_g straight from its TMEM lane.
-// When the gap between them exceeds a bound on the estimate's error the estimate decides;
-// otherwise (about 1% of rows) the row goes to a list, and a second kernel settles it exactly:
-// an fp32 pass over all centroids keeps those within a relative 1e-4 of the nearest, and each
-// of those gets ||x||^2 - 2 x.c + ||c||^2 in fp64 from the fp32 rows and centroids, rounded to
-// fp32, ties to the lowest group. The labels are therefore those of the fp32 distances
-// themselves.
+// reads dd_g = ||c_g||^2 - 2 x.c_g straight from its TMEM lane in two passes: the first keeps
+// only the smallest dd of every 32-column chunk (three-input minima, about half an ALU
+// instruction per distance), the second reloads the winning chunk to find its argmin (lowest
+// column on ties) and to count its distances within the certificate's gap of the minimum.
+// When no other distance (in that chunk, or as another chunk's minimum) lies within a bound on
+// the estimate's error, the estimate decides; otherwise (about 1% of rows) the row goes to a
+// list that the same CTA settles exactly at its end: an fp32 pass over all centroids keeps
+// those within a relative 1e-4 of the nearest, and each of those gets ||x||^2 - 2 x.c + ||c||^2
+// in fp64 from the fp32 rows and centroids, rounded to fp32, ties to the lowest group. The
+// labels are therefore those of the fp32 distances themselves.
 //
 // Warps 0-7 epilogue (two warpgroups taking alternate tiles, one TMEM buffer each), warp 8
-// TMA producer (centroids once, row tiles in a 3-stage ring), warp 9 MMA issuer.
+// TMA producer (centroids once, row tiles in a 3-stage ring), warp 9 MMA issuer; all ten warps
+// share the exact settlement of the flagged rows at the end.
 #include <float.h>
 #include <math.h>
 #include <string.h>
@@ -66,7 +70,6 @@ struct KmParams {
     const int* done;       // [P] or null
     int* status;
     int4* fix;             // flagged rows {row, previous label, estimate, 0}; fix_cap slots per CTA
-    int* fix_count;        // [P * gridDim.x] rows each CTA flagged
     int n, G, G16, G32, DP, ksteps, first, fix_cap;
 };
 
@@ -82,12 +85,13 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
     return r;
 }
 
-__device__ __forceinline__ double warp_sum_d(double v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-    return v;
-}
 
+template <int DP>
+__device__ __forceinline__ void settle_row(const int4 h, const float* __restrict__ X, const float* sCk,
+                                           const float* sCC, float cmax2, int G, int32_t* labels, int* changed,
+                                           int z, int lane);
+
+template <int DP>
 __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_constant__ KmMaps maps,
                                                                    const KmParams p) {
     const int z = blockIdx.y;
@@ -204,40 +208,43 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
             const long long o = (long long)z * p.n + row;
             const float xxr = valid ? __ldg(p.xx + o) : 0.f;
             const int prev = (valid && !p.first) ? p.labels[o] : -1;
-            // Keys: dd with its low 5 bits replaced by the column within the 32-column chunk,
-            // so one min also carries the argmin; four chains (column mod 4) for ILP, and the
-            // chunk that last lowered each chain's minimum.
-            float b1[4], b2[4];
-            int bc[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) { b1[j] = INFINITY; b2[j] = INFINITY; bc[j] = 0; }
-            auto scan = [&](const uint32_t* v, int c) {
-                float old[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) old[j] = b1[j];
-                const float4* cc4 = reinterpret_cast<const float4*>(sCC + c);
-#pragma unroll
-                for (int q = 0; q < 8; q += 2) {
-                    const float4 ca = cc4[q], cb = cc4[q + 1];
-                    const float ce[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // Columns e and e + 4 of chain j: the two smallest of {b1, b2, k1, k2}.
-                        const uint32_t e = (uint32_t)(4 * q + j);
-                        const float d1 = fmaf(-2.f, __uint_as_float(v[e]), ce[j]);
-                        const float d2 = fmaf(-2.f, __uint_as_float(v[e + 4]), ce[j + 4]);
-                        const float k1 = __uint_as_float((__float_as_uint(d1) & ~31u) | e);
-                        const float k2 = __uint_as_float((__float_as_uint(d2) & ~31u) | (e + 4));
-                        const float lo = fminf(k1, k2), hi = fmaxf(k1, k2);
-                        b2[j] = fmin3(b2[j], fmaxf(b1[j], lo), hi);
-                        b1[j] = fminf(b1[j], lo);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) bc[j] = b1[j] != old[j] ? c : bc[j];
-            };
             if (!__all_sync(kFull, tc::mbar_wait(bar(kBarDF + wg), (i >> 1) & 1, abort_flag))) break;
             tc::fence_after_sync();
+            // One pass over the row's distances, 32 columns (one TMEM load) at a time: dd of the
+            // chunk, its minimum by three-input minima, and, when that minimum is a new best (B1),
+            // the chunk's 32 values copied into `best` by predicated selects; B2c is the smallest
+            // of the other chunks' minima. The near-tie count and the argmin (lowest column on
+            // ties) then come from `best` in registers, with no second read of TMEM.
+            float B1 = INFINITY, B2c = INFINITY;
+            int cb = 0;
+            float best[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) best[e] = INFINITY;
+            auto chunk = [&](uint32_t* v, int c) {
+                // dd overwrites the loaded dot products in place
+                const float4* cc4 = reinterpret_cast<const float4*>(sCC + c);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 ce = cc4[q];
+                    v[4 * q] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q]), ce.x));
+                    v[4 * q + 1] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q + 1]), ce.y));
+                    v[4 * q + 2] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q + 2]), ce.z));
+                    v[4 * q + 3] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q + 3]), ce.w));
+                }
+                auto dd = [&](int e) { return __uint_as_float(v[e]); };
+                float mm[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mm[j] = fmin3(fmin3(dd(j), dd(j + 4), dd(j + 8)), fmin3(dd(j + 12), dd(j + 16), dd(j + 20)),
+                                  fminf(dd(j + 24), dd(j + 28)));
+                const float mc = fminf(fmin3(mm[0], mm[1], mm[2]), mm[3]);
+                const bool nb = mc < B1;
+                B2c = nb ? B1 : fminf(B2c, mc);
+                B1 = nb ? mc : B1;
+                cb = nb ? c : cb;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) best[e] = nb ? dd(e) : best[e];
+            };
             {
                 uint32_t va[32], vb[32];
                 tc::tmem_ld32(tb, va);
@@ -246,12 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                 for (int c = 0; c < p.G32; c += 64) {
                     const bool hb = c + 32 < p.G32, ha = c + 64 < p.G32;
                     if (hb) tc::tmem_ld32(tb + (uint32_t)(c + 32), vb);
-                    scan(va, c);
+                    chunk(va, c);
                     if (hb) {
                         tc::tmem_wait_ld();
                         tc::regs_after_wait(vb);
                         if (ha) tc::tmem_ld32(tb + (uint32_t)(c + 64), va);
-                        scan(vb, c + 32);
+                        chunk(vb, c + 32);
                         if (ha) {
                             tc::tmem_wait_ld();
                             tc::regs_after_wait(va);
@@ -259,22 +266,21 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                     }
                 }
             }
+            const float T = 4.f * kKappa * sqrtf(xxr) * cmax + kSlack * (xxr + cmax2);
+            const float thr = B1 + T;
+            int idx = 31;
+            float near = 0.f;
+#pragma unroll
+            for (int e = 31; e >= 0; --e) {
+                idx = best[e] == B1 ? e : idx;
+                near += best[e] <= thr ? 1.f : 0.f;
+            }
+            const int I1 = min(cb + idx, p.G - 1);
             tc::fence_before_sync();
             tc::mbar_arrive(bar(kBarDE + wg));
-            int jw = 0;
-            float B1 = b1[0];
-            int I1 = bc[0];
-#pragma unroll
-            for (int j = 1; j < 4; ++j)
-                if (b1[j] < B1) { B1 = b1[j]; I1 = bc[j]; jw = j; }
-            I1 += (int)(__float_as_uint(B1) & 31u);
-            float B2 = INFINITY;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) B2 = fminf(B2, j == jw ? b2[j] : fminf(b1[j], b2[j]));
 
-            const float T = 4.f * kKappa * sqrtf(xxr) * cmax + kSlack * (xxr + cmax2);
-            const bool flag = valid && !(B2 - B1 > T);
-            // Hand each flagged row to the exact pass.
+            const bool flag = valid && !(B2c - B1 > T && near < 1.5f);
+            // Hand each flagged row to the exact settlement at the end of the kernel.
             const unsigned fl = __ballot_sync(kFull, flag);
             if (fl) {
                 int slot = 0;
@@ -294,13 +300,100 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
 
     tc::fence_before_sync();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        if (*abort_flag) set_status(p.status, kDevTimeout);
-        p.fix_count[cta] = *sFix;
-    }
+    if (threadIdx.x == 0 && *abort_flag) set_status(p.status, kDevTimeout);
     if (warp == 9) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
+    }
+    // Exact settlement of this CTA's flagged rows, one warp per row. Every copy and MMA has
+    // completed, so the row stages hold the fp32 centroids k-major ([DP][G]: lane g of a warp
+    // reads centroid g's component k without bank conflicts).
+    const int nfix = *sFix;
+    if (nfix > 0 && !*abort_flag) {
+        float* sCk = reinterpret_cast<float*>(sbase + kOffX);
+        const float* src = p.C + (long long)z * p.G * DP;
+        for (int t = threadIdx.x; t < p.G * DP; t += kThreads) sCk[(t % DP) * (p.G + 1) + t / DP] = __ldg(src + t);
+        __syncthreads();
+        float cmax2 = 0.f;
+        for (int g = 0; g < p.G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
+        for (int w = warp; w < nfix; w += kThreads / 32)
+            settle_row<DP>(fix[w], p.X, sCk, sCC, cmax2, p.G, p.labels, p.changed, z, lane);
+    }
+}
+
+// Exact label of one flagged row {row, previous label, estimate, 0}, settled by one warp (centroids
+// k-major in sCk with row stride G + 1, so staging and lane-parallel reads avoid bank conflicts; lane
+// g + 32j takes centroid g + 32j): candidates are the groups whose fp32 ||x||^2 - 2 x.c + ||c||^2
+// (error below 2^-19 (||x||^2 + ||c||^2)) is within 1e-4 (|d_min| + ||x||^2 + max ||c||^2) of the
+// smallest; each gets the fp32 value of its fp64 distance (butterfly sums, identical in every
+// lane), argmin with ties to the lowest group. Corrects the label and the count of rows that
+// moved.
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+template <int DP>
+__device__ __forceinline__ void settle_row(const int4 h, const float* __restrict__ X, const float* sCk,
+                                           const float* sCC, float cmax2, int G, int32_t* labels, int* changed,
+                                           int z, int lane) {
+    static_assert(DP <= 64, "two row components per lane");
+    const long long o = h.x;
+    const float* xr = X + o * DP;
+    const float xa = lane < DP ? __ldg(xr + lane) : 0.f;
+    const float xb = lane + 32 < DP ? __ldg(xr + lane + 32) : 0.f;
+    const float xx = warp_sum(fmaf(xa, xa, xb * xb));
+    const int nj = (G + 31) / 32;
+    float dj[kMaxG / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxG / 32; ++j) dj[j] = INFINITY;
+    float dmin = INFINITY;
+    // not unrolled: each chunk of 32 centroids re-broadcasts the row (keeps registers low)
+#pragma unroll 1
+    for (int j = 0; j < kMaxG / 32; ++j) {
+        if (j < nj) {
+            const int g = 32 * j + lane;
+            const int gc = g < G ? g : G - 1;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < DP; k += 2) {
+                a0 = fmaf(__shfl_sync(kFull, k < 32 ? xa : xb, k & 31), sCk[k * (G + 1) + gc], a0);
+                a1 = fmaf(__shfl_sync(kFull, k + 1 < 32 ? xa : xb, (k + 1) & 31), sCk[(k + 1) * (G + 1) + gc], a1);
+            }
+            const float dg = g < G ? fmaf(-2.f, a0 + a1, xx + sCC[g]) : INFINITY;
+#pragma unroll
+            for (int jj = 0; jj < kMaxG / 32; ++jj) dj[jj] = jj == j ? dg : dj[jj];
+            dmin = fminf(dmin, dg);
+        }
+    }
+    dmin = warp_min(dmin);
+    const float thr = dmin + 1e-4f * (fabsf(dmin) + xx + cmax2);
+    const double xxd = warp_sum_d(fma((double)xa, (double)xa, (double)xb * (double)xb));
+    float best = INFINITY;
+    int bg = h.z;
+#pragma unroll
+    for (int j = 0; j < kMaxG / 32; ++j) {
+        if (j >= nj) break;
+        unsigned m = __ballot_sync(kFull, dj[j] <= thr);
+        while (m) {
+            const int g = 32 * j + __ffs(m) - 1;
+            m &= m - 1;
+            const double ca = lane < DP ? (double)sCk[lane * (G + 1) + g] : 0.0;
+            const double cb = lane + 32 < DP ? (double)sCk[(lane + 32) * (G + 1) + g] : 0.0;
+            const double xc = warp_sum_d(fma((double)xa, ca, (double)xb * cb));
+            const double ccd = warp_sum_d(fma(ca, ca, cb * cb));
+            const float d = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
+            if (d < best || (d == best && g < bg)) { best = d; bg = g; }
+        }
+    }
+    if (lane == 0) {
+        labels[o] = bg;
+        const int prev = h.y;
+        if (prev >= 0) {
+            const int dmoved = (prev != bg ? 1 : 0) - (prev != h.z ? 1 : 0);
+            if (dmoved) atomicAdd(&changed[z], dmoved);
+        }
     }
 }
 
@@ -373,119 +466,6 @@ __global__ void km_split_cent_kernel(const float* __restrict__ C, bf16* C2, long
     if (lane == 0) cc[(long long)z * G32 + g] = g < G ? ss : kFar;
 }
 
-// Exact pass over the flagged rows: kFixSplit blocks per assignment CTA's region, one thread
-// per row, the row in registers and the centroids staged row-major in shared memory (every
-// centroid read is a broadcast to the warp). Candidates are the groups whose fp32
-// ||x||^2 - 2 x.c + ||c||^2 (error below 2^-19 (||x||^2 + ||c||^2)) is within 1e-4 (d + ||x||^2
-// + max ||c||^2) of the smallest: the four smallest are kept while scanning, and only a row with
-// more candidates than that scans again. Each candidate gets the fp32 value of its fp64
-// distance, argmin with ties to the lowest group. Corrects the label and the moved count.
-constexpr int kFixThreads = 128;
-constexpr int kFixSplit = 2;   // blocks per assignment CTA's region
-template <int DP>
-__global__ void __launch_bounds__(kFixThreads) km_fixup_kernel(const int4* __restrict__ fix,
-                                                               const int* __restrict__ fix_count,
-                                                               const float* __restrict__ X,
-                                                               const float* __restrict__ C,
-                                                               const float* __restrict__ cc, int32_t* labels,
-                                                               int* changed, const int* done, int n, int G, int G32,
-                                                               int fix_cap) {
-    const int z = blockIdx.y;
-    if (done && done[z]) return;
-    const int cta = z * gridDim.x + blockIdx.x;
-    const int cnt = fix_count[cta];
-    if (blockIdx.z * kFixThreads >= cnt) return;            // no flagged row for this block
-    extern __shared__ __align__(16) float fsm[];
-    float* sC = fsm;                          // [G][DP]
-    float* sCC = fsm + (size_t)G * DP;        // [G]
-    {
-        const float4* src = reinterpret_cast<const float4*>(C + (long long)z * G * DP);
-        float4* dst = reinterpret_cast<float4*>(sC);
-        for (int t = threadIdx.x; t < G * DP / 4; t += kFixThreads) dst[t] = __ldg(src + t);
-        for (int t = threadIdx.x; t < G; t += kFixThreads) sCC[t] = cc[(long long)z * G32 + t];
-    }
-    __syncthreads();
-    float cmax2 = 0.f;
-    for (int g = 0; g < G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
-    const int4* reg = fix + (long long)cta * fix_cap;
-    for (int w = blockIdx.z * kFixThreads + threadIdx.x; w < cnt; w += gridDim.z * kFixThreads) {
-        const int4 h = reg[w];
-        const long long o = h.x;
-        const float4* xr4 = reinterpret_cast<const float4*>(X + o * DP);
-        float x[DP];
-#pragma unroll
-        for (int k = 0; k < DP / 4; ++k) {
-            const float4 q = __ldg(xr4 + k);
-            x[4 * k] = q.x; x[4 * k + 1] = q.y; x[4 * k + 2] = q.z; x[4 * k + 3] = q.w;
-        }
-        float xx = 0.f;
-#pragma unroll
-        for (int k = 0; k < DP; ++k) xx = fmaf(x[k], x[k], xx);
-        auto dist32 = [&](int g) -> float {
-            const float4* c4 = reinterpret_cast<const float4*>(sC + g * DP);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-            for (int k = 0; k < DP / 4; ++k) {
-                const float4 c = c4[k];
-                a0 = fmaf(x[4 * k], c.x, a0);
-                a1 = fmaf(x[4 * k + 1], c.y, a1);
-                a2 = fmaf(x[4 * k + 2], c.z, a2);
-                a3 = fmaf(x[4 * k + 3], c.w, a3);
-            }
-            return fmaf(-2.f, (a0 + a1) + (a2 + a3), xx + sCC[g]);
-        };
-        // the four smallest fp32 distances (ascending) and their groups
-        float t0 = INFINITY, t1 = INFINITY, t2 = INFINITY, t3 = INFINITY;
-        int i0 = 0, i1 = 0, i2 = 0, i3 = 0;
-#pragma unroll 1
-        for (int g = 0; g < G; ++g) {
-            const float d = dist32(g);
-            if (d < t3) {
-                if (d < t1) {
-                    t3 = t2; i3 = i2; t2 = t1; i2 = i1;
-                    if (d < t0) { t1 = t0; i1 = i0; t0 = d; i0 = g; }
-                    else { t1 = d; i1 = g; }
-                } else if (d < t2) { t3 = t2; i3 = i2; t2 = d; i2 = g; }
-                else { t3 = d; i3 = g; }
-            }
-        }
-        const float thr = t0 + 1e-4f * (fabsf(t0) + xx + cmax2);
-        double xxd = 0.0;
-#pragma unroll
-        for (int k = 0; k < DP; ++k) xxd = fma((double)x[k], (double)x[k], xxd);
-        float best = INFINITY;
-        int bg = h.z;
-        auto exact = [&](int g) {
-            const float* cg = sC + g * DP;
-            double xc = 0.0, ccd = 0.0;
-#pragma unroll
-            for (int k = 0; k < DP; ++k) {
-                const double c = (double)cg[k];
-                xc = fma((double)x[k], c, xc);
-                ccd = fma(c, c, ccd);
-            }
-            const float d = (float)fmax((xxd - 2.0 * xc) + ccd, 0.0);
-            if (d < best || (d == best && g < bg)) { best = d; bg = g; }
-        };
-        // candidates: the (at most three) kept groups within thr, or, when the fourth smallest is
-        // within thr too, every group within thr (found by scanning again)
-        const bool all = t3 <= thr;
-        const int ncand = all ? G : 1 + (t1 <= thr ? 1 : 0) + (t2 <= thr ? 1 : 0);
-#pragma unroll 1
-        for (int q = 0; q < ncand; ++q) {
-            const int g = all ? q : (q == 0 ? i0 : (q == 1 ? i1 : i2));
-            if (all && !(dist32(g) <= thr)) continue;
-            exact(g);
-        }
-        labels[o] = bg;
-        const int prev = h.y;
-        if (prev >= 0) {
-            const int dmoved = (prev != bg ? 1 : 0) - (prev != h.z ? 1 : 0);
-            if (dmoved) atomicAdd(&changed[z], dmoved);
-        }
-    }
-}
-
 // dist[z][i] = fp32(max(||x||^2 - 2 x.c + ||c||^2, 0)) in fp64 for the row's own centroid;
 // one thread per row.
 __global__ void km_dist_kernel(const float* __restrict__ X, const float* __restrict__ C,
@@ -540,8 +520,7 @@ cudaError_t launch_km_split_cent(const float* C, bf16* C2, float* cc, int P, int
 
 cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx, const float* C, const bf16* C2,
                                 const float* cc, int32_t* labels, int* changed, const int* done, int4* fix,
-                                int* fix_count, int* status, int P, int n, int G, int DP, bool first, int num_sms,
-                                cudaStream_t s) {
+                                int* status, int P, int n, int G, int DP, bool first, int num_sms, cudaStream_t s) {
     if (DP < 16 || DP > kMaxDP || DP % 16 != 0 || (long long)P * n >= (1ll << 31)) return cudaErrorInvalidValue;
     const int G16 = (G + 15) / 16 * 16, G32 = (G + 31) / 32 * 32;
     KmMaps maps;
@@ -553,42 +532,27 @@ cudaError_t launch_km_assign_tc(const float* X, const bf16* X2, const float* xx,
     KmParams p;
     memset(&p, 0, sizeof(p));
     p.X = X; p.C = C; p.xx = xx; p.cc = cc; p.labels = labels; p.changed = changed; p.done = done;
-    p.status = status; p.fix = fix; p.fix_count = fix_count;
+    p.status = status; p.fix = fix;
     p.n = n; p.G = G; p.G16 = G16; p.G32 = G32; p.DP = DP; p.ksteps = DP / 16; p.first = first ? 1 : 0;
     int per, cap;
     km_grid(P, n, num_sms, &per, &cap);
     p.fix_cap = cap;
-    cudaError_t e = cudaFuncSetAttribute(km_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    km_assign_tc_kernel<<<dim3(per, P), kThreads, kSmemBytes, s>>>(maps, p);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_km_fixup(const int4* fix, const int* fix_count, const float* X, const float* C, const float* cc,
-                            int32_t* labels, int* changed, const int* done, int P, int n, int G, int DP, int num_sms,
-                            cudaStream_t s) {
-    int per, cap;
-    km_grid(P, n, num_sms, &per, &cap);
-    const int G32 = (G + 31) / 32 * 32;
-    const size_t smem = ((size_t)G * DP + G) * sizeof(float);
-    const dim3 grid(per, P, kFixSplit);
-#define SPR_FIXUP(DPV)                                                                                               \
+#define SPR_ASSIGN(DPV)                                                                                              \
     case DPV: {                                                                                                      \
-        cudaError_t e = cudaFuncSetAttribute(km_fixup_kernel<DPV>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
-                                             (int)smem);                                                             \
+        cudaError_t e = cudaFuncSetAttribute(km_assign_tc_kernel<DPV>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                             kSmemBytes);                                                            \
         if (e != cudaSuccess) return e;                                                                              \
-        km_fixup_kernel<DPV><<<grid, kFixThreads, smem, s>>>(fix, fix_count, X, C, cc, labels, changed, done, n, G,  \
-                                                            G32, cap);                                               \
+        km_assign_tc_kernel<DPV><<<dim3(per, P), kThreads, kSmemBytes, s>>>(maps, p);                                \
         break;                                                                                                       \
     }
     switch (DP) {
-        SPR_FIXUP(16)
-        SPR_FIXUP(32)
-        SPR_FIXUP(48)
-        SPR_FIXUP(64)
+        SPR_ASSIGN(16)
+        SPR_ASSIGN(32)
+        SPR_ASSIGN(48)
+        SPR_ASSIGN(64)
         default: return cudaErrorInvalidValue;
     }
-#undef SPR_FIXUP
+#undef SPR_ASSIGN
     return cudaGetLastError();
 }
 

@@ -49,10 +49,27 @@ __global__ void cell_scores_kernel(const float* __restrict__ u, const float* __r
                 const long long x = (long long)z * g + j;
                 const float* ux = u + x * N * Gk;
                 const float* lx = lse + x * N;
-                for (int p = lo; p < hi; ++p) {
-                    int i = perm[p];
-                    acc += expf(ux[(long long)i * Gk + gk] - lx[i]);
+                // eight rows in flight, four partial sums added in a fixed order
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                int p = lo;
+                for (; p + 8 <= hi; p += 8) {
+                    int i8[8];
+                    float v8[8], l8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) i8[e] = __ldg(perm + p + e);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        v8[e] = __ldg(ux + (long long)i8[e] * Gk + gk);
+                        l8[e] = __ldg(lx + i8[e]);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a4[e & 3] += expf(v8[e] - l8[e]);
                 }
+                for (; p < hi; ++p) {
+                    const int i = __ldg(perm + p);
+                    a4[0] += expf(__ldg(ux + (long long)i * Gk + gk) - __ldg(lx + i));
+                }
+                acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
             }
         }
         scores[((long long)z * Gq + a) * Gk + gk] = ok ? acc / ((float)g * (float)(hi - lo)) : 0.f;

@@ -43,10 +43,16 @@ struct Smem {
 
 enum { kLayoutFeatures = 0, kLayoutRows = 1 };
 
+// Inverse of the order-preserving key the response GEMM's epilogue stores for each column maximum.
+__device__ __forceinline__ float from_max_key(unsigned k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads) support_kernel(const float* __restrict__ src, float* out,
                                                            float* out_union, const int32_t* __restrict__ qoff,
-                                                           int N, int ld, int S, int Gq, int z0) {
+                                                           const unsigned* __restrict__ colmax, int N, int ld,
+                                                           int S, int Gq, int z0) {
     extern __shared__ unsigned char sm_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(sm_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -85,24 +91,30 @@ __global__ void __launch_bounds__(kThreads) support_kernel(const float* __restri
         }
     };
 
-    // ---- pass 1: maxima
+    // ---- pass 1: maxima (taken from the response GEMM's epilogue when it formed them)
     float v[kCols], acc[kCols];
+    if (LAYOUT == kLayoutFeatures && colmax) {
+        if (tid < kCols)
+            sm.red[0][tid] = tid < ncol ? from_max_key(colmax[(long long)z * ld + blockIdx.x * kCols + tid]) : -INFINITY;
+    } else {
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) acc[c] = -INFINITY;
-    for (long long j = tid; j < N; j += kThreads) {
-        load_row(j, v);
+        for (int c = 0; c < kCols; ++c) acc[c] = -INFINITY;
+        for (long long j = tid; j < N; j += kThreads) {
+            load_row(j, v);
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) acc[c] = fmaxf(acc[c], v[c]);
-    }
+            for (int c = 0; c < kCols; ++c) acc[c] = fmaxf(acc[c], v[c]);
+        }
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) {
-        const float r = warp_max(acc[c]);
-        if (lane == 0) sm.red[warp][c] = r;
+        for (int c = 0; c < kCols; ++c) {
+            const float r = warp_max(acc[c]);
+            if (lane == 0) sm.red[warp][c] = r;
+        }
     }
     __syncthreads();
     if (tid < kCols) {
         float r = -INFINITY;
-        for (int w = 0; w < kThreads / 32; ++w) r = fmaxf(r, sm.red[w][tid]);
+        const int nw = (LAYOUT == kLayoutFeatures && colmax) ? 1 : kThreads / 32;
+        for (int w = 0; w < nw; ++w) r = fmaxf(r, sm.red[w][tid]);
         sm.mx[tid] = r;
         sm.lo[tid] = 0.f;
         sm.width[tid] = 0.125f;
@@ -318,14 +330,15 @@ __global__ void __launch_bounds__(kThreads) support_kernel(const float* __restri
 
 }  // namespace
 
-cudaError_t launch_topmass(const float* F, float* out, int P, int N, int DP, int S, cudaStream_t s) {
+cudaError_t launch_topmass(const float* F, float* out, const unsigned* colmax, int P, int N, int DP, int S,
+                           cudaStream_t s) {
     if (DP % kCols != 0 || S > DP) return cudaErrorInvalidValue;
     const size_t smem = sizeof(Smem);
     cudaError_t e = cudaFuncSetAttribute(support_kernel<kLayoutFeatures>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     support_kernel<kLayoutFeatures><<<dim3((S + kCols - 1) / kCols, P), kThreads, smem, s>>>(F, out, nullptr, nullptr,
-                                                                                            N, DP, S, 0, 0);
+                                                                                            colmax, N, DP, S, 0, 0);
     return cudaGetLastError();
 }
 
@@ -336,7 +349,7 @@ cudaError_t launch_shared_support(const float* Z, long long ldz, const int32_t* 
                                          (int)smem);
     if (e != cudaSuccess) return e;
     if (ldz > INT_MAX) return cudaErrorInvalidValue;
-    support_kernel<kLayoutRows><<<dim3(Gq, nz), kThreads, smem, s>>>(Z, row_frac, union_frac, qoff, N, (int)ldz,
+    support_kernel<kLayoutRows><<<dim3(Gq, nz), kThreads, smem, s>>>(Z, row_frac, union_frac, qoff, nullptr, N, (int)ldz,
                                                                      kCols, Gq, z0);
     return cudaGetLastError();
 }

@@ -69,7 +69,7 @@ typedef enum sparsepr_status {
                                                       of width d; `features` then holds the keys); not with
                                                       SPARSEPR_FLAG_TOPMASS */
 #define SPARSEPR_FLAG_STAGE_TIMING      (1u << 8)  /* record per-stage CUDA events (sparsepr_get_stats) */
-#define SPARSEPR_FLAG_TEST_STALL        (1u << 9)  /* TEST ONLY (d = 128): the kernel of sparsepr_dense_attn issues
+#define SPARSEPR_FLAG_TEST_STALL        (1u << 9)  /* TEST ONLY: the kernel of sparsepr_dense_attn issues
                                                       no loads, so its first bounded wait runs out (about 2 s of SM
                                                       clock), every CTA returns with its TMEM freed and nothing in
                                                       flight, the output rows are written as zeros and the device

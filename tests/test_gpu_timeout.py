@@ -56,9 +56,3 @@ def test_bounded_wait_runs_out_and_reports_timeout():
         assert h.device_status() == 0
     assert_close(bf16_to_f64(Od), oracle.dense_attention(Q, K, V), "dense attention after the timeout")
     assert torch.isfinite(O2.float()).all()
-
-
-def test_stall_flag_needs_the_tensor_core_kernel():
-    with pytest.raises(spr.SparsePRError) as e:
-        spr.SparsePR.from_workload(W.replace(d=64), flags=spr.FLAG_TEST_STALL)
-    assert e.value.code == 2
