@@ -68,23 +68,27 @@ def barrier():
         dist.barrier()
 
 
-def attn_traffic_bytes():
-    """DRAM bytes (read + write) of one block-sparse attention launch on the default workload, from the
-    committed ncu summary; None once the kernel source differs from the one the counters were taken on."""
+def attn_traffic_bytes(useful_flops: float):
+    """DRAM bytes (read + write) of one block-sparse attention launch, scaled from the committed
+    small-case ncu capture (profiles/attn_tc_kernel_sweep_n32760_rho22.md: its traffic per launch
+    and its launch's useful FLOPs) by the ratio of useful FLOPs (the attention's DRAM traffic is
+    its K/V tile reads, which grow with the routed pairs). None once the kernel source differs
+    from the one the counters were taken on."""
     import hashlib
     import re
 
     root = os.path.dirname(os.path.abspath(__file__))
     try:
-        text = open(os.path.join(root, "profiles", "attn_tc_kernel_hunyuan720p_n118800.md")).read()
+        text = open(os.path.join(root, "profiles", "attn_tc_kernel_sweep_n32760_rho22.md")).read()
         src = open(os.path.join(root, "free_block_sparse_sparsepr_b200", "csrc", "attention_tc.cu"), "rb").read()
     except OSError:
         return None
     m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    m_f = re.search(r"useful_flops_per_launch:\s*([0-9.eE+]+)", text)
     m_h = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text)
-    if not (m_t and m_h) or hashlib.sha256(src).hexdigest()[:16] != m_h.group(1):
+    if not (m_t and m_f and m_h) or hashlib.sha256(src).hexdigest()[:16] != m_h.group(1):
         return None
-    return int(m_t.group(1))
+    return int(int(m_t.group(1)) * useful_flops / float(m_f.group(1)))
 
 
 def whole_job_value(flops_per_rank: float, world: int, ms_max: float) -> float:
@@ -355,7 +359,8 @@ def run_ours(args):
     peak = peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "kernel": "block-sparse attention (routed cells)", "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": attn_traffic_bytes() if w.name == DEFAULT_WORKLOAD else None,
+                "traffic": attn_traffic_bytes(attn_flops),
+                "traffic_source": "small-case ncu capture scaled by useful FLOPs",
                 "peak_kind": f"bf16 sustained ({peaks['source']})",
                 "useful_flops_per_launch": attn_flops}
 
