@@ -30,7 +30,7 @@ inline int pad64(int v) { return (v + 63) / 64 * 64; }
 
 enum Stage { kStPartition = 0, kStRoute, kStPermute, kStAttn, kStProbeFit, kStWriteback, kStUnused, kStTotal, kNumStages };
 
-constexpr int kHostChunks = 4;     // KV-head chunks of the host-buffer pipeline
+constexpr int kHostChunks = 8;     // KV-head chunks of the host-buffer pipeline
 
 }  // namespace
 

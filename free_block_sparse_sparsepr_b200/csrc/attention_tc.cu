@@ -68,6 +68,7 @@ struct TcParams {
     int* status;
     int N, g, Gq;
     int head_pairs;               // sparse mode, g even: one CTA = the same query tile of two query heads
+    int half_tails;               // sparse mode: a lone last tile of <= 64 rows (or, head pairs, of two heads) is M = 64
     int stall;                    // test only: issue no loads (the first bounded wait runs out)
     // probe mode: M gathered rows per query head against key split blockIdx.x (chunk keys each);
     // unnormalised partial outputs [x][ns][M][d], running maxima (log2 units) and sums [x][ns][M]
@@ -197,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
     // ---- which query tiles
     int qlo, qn0, qn1, a = 0, ntk = 0;
+    bool half = false;   // an M = 64 tile (rows in lanes 0-15 of each 32-lane quarter, 16-lane TMEM shapes)
     long long qrow[2];
     const int2* klist = nullptr;
     if (MODE == kModeSparse) {
@@ -209,15 +211,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         ntk = lo[a + 1] - lo[a];
         const int32_t* qo = p.qoff + (long long)z * (p.Gq + 1);
         if (p.head_pairs) {
-            qlo = qo[a] + (pair - toff[a]) * kBM;
+            // one 128-row tile of two heads per CTA; with half tails, a last tile of at most 64 rows
+            // runs as two M = 64 tiles (one per head)
+            const int c = pair - toff[a];
+            qlo = qo[a] + c * kBM;
             qn0 = qn1 = min(kBM, qo[a + 1] - qlo);
+            half = p.half_tails && qn0 <= kBM / 2;
             qrow[0] = (long long)x * p.N + qlo;
             qrow[1] = (long long)(x + 1) * p.N + qlo;
         } else {
+            // the group's rows in pairs of 128-row tiles; with half tails, a lone last tile of at
+            // most 64 rows runs as an M = 64 tile (its K/V tiles are read for it alone either way)
             qlo = qo[a] + (pair - toff[a]) * 2 * kBM;
             const int rows = qo[a + 1] - qlo;
             qn0 = min(kBM, rows);
             qn1 = min(kBM, rows - kBM);
+            half = p.half_tails && qn1 <= 0 && qn0 <= kBM / 2;
             qrow[0] = (long long)x * p.N + qlo;
             qrow[1] = qrow[0] + kBM;
         }
@@ -313,9 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
     } else if (warp == 9) {
         // ================= MMA issuer
-        const uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0);
-        const uint32_t idS64 = tc::idesc_bf16_f32(kBM, 64, 0);   // half tile: at most 64 valid keys
-        const uint32_t idO = tc::idesc_bf16_f32(kBM, D, 1);
+        const int mrows = half ? kBM / 2 : kBM;
+        const uint32_t idS = tc::idesc_bf16_f32(mrows, kBN, 0);
+        const uint32_t idS64 = tc::idesc_bf16_f32(mrows, 64, 0);   // half key tile: at most 64 valid keys
+        const uint32_t idO = tc::idesc_bf16_f32(mrows, D, 1);
         // PV k-steps of key tile j (16 keys each): 4 for a half tile, else 8
         auto pv_steps = [&](int j) { return key_tile(p, MODE, klist, j).y <= 64 ? 4 : kBN / 16; };
         const int ntiles = two ? 2 : 1;
@@ -428,6 +438,201 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         __syncwarp();
         int never = 0;
         tc::mbar_wait(bar(kBarMma), 0, &never);
+    } else if (half) {
+        // ================= softmax of an M = 64 tile: warp q of warpgroup t reads lanes 32q .. 32q + 15
+        // with the 16-lane shapes; thread i holds rows 16q + i/4 (A) and 16q + i/4 + 8 (B) and, of
+        // every 8 key columns, the two at 2 (i % 4), so each thread forms half the exponentials of
+        // a 128-row tile's thread. In split mode warpgroup t takes key tiles j % 2 == t and
+        // warpgroup 0 merges; with a single key tile warpgroup 0 alone.
+        const int t = warp >> 2, wq = warp & 3, q4 = lane & 3;
+        const int rA = 16 * wq + (lane >> 2), rB = rA + 8;
+        const int qn = two ? (t == 0 ? qn0 : qn1) : qn0;     // two: head pairs, tile t = head x + t
+        const long long qrow_t = t ? qrow[1] : qrow[0];
+        float* sML = reinterpret_cast<float*>(sbase + kOffML);   // split mode: [0][row] max, [1][row] sum
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + (uint32_t)(t * 128) + lane_off;
+        const uint32_t tO = tmem + 256 + (uint32_t)(t * 128) + lane_off;
+        const float c_log2 = p.scale_log2;
+        const int kj0 = split ? t : 0, kjs = split ? 2 : 1;
+        const int nloc = split ? (ntk - t + 1) / 2 : ((t == 0 || two) ? ntk : 0);
+        int j = 0;
+        float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;   // l: this thread's partial sums
+        bool ok = true;
+        int lim_next = nloc > 0 ? key_tile(p, MODE, klist, kj0).y : 0;
+        for (; j < nloc; ++j) {
+            const int lim = lim_next;
+            if (j + 1 < nloc) lim_next = key_tile(p, MODE, klist, kj0 + (j + 1) * kjs).y;
+            const bool got_s = tc::mbar_wait(bar(kBarS + t), j & 1, abort_flag);
+            if (!__all_sync(kFull, got_s)) { ok = false; break; }
+            tc::fence_after_sync();
+            uint32_t v[2][32];
+            tc::tmem_ld_16x256b_x8(tS, v[0]);
+            if (lim > 64) tc::tmem_ld_16x256b_x8(tS + 64, v[1]);
+            tc::tmem_wait_ld();
+            tc::regs_after_wait(v[0]);
+            if (lim > 64) tc::regs_after_wait(v[1]);
+            float xA = -INFINITY, xB = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h == 1 && lim <= 64) break;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if (64 * h + 8 * jj + 2 * q4 + e >= lim) {
+                            v[h][4 * jj + e] = __float_as_uint(-INFINITY);
+                            v[h][4 * jj + 2 + e] = __float_as_uint(-INFINITY);
+                        }
+                        xA = fmaxf(xA, __uint_as_float(v[h][4 * jj + e]));
+                        xB = fmaxf(xB, __uint_as_float(v[h][4 * jj + 2 + e]));
+                    }
+            }
+            xA = fmaxf(xA, __shfl_xor_sync(kFull, xA, 1));
+            xA = fmaxf(xA, __shfl_xor_sync(kFull, xA, 2));
+            xB = fmaxf(xB, __shfl_xor_sync(kFull, xB, 1));
+            xB = fmaxf(xB, __shfl_xor_sync(kFull, xB, 2));
+            // lazy rescale: only when a row's maximum rises by more than 2^8
+            const bool grow = xA > (mA + kRescaleLog2) / c_log2 || xB > (mB + kRescaleLog2) / c_log2;
+            if (__any_sync(kFull, grow)) {
+                const float nA = fmaxf(mA, xA * c_log2), nB = fmaxf(mB, xB * c_log2);
+                const bool rsA = nA > mA + kRescaleLog2, rsB = nB > mB + kRescaleLog2;
+                if (j > 0 && __any_sync(kFull, rsA || rsB)) {
+                    // S_t(j) complete => PV_t(j-1) complete: O_t may be rescaled now
+                    const float fA = rsA ? exp2f(mA - nA) : 1.f, fB = rsB ? exp2f(mB - nB) : 1.f;
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) {
+                        uint32_t ov[32];
+                        tc::tmem_ld_16x256b_x8(tO + 64 * h, ov);
+                        tc::tmem_wait_ld();
+                        tc::regs_after_wait(ov);
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) {
+                            ov[4 * jj] = __float_as_uint(__uint_as_float(ov[4 * jj]) * fA);
+                            ov[4 * jj + 1] = __float_as_uint(__uint_as_float(ov[4 * jj + 1]) * fA);
+                            ov[4 * jj + 2] = __float_as_uint(__uint_as_float(ov[4 * jj + 2]) * fB);
+                            ov[4 * jj + 3] = __float_as_uint(__uint_as_float(ov[4 * jj + 3]) * fB);
+                        }
+                        tc::tmem_st_16x256b_x8(tO + 64 * h, ov);
+                    }
+                    if (rsA) lA *= fA;
+                    if (rsB) lB *= fB;
+                }
+                if (rsA) mA = nA;
+                if (rsB) mB = nB;
+            }
+            // P = 2^(s c - m) as bf16 pairs: the pair of columns 8jj + 2 q4 is packed column 4jj + q4
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h == 1 && lim <= 64) break;
+                uint32_t pk[16];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float p0 = ex2_sfu(fmaf(__uint_as_float(v[h][4 * jj]), c_log2, -mA));
+                    const float p1 = ex2_sfu(fmaf(__uint_as_float(v[h][4 * jj + 1]), c_log2, -mA));
+                    const float p2 = ex2_sfu(fmaf(__uint_as_float(v[h][4 * jj + 2]), c_log2, -mB));
+                    const float p3 = ex2_sfu(fmaf(__uint_as_float(v[h][4 * jj + 3]), c_log2, -mB));
+                    lA += p0 + p1;
+                    lB += p2 + p3;
+                    __nv_bfloat162 b0 = __floats2bfloat162_rn(p0, p1), b1 = __floats2bfloat162_rn(p2, p3);
+                    pk[2 * jj] = *reinterpret_cast<uint32_t*>(&b0);
+                    pk[2 * jj + 1] = *reinterpret_cast<uint32_t*>(&b1);
+                }
+                tc::tmem_st_16x128b_x8(tS + 32 * h, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(kBarP + t));
+        }
+        lA += __shfl_xor_sync(kFull, lA, 1);
+        lA += __shfl_xor_sync(kFull, lA, 2);
+        lB += __shfl_xor_sync(kFull, lB, 1);
+        lB += __shfl_xor_sync(kFull, lB, 2);
+        // epilogue: O / l written as bf16 pairs of the thread's columns, and lse
+        auto store_rows = [&](const uint32_t (&o0)[32], const uint32_t* o1, int h, float a0A, float a1A, float a0B,
+                              float a1B) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const int col = 64 * h + 8 * jj + 2 * q4;
+                float vA0 = __uint_as_float(o0[4 * jj]) * a0A, vA1 = __uint_as_float(o0[4 * jj + 1]) * a0A;
+                float vB0 = __uint_as_float(o0[4 * jj + 2]) * a0B, vB1 = __uint_as_float(o0[4 * jj + 3]) * a0B;
+                if (o1) {
+                    vA0 = fmaf(__uint_as_float(o1[4 * jj]), a1A, vA0);
+                    vA1 = fmaf(__uint_as_float(o1[4 * jj + 1]), a1A, vA1);
+                    vB0 = fmaf(__uint_as_float(o1[4 * jj + 2]), a1B, vB0);
+                    vB1 = fmaf(__uint_as_float(o1[4 * jj + 3]), a1B, vB1);
+                }
+                if (rA < qn) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(vA0, vA1);
+                    *reinterpret_cast<__nv_bfloat162*>(p.O + (qrow_t + rA) * D + col) = b2;
+                }
+                if (rB < qn) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(vB0, vB1);
+                    *reinterpret_cast<__nv_bfloat162*>(p.O + (qrow_t + rB) * D + col) = b2;
+                }
+            }
+        };
+        if (split) {
+            if (t == 1 && q4 == 0) {
+                sML[rA] = mA; sML[kBM + rA] = lA;
+                sML[rB] = mB; sML[kBM + rB] = lB;
+            }
+            tc::named_bar_sync(1, 2 * kBM);
+            if (t == 0) {
+                bool got = false;
+                if (ok) got = tc::mbar_wait(bar(kBarO), 0, abort_flag) && tc::mbar_wait(bar(kBarO + 1), 0, abort_flag);
+                if (__all_sync(kFull, got)) {
+                    tc::fence_after_sync();
+                    const float m1A = sML[rA], l1A = sML[kBM + rA], m1B = sML[rB], l1B = sML[kBM + rB];
+                    const float mmA = fmaxf(mA, m1A), mmB = fmaxf(mB, m1B);
+                    const float f0A = mmA == -INFINITY ? 0.f : exp2f(mA - mmA), f1A = mmA == -INFINITY ? 0.f : exp2f(m1A - mmA);
+                    const float f0B = mmB == -INFINITY ? 0.f : exp2f(mB - mmB), f1B = mmB == -INFINITY ? 0.f : exp2f(m1B - mmB);
+                    const float LA = lA * f0A + l1A * f1A, LB = lB * f0B + l1B * f1B;
+                    const float iA = LA > 0.f ? 1.f / LA : 0.f, iB = LB > 0.f ? 1.f / LB : 0.f;
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) {
+                        uint32_t o0[32], o1[32];
+                        tc::tmem_ld_16x256b_x8(tO + 64 * h, o0);
+                        tc::tmem_ld_16x256b_x8(tO + 128 + 64 * h, o1);
+                        tc::tmem_wait_ld();
+                        tc::regs_after_wait(o0);
+                        tc::regs_after_wait(o1);
+                        store_rows(o0, o1, h, f0A * iA, f1A * iA, f0B * iB, f1B * iB);
+                    }
+                    if (q4 == 0 && p.lse) {
+                        if (rA < qn) p.lse[qrow_t + rA] = (mmA + log2f(LA)) * kLn2;
+                        if (rB < qn) p.lse[qrow_t + rB] = (mmB + log2f(LB)) * kLn2;
+                    }
+                }
+            }
+        } else if (t == 0 || two) {
+            bool got_last = false;
+            if (ok && j > 0) got_last = tc::mbar_wait(bar(kBarO + t), 0, abort_flag);
+            if (j > 0 && __all_sync(kFull, got_last)) {
+                tc::fence_after_sync();
+                const float iA = lA > 0.f ? 1.f / lA : 0.f, iB = lB > 0.f ? 1.f / lB : 0.f;
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) {
+                    uint32_t o0[32];
+                    tc::tmem_ld_16x256b_x8(tO + 64 * h, o0);
+                    tc::tmem_wait_ld();
+                    tc::regs_after_wait(o0);
+                    store_rows(o0, nullptr, h, iA, 0.f, iB, 0.f);
+                }
+                if (q4 == 0 && p.lse) {
+                    if (rA < qn) p.lse[qrow_t + rA] = (mA + log2f(lA)) * kLn2;
+                    if (rB < qn) p.lse[qrow_t + rB] = (mB + log2f(lB)) * kLn2;
+                }
+            } else if (j == 0) {
+                uint32_t zr[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) zr[e] = 0u;
+                for (int h = 0; h < D / 64; ++h) store_rows(zr, nullptr, h, 0.f, 0.f, 0.f, 0.f);
+                if (q4 == 0 && p.lse) {
+                    if (rA < qn) p.lse[qrow_t + rA] = -INFINITY;
+                    if (rB < qn) p.lse[qrow_t + rB] = -INFINITY;
+                }
+            }
+        }
     } else {
         // ================= softmax warpgroup t: thread r <-> row r of tile t <-> TMEM lane r
         const int t = warp >> 2;
@@ -797,6 +1002,8 @@ int probe_tc_splits(int N, int ns) { return (N + probe_tc_chunk(N, ns) - 1) / pr
 
 bool attn_tc_head_pairs(int g) { return g % 2 == 0; }
 
+bool attn_tc_half_tails(int g) { return g >= 1; }
+
 int attn_tc_rows_per_cta(int g) { return attn_tc_head_pairs(g) ? kBM : 2 * kBM; }
 
 long long key_tiles_capacity(int N, int Gq, int Gk) { return (long long)Gq * ((N + kBN - 1) / kBN + Gk); }
@@ -823,6 +1030,7 @@ cudaError_t launch_attn_sparse_tc(const bf16* Qp, const bf16* Kp, const bf16* Vp
     p.qoff = qoff; p.tile_off = tile_off; p.klist = klist; p.klist_off = klist_off;
     p.Gq = Gq;
     p.head_pairs = attn_tc_head_pairs(g) ? 1 : 0;
+    p.half_tails = attn_tc_half_tails(g) ? 1 : 0;
     const int rows = attn_tc_rows_per_cta(g);
     dim3 grid((N + rows - 1) / rows + Gq, p.head_pairs ? B * Hq / 2 : B * Hq);
     return launch_tc_d<kModeSparse>(d, Qp, Kp, Vp, p, (long long)B * Hq * N, B, Hkv, grid, s);

@@ -135,8 +135,7 @@ cudaError_t launch_permute_rows(const bf16* src, bf16* dst, const int32_t* perm,
 
 // ---------------------------------------------------------------- attention
 // Per-pair tile offsets of the query groups: tile_off[z][a] = sum_{a'<a} ceil(|Q_a'| / bm).
-cudaError_t launch_tile_offsets(const int32_t* qoff, int32_t* tile_off, int P, int Gq, int bm,
-                                cudaStream_t s);
+cudaError_t launch_tile_offsets(const int32_t* qoff, int32_t* tile_off, int P, int Gq, int bm, cudaStream_t s);
 // Block-sparse attention over group-major Qp/Kp/Vp with the route CSR.
 cudaError_t launch_attn_sparse(const bf16* Qp, const bf16* Kp, const bf16* Vp,
                                const int32_t* qoff, const int32_t* koff, const int32_t* tile_off,
@@ -150,6 +149,9 @@ cudaError_t launch_attn_dense(const bf16* Q, const bf16* K, const bf16* V, bf16*
 bool attn_tc_supported(int d);
 // Query rows one CTA covers: two 128-row tiles of one head, or (g even) one tile of two heads.
 bool attn_tc_head_pairs(int g);
+// A lone last query tile of at most 64 rows (or, with head pairs, such a tile of two heads) runs
+// as an M = 64 tile: half the softmax work per key tile, the same K/V reads.
+bool attn_tc_half_tails(int g);
 int attn_tc_rows_per_cta(int g);
 // Key tiles (start row, valid keys) of every query group's merged kept runs: cnt [P][Gq]
 // scratch, off [P][Gq+1] absolute offsets, list of key_tiles_capacity(N, Gq, Gk) * P entries.
