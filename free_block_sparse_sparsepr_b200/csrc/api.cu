@@ -173,8 +173,11 @@ long long budget_pairs(const sparsepr_config& c, int M) {
 // G <= 256 the assignment runs on tensor cores (bf16 split operands, near ties settled in fp64)
 // and the radial distances come from one exact pass after the last assignment.
 // rows_split: the caller already wrote the rows' bf16 parts and squared norms (kmX2, kmxx).
+// need_dist: the rows' distances to their centroids are used (the query partition's radial
+// key); the key partition's are not, so its exact distance pass is skipped.
 sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t* labels, float* dist,
-                       int32_t* perm, int32_t* off, cudaStream_t s, bool rows_split = false) {
+                       int32_t* perm, int32_t* off, cudaStream_t s, bool rows_split = false,
+                       bool need_dist = true) {
     const int P = h->P, n = h->cfg.N;
     const bool tc = spr::km_tc_supported(G) && DP <= 64;
     auto assign = [&](bool first, const int* done) -> cudaError_t {
@@ -196,7 +199,7 @@ sparsepr_status kmeans(sparsepr_handle h, const float* X, int DP, int G, int32_t
         SPR_TRY(assign(false, h->km_done));
         SPR_TRY(spr::launch_km_check(h->km_changed, h->km_done, P, s));
     }
-    if (tc) SPR_TRY(spr::launch_km_dist(X, h->kmC, labels, dist, P, n, G, DP, s));
+    if (tc && need_dist) SPR_TRY(spr::launch_km_dist(X, h->kmC, labels, dist, P, n, G, DP, s));
     SPR_TRY(spr::launch_group_sort(labels, perm, off, h->counts, h->bases, nullptr, P, n, G, s));
     h->launches += 2;
     return SPARSEPR_OK;
@@ -233,7 +236,7 @@ sparsepr_status partition_semantic(sparsepr_handle h, const bf16* Q, const bf16*
     const sparsepr_config& c = h->cfg;
     const int P = h->P, N = c.N, d = c.d;
     SPR_TRY(spr::launch_mean_heads_f32(K, h->features, P, 1, N, d, s));
-    sparsepr_status st = kmeans(h, h->features, d, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s);
+    sparsepr_status st = kmeans(h, h->features, d, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s, false, false);
     if (st) return st;
     SPR_TRY(spr::launch_group_mean_bf16(K, h->kperm, h->koff, h->kcent, h->chi, h->clo, P, N, c.Gk, d, s));
     st = query_logits(h, Q, h->chi, h->clo, h->koff, s);
@@ -272,7 +275,7 @@ sparsepr_status partition_impl(sparsepr_handle h, const bf16* Q, const bf16* K, 
     // (2a) key groups and their means in the original key space
     const bool key_rows_split = resp_tc && spr::km_tc_supported(c.Gk);
     sparsepr_status st = kmeans(h, h->features, h->DPk, c.Gk, h->kgroup, h->kdist, h->kperm, h->koff, s,
-                                key_rows_split);
+                                key_rows_split, false);
     if (st) return st;
     SPR_TRY(spr::launch_group_mean_bf16(K, h->kperm, h->koff, h->kcent, h->chi, h->clo, P, N, c.Gk, d, s));
     // (2b) query coordinates and query groups

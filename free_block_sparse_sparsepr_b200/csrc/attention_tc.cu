@@ -19,7 +19,9 @@
 // Key tiles are cut from merged runs of consecutive kept key groups; keys past a run's end
 // (the next group's, or zero fill past the tensor) are masked to -inf. A tile with at most 64
 // valid keys is a half tile: its S and PV MMAs run with 64 keys and the softmax neither loads
-// nor writes the other half.
+// nor writes the other half. A query tile of at most 64 rows (a group's last) runs its MMAs
+// with M = 64; its warpgroup then reads S and writes P with the 16-lane TMEM shapes, two rows
+// per thread.
 #include <cuda.h>
 #include <float.h>
 #include <math.h>
@@ -68,7 +70,7 @@ struct TcParams {
     int* status;
     int N, g, Gq;
     int head_pairs;               // sparse mode, g even: one CTA = the same query tile of two query heads
-    int half_tails;               // sparse mode: a lone last tile of <= 64 rows (or, head pairs, of two heads) is M = 64
+    int half_tails;               // sparse mode: a last query tile of <= 64 rows (of one head, or of both in a head pair) is M = 64
     int stall;                    // test only: issue no loads (the first bounded wait runs out)
     // probe mode: M gathered rows per query head against key split blockIdx.x (chunk keys each);
     // unnormalised partial outputs [x][ns][M][d], running maxima (log2 units) and sums [x][ns][M]
@@ -198,7 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
     // ---- which query tiles
     int qlo, qn0, qn1, a = 0, ntk = 0;
-    bool half = false;   // an M = 64 tile (rows in lanes 0-15 of each 32-lane quarter, 16-lane TMEM shapes)
+    // half0 / half1: query tile 0 / 1 is an M = 64 tile (rows in lanes 0-15 of each 32-lane
+    // quarter, read and written with the 16-lane TMEM shapes)
+    bool half0 = false, half1 = false;
     long long qrow[2];
     const int2* klist = nullptr;
     if (MODE == kModeSparse) {
@@ -216,17 +220,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int c = pair - toff[a];
             qlo = qo[a] + c * kBM;
             qn0 = qn1 = min(kBM, qo[a + 1] - qlo);
-            half = p.half_tails && qn0 <= kBM / 2;
+            half0 = half1 = p.half_tails && qn0 <= kBM / 2;
             qrow[0] = (long long)x * p.N + qlo;
             qrow[1] = (long long)(x + 1) * p.N + qlo;
         } else {
-            // the group's rows in pairs of 128-row tiles; with half tails, a lone last tile of at
-            // most 64 rows runs as an M = 64 tile (its K/V tiles are read for it alone either way)
+            // the group's rows in pairs of 128-row tiles; with half tails, a last tile of at most
+            // 64 rows (lone, or the second of its pair) runs as an M = 64 tile
             qlo = qo[a] + (pair - toff[a]) * 2 * kBM;
             const int rows = qo[a + 1] - qlo;
             qn0 = min(kBM, rows);
             qn1 = min(kBM, rows - kBM);
-            half = p.half_tails && qn1 <= 0 && qn0 <= kBM / 2;
+            half0 = p.half_tails && qn1 <= 0 && qn0 <= kBM / 2;
+            half1 = p.half_tails && qn1 > 0 && qn1 <= kBM / 2;
             qrow[0] = (long long)x * p.N + qlo;
             qrow[1] = qrow[0] + kBM;
         }
@@ -253,6 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // the same rows, warpgroup t the key tiles j with j % 2 == t, and warpgroup 0 merges the two
     // partial softmax states at the end, so the tensor core still alternates between two S tiles.
     const bool split = !two && ntk >= 2;
+    // the M of the S and PV MMAs into S_t / O_t, and the softmax path of warpgroup t
+    auto half_of = [&](int t) { return split ? half0 : (t ? half1 : half0); };
 
     // ---- set-up: barriers (thread 0), TMEM (warp 9)
     if (threadIdx.x == 0) {
@@ -322,10 +329,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
     } else if (warp == 9) {
         // ================= MMA issuer
-        const int mrows = half ? kBM / 2 : kBM;
-        const uint32_t idS = tc::idesc_bf16_f32(mrows, kBN, 0);
-        const uint32_t idS64 = tc::idesc_bf16_f32(mrows, 64, 0);   // half key tile: at most 64 valid keys
-        const uint32_t idO = tc::idesc_bf16_f32(mrows, D, 1);
+        // instruction descriptors of S_t (full and half key tile) and O_t by the M of tile t
+        auto idS = [&](int t, bool half_keys) {
+            return tc::idesc_bf16_f32(half_of(t) ? kBM / 2 : kBM, half_keys ? 64 : kBN, 0);
+        };
+        auto idO = [&](int t) { return tc::idesc_bf16_f32(half_of(t) ? kBM / 2 : kBM, D, 1); };
         // PV k-steps of key tile j (16 keys each): 4 for a half tile, else 8
         auto pv_steps = [&](int j) { return key_tile(p, MODE, klist, j).y <= 64 ? 4 : kBN / 16; };
         const int ntiles = two ? 2 : 1;
@@ -334,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         auto issue_S = [&](int t, int j) {
             const uint32_t kb = sK + (j % kStages) * 2 * kRegion;
             const uint32_t qb = sQ + (split ? 0 : t) * 2 * kRegion;
-            const uint32_t id = key_tile(p, MODE, klist, j).y <= 64 ? idS64 : idS;
+            const uint32_t id = idS(t, key_tile(p, MODE, klist, j).y <= 64);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint32_t off = (uint32_t)((k >> 2) * kRegion + (k & 3) * 32);
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     for (int k = 0; k < kBN / 16; ++k)
                         if (k < nk)
                             tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
-                                           tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
+                                           tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO(t),
                                            (j >= 2 || k > 0) ? 1u : 0u);
                     tc::commit(bar(kBarEV + s));
                     if (nh) {
@@ -416,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     for (int k = 0; k < kBN / 16; ++k)
                         if (k < nk)
                             tc::mma_f16_ts(tmem + 256 + (uint32_t)(t * 128), pt + (uint32_t)(8 * k),
-                                           tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO,
+                                           tc::smem_desc_sw128(vb + (uint32_t)(k * 2048), kRegion, 1024), idO(t),
                                            (j > 0 || k > 0) ? 1u : 0u);
                     const bool last = t + 1 == ntiles;
                     if (last) tc::commit(bar(kBarEV + s));                  // V(j) read by every PV
@@ -438,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         __syncwarp();
         int never = 0;
         tc::mbar_wait(bar(kBarMma), 0, &never);
-    } else if (half) {
+    } else if (half_of(warp >> 2)) {
         // ================= softmax of an M = 64 tile: warp q of warpgroup t reads lanes 32q .. 32q + 15
         // with the 16-lane shapes; thread i holds rows 16q + i/4 (A) and 16q + i/4 + 8 (B) and, of
         // every 8 key columns, the two at 2 (i % 4), so each thread forms half the exponentials of

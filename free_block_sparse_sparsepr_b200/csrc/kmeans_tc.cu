@@ -4,11 +4,13 @@
 // For a tile of 128 rows the dot products with every centroid form one 128 x G x D GEMM.
 // Rows and centroids are split into two bf16 parts (x = x0 + x1 + e, |e| <= 2^-16 |x|
 // elementwise) and the three terms x0 c0 + x0 c1 + x1 c0 are accumulated in fp32 TMEM, so
-// each dot product is known to within about 2^-14 ||x|| ||c||. One epilogue thread per row
-// reads dd_g = ||c_g||^2 - 2 x.c_g straight from its TMEM lane in two passes: the first keeps
-// only the smallest dd of every 32-column chunk (three-input minima, about half an ALU
-// instruction per distance), the second reloads the winning chunk to find its argmin (lowest
-// column on ties) and to count its distances within the certificate's gap of the minimum.
+// each dot product is known to within about 2^-14 ||x|| ||c||. One more K = 16 step multiplies
+// a constant tile of ones (columns 0-2) by the three bf16 parts of -||c_g||^2 / 2, so the
+// accumulator holds v_g = x.c_g - ||c_g||^2 / 2 = (||x||^2 - dd_g) / 2 and the nearest centroid
+// is the largest v. One epilogue thread per row reads v straight from its TMEM lane, 32
+// columns at a time, keeps the largest v of every chunk (three-input maxima) and a register
+// copy of the chunk holding the largest so far, from which come the argmax (lowest column on
+// ties) and the count of values within the certificate's gap (half the gap in dd) of it.
 // When no other distance (in that chunk, or as another chunk's minimum) lies within a bound on
 // the estimate's error, the estimate decides; otherwise (about 1% of rows) the row goes to a
 // list that the same CTA settles exactly at its end: an fp32 pass over all centroids keeps
@@ -43,7 +45,9 @@ constexpr uint32_t kTmemCols = 512;
 
 constexpr int kOffC = 0;                                     // part q at kOffC + q * kMaxG * 128
 constexpr int kOffX = kOffC + kParts * kMaxG * 128;          // stage s, part q at + (s * kParts + q) * kTile
-constexpr int kOffCC = kOffX + kStages * kParts * kTile;     // kMaxG floats
+constexpr int kOffOnes = kOffX + kStages * kParts * kTile;   // [128][64] bf16, ones in columns 0-2
+constexpr int kOffCCt = kOffOnes + kTile;                     // [kMaxG][64] bf16, -||c||^2/2 in three parts
+constexpr int kOffCC = kOffCCt + kMaxG * 128;                 // kMaxG floats
 constexpr int kOffBar = kOffCC + kMaxG * 4;
 constexpr int kBarC = 0, kBarXF = 1, kBarXE = kBarXF + kStages, kBarDF = kBarXE + kStages, kBarDE = kBarDF + 2,
               kBarMma = kBarDE + 2, kNumBars = kBarMma + 1;
@@ -51,13 +55,14 @@ constexpr int kOffMisc = kOffBar + 8 * kNumBars;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// Gap below which a row is recomputed exactly: 4 kKappa ||x|| max_g ||c_g|| covers twice the
-// error of two dot-product estimates (each at most ~3.1 * 2^-16 ||x|| ||c|| from the dropped
-// split terms plus fp32 accumulation); kSlack (||x||^2 + max ||c||^2) covers the fp32
-// rounding of ||c||^2 and of dd, and the low bits that the keys below give up to the column index.
+// Gap in dd below which a row is recomputed exactly: 4 kKappa ||x|| max_g ||c_g|| covers twice
+// the error of two dot-product estimates (each at most ~3.1 * 2^-16 ||x|| ||c|| from the
+// dropped split terms plus fp32 accumulation); kSlack (||x||^2 + max ||c||^2) covers the fp32
+// rounding of ||c||^2, its three-part bf16 split (about 2^-24 ||c||^2) and the fp32
+// accumulation of v, with a wide margin.
 constexpr float kKappa = 1.0f / 8192.0f;   // 2^-13
-constexpr float kSlack = 1.0f / 32768.0f;  // 2^-15 (also covers the 5 index bits packed into keys)
-// ||c||^2 of padding columns: finite (so packed keys never form a NaN) and far above any distance.
+constexpr float kSlack = 1.0f / 32768.0f;  // 2^-15
+// ||c||^2 of padding columns: finite (so its bf16 parts never form a NaN) and far above any distance.
 constexpr float kFar = 1.0e37f;
 
 struct KmParams {
@@ -78,10 +83,10 @@ struct KmMaps {
     CUtensorMap c[kParts];   // centroid parts [P*G16][64] bf16
 };
 
-// Three-input fp32 minimum.
-__device__ __forceinline__ float fmin3(float a, float b, float c) {
+// Three-input fp32 maximum.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
 
@@ -113,6 +118,35 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
     const int tiles = (p.n + kRows - 1) / kRows;
 
     for (int t = threadIdx.x; t < kMaxG; t += kThreads) sCC[t] = t < p.G32 ? p.cc[(long long)z * p.G32 + t] : kFar;
+    // The two constant operands of the extra K step, written in the 128-byte swizzled layout
+    // (16-byte chunk k of row r at chunk k ^ (r % 8)): row r of the ones tile holds 1, 1, 1 in
+    // columns 0-2, row g of the other the bf16 parts of -||c_g||^2 / 2; every other element is 0.
+    {
+        uint4* ones = reinterpret_cast<uint4*>(sbase + kOffOnes);
+        uint4* cct = reinterpret_cast<uint4*>(sbase + kOffCCt);
+        const uint32_t one = 0x3F80u;   // bf16 1.0
+        for (int q = threadIdx.x; q < kRows * 8 + p.G16 * 8; q += kThreads) {
+            const bool isc = q >= kRows * 8;
+            const int row = (isc ? q - kRows * 8 : q) >> 3, k = (q & 7) ^ (row & 7);
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (k == 0) {
+                if (!isc) {
+                    v.x = one | (one << 16);
+                    v.y = one;
+                } else {
+                    const float a = -0.5f * p.cc[(long long)z * p.G32 + row];
+                    const bf16 h0 = __float2bfloat16_rn(a);
+                    const float r1 = a - __bfloat162float(h0);
+                    const bf16 h1 = __float2bfloat16_rn(r1);
+                    const bf16 h2 = __float2bfloat16_rn(r1 - __bfloat162float(h1));
+                    v.x = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                    v.y = (uint32_t)__bfloat16_as_ushort(h2);
+                }
+            }
+            (isc ? cct : ones)[isc ? q - kRows * 8 : q] = v;
+        }
+        tc::fence_proxy_async_smem();
+    }
     if (threadIdx.x == 0) {
         *sFix = 0;
         tc::mbar_init(bar(kBarC), 1);
@@ -178,6 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                     tc::mma_f16_ss(d, x0, c1, idesc, 1u);
                     tc::mma_f16_ss(d, x1, c0, idesc, 1u);
                 }
+                tc::mma_f16_ss(d, tc::smem_desc_sw128(base + kOffOnes, 16, 1024),
+                               tc::smem_desc_sw128(base + kOffCCt, 16, 1024), idesc, 1u);
                 tc::commit(bar(kBarXE + s));
                 tc::commit(bar(kBarDF + b));
             }
@@ -190,11 +226,11 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
     } else {
         const int wg = warp >> 2, wr = (warp & 3) * 32;
         const uint32_t tb = tmem + (uint32_t)(wg * 256) + ((uint32_t)wr << 16);
-        // Columns [G16, G32) are never written by the MMA: make them read as zero (dd = +inf).
+        // Columns [G16, G32) are never written by the MMA: make them read as -kFar (never the largest).
         if (p.G16 < p.G32) {
             uint32_t zr[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) zr[e] = 0u;
+            for (int e = 0; e < 16; ++e) zr[e] = __float_as_uint(-kFar);
             tc::tmem_st16(tb + (uint32_t)p.G16, zr);
             tc::tmem_wait_st();
         }
@@ -210,40 +246,30 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
             const int prev = (valid && !p.first) ? p.labels[o] : -1;
             if (!__all_sync(kFull, tc::mbar_wait(bar(kBarDF + wg), (i >> 1) & 1, abort_flag))) break;
             tc::fence_after_sync();
-            // One pass over the row's distances, 32 columns (one TMEM load) at a time: dd of the
-            // chunk, its minimum by three-input minima, and, when that minimum is a new best (B1),
-            // the chunk's 32 values copied into `best` by predicated selects; B2c is the smallest
-            // of the other chunks' minima. The near-tie count and the argmin (lowest column on
-            // ties) then come from `best` in registers, with no second read of TMEM.
-            float B1 = INFINITY, B2c = INFINITY;
+            // One pass over the row's values, 32 columns (one TMEM load) at a time: the chunk's
+            // largest v by three-input maxima and, when it is a new best (B1), the chunk's 32
+            // values copied into `best` by predicated selects; B2c is the largest of the other
+            // chunks' maxima. The near-tie count and the argmax (lowest column on ties) then come
+            // from `best` in registers, with no second read of TMEM.
+            float B1 = -INFINITY, B2c = -INFINITY;
             int cb = 0;
             float best[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) best[e] = INFINITY;
-            auto chunk = [&](uint32_t* v, int c) {
-                // dd overwrites the loaded dot products in place
-                const float4* cc4 = reinterpret_cast<const float4*>(sCC + c);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 ce = cc4[q];
-                    v[4 * q] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q]), ce.x));
-                    v[4 * q + 1] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q + 1]), ce.y));
-                    v[4 * q + 2] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q + 2]), ce.z));
-                    v[4 * q + 3] = __float_as_uint(fmaf(-2.f, __uint_as_float(v[4 * q + 3]), ce.w));
-                }
-                auto dd = [&](int e) { return __uint_as_float(v[e]); };
+            for (int e = 0; e < 32; ++e) best[e] = -INFINITY;
+            auto chunk = [&](const uint32_t* v, int c) {
+                auto vv = [&](int e) { return __uint_as_float(v[e]); };
                 float mm[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    mm[j] = fmin3(fmin3(dd(j), dd(j + 4), dd(j + 8)), fmin3(dd(j + 12), dd(j + 16), dd(j + 20)),
-                                  fminf(dd(j + 24), dd(j + 28)));
-                const float mc = fminf(fmin3(mm[0], mm[1], mm[2]), mm[3]);
-                const bool nb = mc < B1;
-                B2c = nb ? B1 : fminf(B2c, mc);
+                    mm[j] = fmax3(fmax3(vv(j), vv(j + 4), vv(j + 8)), fmax3(vv(j + 12), vv(j + 16), vv(j + 20)),
+                                  fmaxf(vv(j + 24), vv(j + 28)));
+                const float mc = fmaxf(fmax3(mm[0], mm[1], mm[2]), mm[3]);
+                const bool nb = mc > B1;
+                B2c = nb ? B1 : fmaxf(B2c, mc);
                 B1 = nb ? mc : B1;
                 cb = nb ? c : cb;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) best[e] = nb ? dd(e) : best[e];
+                for (int e = 0; e < 32; ++e) best[e] = nb ? vv(e) : best[e];
             };
             {
                 uint32_t va[32], vb[32];
@@ -266,20 +292,21 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                     }
                 }
             }
-            const float T = 4.f * kKappa * sqrtf(xxr) * cmax + kSlack * (xxr + cmax2);
-            const float thr = B1 + T;
+            // T bounds the error of a difference of two dd estimates; differences of v are half those of dd
+            const float Th = 0.5f * (4.f * kKappa * sqrtf(xxr) * cmax + kSlack * (xxr + cmax2));
+            const float thr = B1 - Th;
             int idx = 31;
             float near = 0.f;
 #pragma unroll
             for (int e = 31; e >= 0; --e) {
                 idx = best[e] == B1 ? e : idx;
-                near += best[e] <= thr ? 1.f : 0.f;
+                near += best[e] >= thr ? 1.f : 0.f;
             }
             const int I1 = min(cb + idx, p.G - 1);
             tc::fence_before_sync();
             tc::mbar_arrive(bar(kBarDE + wg));
 
-            const bool flag = valid && !(B2c - B1 > T && near < 1.5f);
+            const bool flag = valid && !(B1 - B2c > Th && near < 1.5f);
             // Hand each flagged row to the exact settlement at the end of the kernel.
             const unsigned fl = __ballot_sync(kFull, flag);
             if (fl) {
