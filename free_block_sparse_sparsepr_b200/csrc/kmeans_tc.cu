@@ -74,7 +74,7 @@ struct KmParams {
     int* changed;          // [P]
     const int* done;       // [P] or null
     int* status;
-    int4* fix;             // flagged rows {row, previous label, estimate, 0}; fix_cap slots per CTA
+    int4* fix;             // flagged rows {row, previous label, estimate, chunk mask}; fix_cap slots per CTA
     int n, G, G16, G32, DP, ksteps, first, fix_cap;
 };
 
@@ -253,10 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
             // from `best` in registers, with no second read of TMEM.
             float B1 = -INFINITY, B2c = -INFINITY;
             int cb = 0;
-            float best[32];
+            float best[32], cm[kMaxG / 32];   // cm: every chunk's largest v
 #pragma unroll
             for (int e = 0; e < 32; ++e) best[e] = -INFINITY;
-            auto chunk = [&](const uint32_t* v, int c) {
+#pragma unroll
+            for (int e = 0; e < kMaxG / 32; ++e) cm[e] = -INFINITY;
+            auto chunk = [&](const uint32_t* v, int c, float& cmax_c) {
                 auto vv = [&](int e) { return __uint_as_float(v[e]); };
                 float mm[4];
 #pragma unroll
@@ -264,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                     mm[j] = fmax3(fmax3(vv(j), vv(j + 4), vv(j + 8)), fmax3(vv(j + 12), vv(j + 16), vv(j + 20)),
                                   fmaxf(vv(j + 24), vv(j + 28)));
                 const float mc = fmaxf(fmax3(mm[0], mm[1], mm[2]), mm[3]);
+                cmax_c = mc;
                 const bool nb = mc > B1;
                 B2c = nb ? B1 : fmaxf(B2c, mc);
                 B1 = nb ? mc : B1;
@@ -276,18 +279,22 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                 tc::tmem_ld32(tb, va);
                 tc::tmem_wait_ld();
                 tc::regs_after_wait(va);
-                for (int c = 0; c < p.G32; c += 64) {
-                    const bool hb = c + 32 < p.G32, ha = c + 64 < p.G32;
-                    if (hb) tc::tmem_ld32(tb + (uint32_t)(c + 32), vb);
-                    chunk(va, c);
-                    if (hb) {
-                        tc::tmem_wait_ld();
-                        tc::regs_after_wait(vb);
-                        if (ha) tc::tmem_ld32(tb + (uint32_t)(c + 64), va);
-                        chunk(vb, c + 32);
-                        if (ha) {
+#pragma unroll
+                for (int q = 0; q < kMaxG / 64; ++q) {
+                    const int c = 64 * q;
+                    if (c < p.G32) {
+                        const bool hb = c + 32 < p.G32, ha = c + 64 < p.G32;
+                        if (hb) tc::tmem_ld32(tb + (uint32_t)(c + 32), vb);
+                        chunk(va, c, cm[2 * q]);
+                        if (hb) {
                             tc::tmem_wait_ld();
-                            tc::regs_after_wait(va);
+                            tc::regs_after_wait(vb);
+                            if (ha) tc::tmem_ld32(tb + (uint32_t)(c + 64), va);
+                            chunk(vb, c + 32, cm[2 * q + 1]);
+                            if (ha) {
+                                tc::tmem_wait_ld();
+                                tc::regs_after_wait(va);
+                            }
                         }
                     }
                 }
@@ -303,6 +310,11 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                 near += best[e] >= thr ? 1.f : 0.f;
             }
             const int I1 = min(cb + idx, p.G - 1);
+            // Chunks that can hold the nearest centroid: a chunk whose largest v is more than the
+            // gap below B1 holds only centroids certified farther than the estimated best.
+            unsigned cmask = 0u;
+#pragma unroll
+            for (int e = 0; e < kMaxG / 32; ++e) cmask |= (cm[e] >= thr ? 1u : 0u) << e;
             tc::fence_before_sync();
             tc::mbar_arrive(bar(kBarDE + wg));
 
@@ -313,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
                 int slot = 0;
                 if (lane == 0) slot = atomicAdd(sFix, __popc(fl));
                 slot = __shfl_sync(kFull, slot, 0) + __popc(fl & ((1u << lane) - 1u));
-                if (flag) fix[slot] = make_int4((int)o, prev, I1, 0);
+                if (flag) fix[slot] = make_int4((int)o, prev, I1, (int)cmask);
             }
             int moved = 0;
             if (valid) {
@@ -348,9 +360,11 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
     }
 }
 
-// Exact label of one flagged row {row, previous label, estimate, 0}, settled by one warp (centroids
-// k-major in sCk with row stride G + 1, so staging and lane-parallel reads avoid bank conflicts; lane
-// g + 32j takes centroid g + 32j): candidates are the groups whose fp32 ||x||^2 - 2 x.c + ||c||^2
+// Exact label of one flagged row {row, previous label, estimate, chunk mask}, settled by one warp
+// (centroids k-major in sCk with row stride G + 1, so staging and lane-parallel reads avoid bank
+// conflicts; lane g + 32j takes centroid g + 32j). Only the 32-centroid chunks in the mask are
+// screened: every centroid of another chunk is certified farther than the estimated best, so it
+// can neither be the nearest nor tie with it. Candidates are the groups whose fp32 ||x||^2 - 2 x.c + ||c||^2
 // (error below 2^-19 (||x||^2 + ||c||^2)) is within 1e-4 (|d_min| + ||x||^2 + max ||c||^2) of the
 // smallest; each gets the fp32 value of its fp64 distance (butterfly sums, identical in every
 // lane), argmin with ties to the lowest group. Corrects the label and the count of rows that
@@ -376,19 +390,19 @@ __device__ __forceinline__ void settle_row(const int4 h, const float* __restrict
 #pragma unroll
     for (int j = 0; j < kMaxG / 32; ++j) dj[j] = INFINITY;
     float dmin = INFINITY;
-    // not unrolled: each chunk of 32 centroids re-broadcasts the row (keeps registers low)
+    // the row in every lane's registers, broadcast once
+    float xv[DP];
+#pragma unroll
+    for (int k = 0; k < DP; ++k) xv[k] = __shfl_sync(kFull, k < 32 ? xa : xb, k & 31);
 #pragma unroll 1
     for (int j = 0; j < kMaxG / 32; ++j) {
-        if (j < nj) {
+        if (j < nj && ((h.w >> j) & 1)) {
             const int g = 32 * j + lane;
             const int gc = g < G ? g : G - 1;
-            float a0 = 0.f, a1 = 0.f;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < DP; k += 2) {
-                a0 = fmaf(__shfl_sync(kFull, k < 32 ? xa : xb, k & 31), sCk[k * (G + 1) + gc], a0);
-                a1 = fmaf(__shfl_sync(kFull, k + 1 < 32 ? xa : xb, (k + 1) & 31), sCk[(k + 1) * (G + 1) + gc], a1);
-            }
-            const float dg = g < G ? fmaf(-2.f, a0 + a1, xx + sCC[g]) : INFINITY;
+            for (int k = 0; k < DP; ++k) a[k & 3] = fmaf(xv[k], sCk[k * (G + 1) + gc], a[k & 3]);
+            const float dg = g < G ? fmaf(-2.f, (a[0] + a[1]) + (a[2] + a[3]), xx + sCC[g]) : INFINITY;
 #pragma unroll
             for (int jj = 0; jj < kMaxG / 32; ++jj) dj[jj] = jj == j ? dg : dj[jj];
             dmin = fminf(dmin, dg);
