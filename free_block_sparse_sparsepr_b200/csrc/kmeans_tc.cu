@@ -235,7 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
             tc::tmem_wait_st();
         }
         float cmax2 = 0.f;
-        for (int g = 0; g < p.G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
+        for (int g = lane; g < p.G; g += 32) cmax2 = fmaxf(cmax2, sCC[g]);
+        cmax2 = warp_max(cmax2);   // the same value in every lane
         const float cmax = sqrtf(cmax2);
         for (int i = wg, t = blockIdx.x + wg * gridDim.x; t < tiles; i += 2, t += 2 * gridDim.x) {
             // The row's ||x||^2 and previous label are fetched before waiting for the tile.
@@ -354,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) km_assign_tc_kernel(const __grid_
         for (int t = threadIdx.x; t < p.G * DP; t += kThreads) sCk[(t % DP) * (p.G + 1) + t / DP] = __ldg(src + t);
         __syncthreads();
         float cmax2 = 0.f;
-        for (int g = 0; g < p.G; ++g) cmax2 = fmaxf(cmax2, sCC[g]);
+        for (int g = lane; g < p.G; g += 32) cmax2 = fmaxf(cmax2, sCC[g]);
+        cmax2 = warp_max(cmax2);   // the same value in every lane
         for (int w = warp; w < nfix; w += kThreads / 32)
             settle_row<DP>(fix[w], p.X, sCk, sCC, cmax2, p.G, p.labels, p.changed, z, lane);
     }
