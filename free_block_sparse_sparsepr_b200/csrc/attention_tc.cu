@@ -9,7 +9,7 @@
 //              forms 2^(s c - m) against the running max, writes P_t as bf16 pairs into the first 64 columns of S_t's
 //              own TMEM buffer, rescales its O_t row when the max grows by more than 2^8, and
 //              finally normalises and stores O_t;
-//   warp 8     TMA producer: both Q tiles once, then K and V tiles into a 2-stage ring;
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles into rings of 2 and 3 stages;
 //   warp 9     TMEM allocation and the MMA issue (one thread): S_t = Q_t K^T (A and B from
 //              shared memory), O_t += P_t V (A from TMEM), completions via tcgen05.commit.
 // The tensor core alternates between the tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)), so one
@@ -37,7 +37,8 @@ namespace {
 
 constexpr int kBM = 128;            // rows per query tile (two tiles per CTA)
 constexpr int kBN = 128;            // keys per tile
-constexpr int kStages = 2;          // K/V ring depth
+constexpr int kKStages = 2;         // K ring depth
+constexpr int kVStages = 3;         // V ring depth (a V tile is freed a step later than a K tile)
 constexpr int kRegion = 16384;      // one [128 rows][64 bf16] 128B-swizzled region
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512; // S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512)
@@ -46,17 +47,19 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr int kOffQ = 0;                                   // tile t at + t * 2 * kRegion
 constexpr int kOffK = kOffQ + 2 * 2 * kRegion;
-constexpr int kOffV = kOffK + kStages * 2 * kRegion;
-constexpr int kOffBar = kOffV + kStages * 2 * kRegion;
-// barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_last[2],
-// mma_done. K and V stages are released separately: a K tile as soon as the last S MMA that
-// reads it completes, a V tile after the last PV MMA, so the next K load starts a step early.
-constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kStages, kBarEK = kBarV + kStages, kBarEV = kBarEK + kStages,
-              kBarS = kBarEV + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2,
+constexpr int kOffV = kOffK + kKStages * 2 * kRegion;
+constexpr int kOffBar = kOffV + kVStages * 2 * kRegion;
+// barriers: q_full, k_full[KS], v_full[VS], k_empty[KS], v_empty[VS], s_full[2], p_full[2],
+// o_last[2], mma_done. K and V stages are released separately: a K tile as soon as the last S MMA
+// that reads it completes, a V tile after the last PV MMA. V(j) is read a step after K(j), so its
+// ring is one stage deeper: the load of V(j + 3) has two steps to land instead of one.
+constexpr int kBarQ = 0, kBarK = 1, kBarV = kBarK + kKStages, kBarEK = kBarV + kVStages, kBarEV = kBarEK + kKStages,
+              kBarS = kBarEV + kVStages, kBarP = kBarS + 2, kBarO = kBarP + 2, kBarMma = kBarO + 2,
               kNumBars = kBarMma + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;          // tmem base (u32), abort flag (int)
 constexpr int kOffML = kOffMisc + 16;                      // split mode: tile 1's running max and sum [2][128]
 constexpr int kSmemBytes = kOffML + 2 * kBM * 4 + 1024;   // + slack to align the base to 1024
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum { kModeSparse = 0, kModeDense = 1, kModeProbe = 2 };
 
@@ -264,10 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ---- set-up: barriers (thread 0), TMEM (warp 9)
     if (threadIdx.x == 0) {
         tc::mbar_init(bar(kBarQ), 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             tc::mbar_init(bar(kBarK + s), 1);
-            tc::mbar_init(bar(kBarV + s), 1);
             tc::mbar_init(bar(kBarEK + s), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            tc::mbar_init(bar(kBarV + s), 1);
             tc::mbar_init(bar(kBarEV + s), 1);
         }
         for (int t = 0; t < 2; ++t) {
@@ -299,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tc::tma_load_2d(sQ + (2 + h) * kRegion, &tmQ, bar(kBarQ), 64 * h, (int)qrow[1]);
             // K runs one tile ahead of V: K(0), then K(j+1) before V(j).
             auto load = [&](int m, bool isv) -> bool {
-                const int s = m % kStages;
-                if (m >= kStages && !tc::mbar_wait(bar((isv ? kBarEV : kBarEK) + s), ((m / kStages) - 1) & 1, abort_flag))
+                const int ns = isv ? kVStages : kKStages, s = m % ns;
+                if (m >= ns && !tc::mbar_wait(bar((isv ? kBarEV : kBarEK) + s), ((m / ns) - 1) & 1, abort_flag))
                     return false;
                 const int krow = z * p.N + key_tile(p, MODE, klist, m).x;
                 const uint32_t d = (isv ? sV : sK) + s * 2 * kRegion;
@@ -321,10 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
             // every issued load must land before the CTA can exit
             int never = 0;
-            for (int m = (nk > kStages ? nk - kStages : 0); m < nk; ++m)
-                tc::mbar_wait(bar(kBarK + m % kStages), (m / kStages) & 1, &never);
-            for (int m = (nv > kStages ? nv - kStages : 0); m < nv; ++m)
-                tc::mbar_wait(bar(kBarV + m % kStages), (m / kStages) & 1, &never);
+            for (int m = (nk > kKStages ? nk - kKStages : 0); m < nk; ++m)
+                tc::mbar_wait(bar(kBarK + m % kKStages), (m / kKStages) & 1, &never);
+            for (int m = (nv > kVStages ? nv - kVStages : 0); m < nv; ++m)
+                tc::mbar_wait(bar(kBarV + m % kVStages), (m / kVStages) & 1, &never);
             tc::mbar_wait(bar(kBarQ), 0, &never);
         }
     } else if (warp == 9) {
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         bool have = ntk > 0;
         bool ok = __all_sync(kFull, tc::mbar_wait(bar(kBarQ), 0, abort_flag));
         auto issue_S = [&](int t, int j) {
-            const uint32_t kb = sK + (j % kStages) * 2 * kRegion;
+            const uint32_t kb = sK + (j % kKStages) * 2 * kRegion;
             const uint32_t qb = sQ + (split ? 0 : t) * 2 * kRegion;
             const uint32_t id = idS(t, key_tile(p, MODE, klist, j).y <= 64);
 #pragma unroll
@@ -365,10 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 __syncwarp();
             }
             for (; ok && j < ntk; ++j) {
-                const int t = j & 1, s = j % kStages;
+                const int t = j & 1, s = j % kVStages;
                 const bool nh = j + 2 < ntk;
-                if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kStages) & 1, abort_flag))) break;
-                if (nh && !__all_sync(kFull, tc::mbar_wait(bar(kBarK + ((j + 2) % kStages)), ((j + 2) / kStages) & 1,
+                if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kVStages) & 1, abort_flag))) break;
+                if (nh && !__all_sync(kFull, tc::mbar_wait(bar(kBarK + ((j + 2) % kKStages)), ((j + 2) / kKStages) & 1,
                                                           abort_flag)))
                     break;
                 if (!__all_sync(kFull, tc::mbar_wait(bar(kBarP + t), (j >> 1) & 1, abort_flag))) break;
@@ -386,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tc::commit(bar(kBarEV + s));
                     if (nh) {
                         issue_S(t, j + 2);
-                        tc::commit(bar(kBarEK + (j + 2) % kStages));
+                        tc::commit(bar(kBarEK + (j + 2) % kKStages));
                     } else {
                         tc::commit(bar(kBarO + t));
                     }
@@ -408,9 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         while (ok && have) {
             const bool nhave = j + 1 < ntk;
-            const int s = j % kStages;
-            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kStages) & 1, abort_flag))) break;
-            if (nhave && !__all_sync(kFull, tc::mbar_wait(bar(kBarK + ((j + 1) % kStages)), ((j + 1) / kStages) & 1,
+            const int s = j % kVStages;
+            if (!__all_sync(kFull, tc::mbar_wait(bar(kBarV + s), (j / kVStages) & 1, abort_flag))) break;
+            if (nhave && !__all_sync(kFull, tc::mbar_wait(bar(kBarK + ((j + 1) % kKStages)), ((j + 1) / kKStages) & 1,
                                                          abort_flag)))
                 break;
             for (int t = 0; t < ntiles && ok; ++t) {
@@ -430,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     if (last) tc::commit(bar(kBarEV + s));                  // V(j) read by every PV
                     if (nhave) {
                         issue_S(t, j + 1);
-                        if (last) tc::commit(bar(kBarEK + (j + 1) % kStages));   // K(j+1) read by every S
+                        if (last) tc::commit(bar(kBarEK + (j + 1) % kKStages));   // K(j+1) read by every S
                     } else {
                         tc::commit(bar(kBarO + t));
                     }
