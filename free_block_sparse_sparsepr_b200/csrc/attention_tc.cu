@@ -43,6 +43,7 @@ constexpr int kRegion = 16384;      // one [128 rows][64 bf16] 128B-swizzled reg
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512; // S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512)
 constexpr float kRescaleLog2 = 8.f; // lazy rescale threshold (P <= 2^8)
+constexpr float kRescaleMax = 256.f; // 2^kRescaleLog2
 constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr int kOffQ = 0;                                   // tile t at + t * 2 * kRegion
@@ -113,6 +114,24 @@ __device__ __forceinline__ void load_half(uint32_t tS, int h, int lim, uint32_t 
             pm[(i >> 1) & 3] = fmax3(pm[(i >> 1) & 3], __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
     }
     mx = fmax3(fmaxf(pm[0], pm[1]), pm[2], pm[3]);
+}
+
+// Half h (64 columns) of this thread's row of S from TMEM, keys at or past `lim` set to -inf.
+__device__ __forceinline__ void load_half_nomax(uint32_t tS, int h, int lim, uint32_t (&sv)[2][32]) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tc::tmem_ld32(tS + 64 * h + 32 * c, sv[c]);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tc::regs_after_wait(sv[c]);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const int c0 = 64 * h + 32 * c;
+        if (c0 + 32 > lim) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i >= lim) sv[c][i] = __float_as_uint(-INFINITY);
+        }
+    }
 }
 
 // 2^x on the special-function unit (flushes results below 2^-126 to zero).
@@ -677,38 +696,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // registers; only when some row of the warp has a logit more than 2^8 above its
                 // running max (rare after the first tile) is the tile redone from S, which stays
                 // in TMEM until P is written.
-                const float thr = (m_run + kRescaleLog2) / c_log2;      // raw-logit threshold
-                uint32_t pk0[32];                                       // P of columns 0..63
+                // P is formed against the running max m_run without looking at this tile's maxima:
+                // every p is at most the row's sum over the tile, so a sum of at most 2^8 proves
+                // that no logit rose by more than 2^8 above m_run (inf and NaN fail the test too).
+                // Otherwise, and on the warpgroup's first key tile, the tile is redone from S, which
+                // stays in TMEM until P is written: the row maxima are taken, m_run moves up to the
+                // new maximum (O and l rescaled), and P is formed again.
+                uint32_t pk0[32], pk1[32];                              // P of columns 0..63, 64..127
                 uint64_t ps[4] = {0ull, 0ull, 0ull, 0ull};              // packed pair sums
-                bool slow = false;
-                float mx0 = -INFINITY, mx1 = -INFINITY;
-                {
-                    uint32_t sv[2][32];
-                    load_half(tS, 0, lim, sv, mx0);
-                    slow = __any_sync(kFull, mx0 > thr);
-                    if (!slow) exp_half(sv, c_log2, -m_run, pk0, ps);
-                }
-                if (lim > 64) {
-                    uint32_t sv[2][32];
-                    load_half(tS, 1, lim, sv, mx1);
-                    slow = slow || __any_sync(kFull, mx1 > thr);
-                    if (!slow) {
-                        uint32_t pk1[32];
+                bool slow = j == 0;
+                if (!slow) {
+                    {
+                        uint32_t sv[2][32];
+                        load_half_nomax(tS, 0, lim, sv);
+                        exp_half(sv, c_log2, -m_run, pk0, ps);
+                    }
+                    if (lim > 64) {
+                        uint32_t sv[2][32];
+                        load_half_nomax(tS, 1, lim, sv);
                         exp_half(sv, c_log2, -m_run, pk1, ps);
+                    }
+                    float a0, a1, b0, b1;
+                    up2(add2(ps[0], ps[1]), a0, a1);
+                    up2(add2(ps[2], ps[3]), b0, b1);
+                    const float tsum = (a0 + a1) + (b0 + b1);
+                    slow = __any_sync(kFull, !(tsum <= kRescaleMax));
+                    if (!slow) {
                         tc::tmem_st16(tS, pk0);
                         tc::tmem_st16(tS + 16, pk0 + 16);
-                        tc::tmem_st16(tS + 32, pk1);
-                        tc::tmem_st16(tS + 48, pk1 + 16);
+                        if (lim > 64) {
+                            tc::tmem_st16(tS + 32, pk1);
+                            tc::tmem_st16(tS + 48, pk1 + 16);
+                        }
+                        l_run += tsum;
                     }
-                } else if (!slow) {
-                    // a half tile (S and PV run with 64 keys): P of the first 64 keys only
-                    tc::tmem_st16(tS, pk0);
-                    tc::tmem_st16(tS + 16, pk0 + 16);
                 }
                 if (slow) {
-                    // some row's max moved by more than 2^8: new per-row max, rescale O and l
+                    float mx0 = -INFINITY, mx1 = -INFINITY;
+                    {
+                        uint32_t sv[2][32];
+                        load_half(tS, 0, lim, sv, mx0);
+                    }
+                    if (lim > 64) {
+                        uint32_t sv[2][32];
+                        load_half(tS, 1, lim, sv, mx1);
+                    }
                     const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * c_log2);
-                    const bool rescale = m_new > m_run + kRescaleLog2;
+                    const bool rescale = m_new > m_run;
                     if (j > 0 && __any_sync(kFull, rescale)) {
                         // S_t(j) complete => PV_t(j-1) complete: O_t may be rescaled now
                         const float f = rescale ? exp2f(m_run - m_new) : 1.f;
@@ -727,17 +761,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     if (rescale) m_run = m_new;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) ps[e] = 0ull;
-                    uint32_t pk1[32];
                     {
                         uint32_t sv[2][32];
-                        float dummy;
-                        load_half(tS, 0, lim, sv, dummy);
+                        load_half_nomax(tS, 0, lim, sv);
                         exp_half(sv, c_log2, -m_run, pk0, ps);
                     }
                     if (lim > 64) {
                         uint32_t sv[2][32];
-                        float dummy;
-                        load_half(tS, 1, lim, sv, dummy);
+                        load_half_nomax(tS, 1, lim, sv);
                         exp_half(sv, c_log2, -m_run, pk1, ps);
                     } else {
 #pragma unroll
@@ -747,8 +778,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tc::tmem_st16(tS + 16, pk0 + 16);
                     tc::tmem_st16(tS + 32, pk1);
                     tc::tmem_st16(tS + 48, pk1 + 16);
-                }
-                {
                     float a0, a1, b0, b1;
                     up2(add2(ps[0], ps[1]), a0, a1);
                     up2(add2(ps[2], ps[3]), b0, b1);
