@@ -30,7 +30,53 @@ inline int pad64(int v) { return (v + 63) / 64 * 64; }
 
 enum Stage { kStPartition = 0, kStRoute, kStPermute, kStAttn, kStProbeFit, kStWriteback, kStUnused, kStTotal, kNumStages };
 
-constexpr int kHostChunks = 8;     // KV-head chunks of the host-buffer pipeline
+constexpr int kHostChunks = 9;     // KV-head chunks of the host-buffer pipeline
+// Compute streams of the pipeline, taken by the chunks in turn: the latency-bound steps of a
+// chunk (the route selection, the fit, the small k-means kernels of a few heads) then overlap
+// other chunks' throughput-bound kernels instead of running alone.
+constexpr int kHostStreams = 8;
+// Relative chunk sizes: small at both ends, so that the first chunk's inputs land and the last
+// chunk's output leaves quickly (a head's copy in is shorter than its call, so after the first
+// chunks the copies stay ahead of the compute).
+constexpr int kChunkWeight[kHostChunks] = {1, 2, 3, 4, 4, 4, 3, 2, 1};
+
+// Chunk boundaries z0[0..nc] of P KV heads: one head per chunk up to kHostChunks heads, else the
+// weights scaled to P (largest remainders, at least one head each).
+int host_chunks(int P, int* z0) {
+    if (P <= kHostChunks) {
+        for (int i = 0; i <= P; ++i) z0[i] = i;
+        return P;
+    }
+    int wsum = 0;
+    for (int i = 0; i < kHostChunks; ++i) wsum += kChunkWeight[i];
+    int size[kHostChunks], left = P;
+    long long rem[kHostChunks];
+    for (int i = 0; i < kHostChunks; ++i) {
+        const long long num = (long long)kChunkWeight[i] * P;
+        size[i] = (int)(num / wsum);
+        if (size[i] < 1) size[i] = 1;
+        rem[i] = num % wsum;
+        left -= size[i];
+    }
+    while (left > 0) {   // the largest remainders (earliest on ties) take the heads still unassigned
+        int b = 0;
+        for (int i = 1; i < kHostChunks; ++i)
+            if (rem[i] > rem[b]) b = i;
+        ++size[b];
+        rem[b] = -1;
+        --left;
+    }
+    while (left < 0) {   // the clamp to one head overshot: the largest chunks give heads back
+        int b = 0;
+        for (int i = 1; i < kHostChunks; ++i)
+            if (size[i] > size[b]) b = i;
+        --size[b];
+        ++left;
+    }
+    z0[0] = 0;
+    for (int i = 0; i < kHostChunks; ++i) z0[i + 1] = z0[i] + size[i];
+    return kHostChunks;
+}
 
 }  // namespace
 
@@ -41,8 +87,8 @@ struct HostPipe {
     int nc = 0;
     int z0[kHostChunks + 1] = {};
     sparsepr_handle_s* sub[kHostChunks] = {};
-    cudaStream_t in = nullptr, comp[2] = {}, out = nullptr;   // chunks alternate between two compute streams
-    cudaEvent_t start = nullptr, end_comp[2] = {}, end_out = nullptr;
+    cudaStream_t in = nullptr, comp[kHostStreams] = {}, out = nullptr;   // chunk i on compute stream i % kHostStreams
+    cudaEvent_t start = nullptr, end_comp[kHostStreams] = {}, end_out = nullptr;
     cudaEvent_t ev_in[kHostChunks] = {}, ev_done[kHostChunks] = {};
 };
 
@@ -539,9 +585,13 @@ static void destroy_pipe(HostPipe* pp) {
     if (!pp) return;
     for (int i = 0; i < pp->nc; ++i)
         if (pp->sub[i]) sparsepr_destroy(pp->sub[i]);
-    for (cudaStream_t st : {pp->in, pp->comp[0], pp->comp[1], pp->out})
+    for (cudaStream_t st : {pp->in, pp->out})
         if (st) cudaStreamDestroy(st);
-    for (cudaEvent_t e : {pp->start, pp->end_comp[0], pp->end_comp[1], pp->end_out})
+    for (int k = 0; k < kHostStreams; ++k) {
+        if (pp->comp[k]) cudaStreamDestroy(pp->comp[k]);
+        if (pp->end_comp[k]) cudaEventDestroy(pp->end_comp[k]);
+    }
+    for (cudaEvent_t e : {pp->start, pp->end_out})
         if (e) cudaEventDestroy(e);
     for (int i = 0; i < kHostChunks; ++i) {
         if (pp->ev_in[i]) cudaEventDestroy(pp->ev_in[i]);
@@ -772,9 +822,7 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
     if (!h->pipe) {
         HostPipe* pp = new (std::nothrow) HostPipe();
         if (!pp) return SPARSEPR_ERR_WORKSPACE;
-        pp->nc = h->P < kHostChunks ? h->P : kHostChunks;
-        const int base = h->P / pp->nc, extra = h->P % pp->nc;
-        for (int i = 0; i < pp->nc; ++i) pp->z0[i + 1] = pp->z0[i] + base + (i < extra ? 1 : 0);
+        pp->nc = host_chunks(h->P, pp->z0);
         bool ok = true;
         for (int i = 0; i < pp->nc && ok; ++i) {
             sparsepr_config sc = c;
@@ -785,10 +833,11 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
             ok = sparsepr_create(&sc, &pp->sub[i]) == SPARSEPR_OK;
         }
         ok = ok && cudaStreamCreateWithFlags(&pp->in, cudaStreamNonBlocking) == cudaSuccess &&
-             cudaStreamCreateWithFlags(&pp->comp[0], cudaStreamNonBlocking) == cudaSuccess &&
-             cudaStreamCreateWithFlags(&pp->comp[1], cudaStreamNonBlocking) == cudaSuccess &&
              cudaStreamCreateWithFlags(&pp->out, cudaStreamNonBlocking) == cudaSuccess;
-        for (cudaEvent_t* e : {&pp->start, &pp->end_comp[0], &pp->end_comp[1], &pp->end_out})
+        for (int k = 0; k < kHostStreams && ok; ++k)
+            ok = cudaStreamCreateWithFlags(&pp->comp[k], cudaStreamNonBlocking) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&pp->end_comp[k], cudaEventDisableTiming) == cudaSuccess;
+        for (cudaEvent_t* e : {&pp->start, &pp->end_out})
             ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
         for (int i = 0; i < pp->nc && ok; ++i)
             ok = cudaEventCreateWithFlags(&pp->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
@@ -807,8 +856,9 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
     const bf16* hV = static_cast<const bf16*>(V);
     bf16* hO = static_cast<bf16*>(O);
     bool ok = cudaEventRecord(pp->start, s) == cudaSuccess;
-    for (cudaStream_t st : {pp->in, pp->comp[0], pp->comp[1], pp->out})
+    for (cudaStream_t st : {pp->in, pp->out})
         ok = ok && cudaStreamWaitEvent(st, pp->start, 0) == cudaSuccess;
+    for (int k = 0; k < kHostStreams; ++k) ok = ok && cudaStreamWaitEvent(pp->comp[k], pp->start, 0) == cudaSuccess;
     // every chunk's inputs in order on the copy-in stream
     for (int i = 0; i < pp->nc && ok; ++i) {
         const size_t z = pp->z0[i], n = pp->z0[i + 1] - pp->z0[i];
@@ -820,12 +870,12 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
                  cudaSuccess &&
              cudaEventRecord(pp->ev_in[i], pp->in) == cudaSuccess;
     }
-    // each chunk's call once its inputs have landed (consecutive chunks on alternate compute
-    // streams, so one chunk's latency-bound kernels overlap the other's), its output copied back
+    // each chunk's call once its inputs have landed (chunk i on compute stream i % kHostStreams,
+    // so one chunk's latency-bound kernels overlap the others'), its output copied back
     int launches = 0;
     for (int i = 0; i < pp->nc && ok; ++i) {
         const size_t z = pp->z0[i], n = pp->z0[i + 1] - pp->z0[i];
-        cudaStream_t cs = pp->comp[i & 1];
+        cudaStream_t cs = pp->comp[i % kHostStreams];
         ok = cudaStreamWaitEvent(cs, pp->ev_in[i], 0) == cudaSuccess;
         if (ok && sparsepr_attention(pp->sub[i], h->sQ + z * qh, h->sK + z * kh, h->sV + z * kh, h->sO + z * qh,
                                      cs) != SPARSEPR_OK)
@@ -838,15 +888,15 @@ sparsepr_status sparsepr_attention_host(sparsepr_handle h, const void* Q, const 
              cudaMemcpyAsync(hO + z * qh, h->sO + z * qh, n * qh * sizeof(bf16), cudaMemcpyDeviceToHost, pp->out) ==
                  cudaSuccess;
     }
-    for (int k = 0; k < 2; ++k)
+    for (int k = 0; k < kHostStreams; ++k)
         ok = ok && cudaEventRecord(pp->end_comp[k], pp->comp[k]) == cudaSuccess &&
              cudaStreamWaitEvent(s, pp->end_comp[k], 0) == cudaSuccess;
     ok = ok && cudaEventRecord(pp->end_out, pp->out) == cudaSuccess &&
          cudaStreamWaitEvent(s, pp->end_out, 0) == cudaSuccess;
     // every internal stream drains before returning, even after an error, so no work outlives the call
     bool drained = cudaStreamSynchronize(s) == cudaSuccess;
-    for (cudaStream_t st : {pp->in, pp->comp[0], pp->comp[1], pp->out})
-        drained = cudaStreamSynchronize(st) == cudaSuccess && drained;
+    for (cudaStream_t st : {pp->in, pp->out}) drained = cudaStreamSynchronize(st) == cudaSuccess && drained;
+    for (int k = 0; k < kHostStreams; ++k) drained = cudaStreamSynchronize(pp->comp[k]) == cudaSuccess && drained;
     if (!drained || !ok) return SPARSEPR_ERR_CUDA;
     // statistics and the device status of the chunk calls on the handle
     int worst = 0;
