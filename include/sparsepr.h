@@ -297,8 +297,8 @@ sparsepr_status sparsepr_attention(sparsepr_handle h, const void* Q, const void*
  * Same as sparsepr_attention but Q/K/V/O are HOST buffers (pinned or
  * pageable): copies them to and from the handle's device staging buffers and
  * synchronises before returning. The KV heads are processed in up to nine
- * chunks, each by an internal sub-handle on its own stream, so the copies of
- * some chunks overlap the compute of others; the output equals that of
+ * chunks, each by an internal sub-handle, on up to eight internal streams, so
+ * the copies of some chunks overlap the compute of others; the output equals that of
  * sparsepr_attention bit for bit. The first call allocates the staging
  * buffers (4 tensors of the call's size) and the sub-handles.
  */
