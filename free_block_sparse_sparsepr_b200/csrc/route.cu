@@ -33,46 +33,66 @@ __global__ void row_lse_kernel(const float* __restrict__ u, const int32_t* __res
 }
 
 // scores[z][a][g] = mean over the g heads and the queries of group a of exp(u - lse).
-__global__ void cell_scores_kernel(const float* __restrict__ u, const float* __restrict__ lse,
-                                   const int32_t* __restrict__ qperm, const int32_t* __restrict__ qoff,
-                                   const int32_t* __restrict__ koff, float* scores, int g, int N,
-                                   int Gq, int Gk) {
-    const int z = blockIdx.y, a = blockIdx.x;
+// One CTA per (group a, KV head z); thread t takes key-group column t of each 256-column chunk.
+// The group's row indices and their log2-scaled normalisers are staged in shared memory a round
+// of rows at a time (coalesced, out of the loads' dependence chain), and exp(u - lse) is formed as
+// 2^(u log2 e - lse log2 e) on the special-function unit (relative error about 1e-6); eight rows'
+// logits are in flight per thread and four partial sums are added in a fixed order.
+constexpr int kCsThreads = 256;
+constexpr int kCsRows = 1024;   // rows staged per round
+constexpr float kLog2eF = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__global__ void __launch_bounds__(kCsThreads) cell_scores_kernel(const float* __restrict__ u,
+                                                                 const float* __restrict__ lse,
+                                                                 const int32_t* __restrict__ qperm,
+                                                                 const int32_t* __restrict__ qoff,
+                                                                 const int32_t* __restrict__ koff, float* scores,
+                                                                 int g, int N, int Gq, int Gk) {
+    __shared__ int sIdx[kCsRows];
+    __shared__ float sL[kCsRows];
+    const int z = blockIdx.y, a = blockIdx.x, tid = threadIdx.x;
     const int lo = qoff[(long long)z * (Gq + 1) + a], hi = qoff[(long long)z * (Gq + 1) + a + 1];
     const int32_t* ko = koff + (long long)z * (Gk + 1);
     const int32_t* perm = qperm + (long long)z * N;
-    for (int gk = threadIdx.x; gk < Gk; gk += blockDim.x) {
+    for (int gk0 = 0; gk0 < Gk; gk0 += kCsThreads) {
+        const int gk = gk0 + tid;
+        const bool ok = hi > lo && gk < Gk && ko[gk + 1] > ko[gk];
         float acc = 0.f;
-        const bool ok = hi > lo && ko[gk + 1] > ko[gk];
-        if (ok) {
-            for (int j = 0; j < g; ++j) {
-                const long long x = (long long)z * g + j;
-                const float* ux = u + x * N * Gk;
-                const float* lx = lse + x * N;
-                // eight rows in flight, four partial sums added in a fixed order
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-                int p = lo;
-                for (; p + 8 <= hi; p += 8) {
-                    int i8[8];
-                    float v8[8], l8[8];
+        for (int j = 0; j < g; ++j) {
+            const long long x = (long long)z * g + j;
+            const float* ux = u + x * N * Gk + gk;
+            const float* lx = lse + x * N;
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int base = lo; base < hi; base += kCsRows) {
+                const int cnt = min(kCsRows, hi - base);
+                __syncthreads();   // the previous round's rows are no longer read
+                for (int t = tid; t < cnt; t += kCsThreads) {
+                    const int i = __ldg(perm + base + t);
+                    sIdx[t] = i;
+                    sL[t] = __ldg(lx + i) * kLog2eF;
+                }
+                __syncthreads();
+                if (ok) {
+                    int q = 0;
+                    for (; q + 8 <= cnt; q += 8) {
+                        float v8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) i8[e] = __ldg(perm + p + e);
+                        for (int e = 0; e < 8; ++e) v8[e] = __ldg(ux + (long long)sIdx[q + e] * Gk);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        v8[e] = __ldg(ux + (long long)i8[e] * Gk + gk);
-                        l8[e] = __ldg(lx + i8[e]);
+                        for (int e = 0; e < 8; ++e) a4[e & 3] += ex2_approx(fmaf(v8[e], kLog2eF, -sL[q + e]));
                     }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) a4[e & 3] += expf(v8[e] - l8[e]);
+                    for (; q < cnt; ++q) a4[0] += ex2_approx(fmaf(__ldg(ux + (long long)sIdx[q] * Gk), kLog2eF, -sL[q]));
                 }
-                for (; p < hi; ++p) {
-                    const int i = __ldg(perm + p);
-                    a4[0] += expf(__ldg(ux + (long long)i * Gk + gk) - __ldg(lx + i));
-                }
-                acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
             }
+            acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
         }
-        scores[((long long)z * Gq + a) * Gk + gk] = ok ? acc / ((float)g * (float)(hi - lo)) : 0.f;
+        if (gk < Gk) scores[((long long)z * Gq + a) * Gk + gk] = ok ? acc / ((float)g * (float)(hi - lo)) : 0.f;
     }
 }
 
@@ -82,7 +102,8 @@ __global__ void cell_scores_kernel(const float* __restrict__ u, const float* __r
 // exceed the remaining budget; it is kept iff its overshoot < the remaining undershoot.
 constexpr int kSelThreads = 1024;
 constexpr int kRadix = 2048;   // 11-bit digits
-__global__ void __launch_bounds__(kSelThreads) route_select_kernel(
+static_assert(2 * kSelThreads == kRadix, "two digit bins per thread in the scan");
+__global__ void __launch_bounds__(kSelThreads, 1) route_select_kernel(
     const float* __restrict__ scores, const int32_t* __restrict__ qoff, const int32_t* __restrict__ koff,
     int32_t* rowptr, int32_t* kg, int64_t* pairs, int Gq, int Gk, long long budget, int keep_all) {
     const int z = blockIdx.x;
@@ -98,6 +119,8 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
     __shared__ long long s_rem;
     __shared__ unsigned long long s_prefix, s_mask;
     __shared__ int s_found;
+    __shared__ int s_dsel;
+    __shared__ long long s_cum;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const float* S = scores + (long long)z * Gq * Gk;
@@ -176,21 +199,50 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(
                 }
             }
             __syncthreads();
-            if (tid == 0) {
-                long long cum = 0;
-                int dsel = -1;
-                for (int dg = 0; dg <= (int)dmask; ++dg) {
-                    long long h = (long long)hist[dg];
-                    if (h > 0 && cum + h > s_rem) { dsel = dg; break; }
-                    cum += h;
+            // The selected digit is the first bin whose cost, added to the cost of all lower bins,
+            // exceeds the remaining budget: a block-wide exclusive scan of the bins (two per
+            // thread) and the smallest bin that satisfies the test.
+            {
+                const int b0 = 2 * tid;
+                const long long h0 = (long long)hist[b0], h1 = (long long)hist[b0 + 1];
+                long long inc = h0 + h1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const long long n = __shfl_up_sync(kFull, inc, o);
+                    if (lane >= o) inc += n;
                 }
-                if (dsel < 0) {
-                    s_found = 0;  // every remaining candidate fits in the budget
-                } else {
-                    s_rem -= cum;
-                    s_prefix |= (unsigned long long)dsel << sh;
-                    s_mask |= dmask << sh;
-                    s_unique = hcnt[dsel] == 1;
+                if (lane == 31) red[warp] = inc;
+                if (tid == 0) s_dsel = kRadix;
+                __syncthreads();
+                if (warp == 0) {
+                    long long w = lane < nw ? red[lane] : 0;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const long long n = __shfl_up_sync(kFull, w, o);
+                        if (lane >= o) w += n;
+                    }
+                    if (lane < nw) red[lane] = w;   // inclusive totals of warps 0..lane
+                }
+                __syncthreads();
+                const long long before = (warp > 0 ? red[warp - 1] : 0) + inc - (h0 + h1);
+                const long long rem = s_rem;
+                int mine = kRadix;
+                if (h1 > 0 && before + h0 + h1 > rem) mine = b0 + 1;
+                if (h0 > 0 && before + h0 > rem) mine = b0;
+                if (mine < kRadix) atomicMin(&s_dsel, mine);
+                __syncthreads();
+                const int dsel = s_dsel;
+                if (dsel < kRadix && (dsel >> 1) == tid) s_cum = dsel == b0 ? before : before + h0;
+                __syncthreads();
+                if (tid == 0) {
+                    if (dsel == kRadix) {
+                        s_found = 0;  // every remaining candidate fits in the budget
+                    } else {
+                        s_rem -= s_cum;
+                        s_prefix |= (unsigned long long)dsel << sh;
+                        s_mask |= dmask << sh;
+                        s_unique = hcnt[dsel] == 1;
+                    }
                 }
             }
             __syncthreads();
@@ -295,7 +347,7 @@ cudaError_t launch_row_lse(const float* u, const int32_t* koff, float* lse, int 
 cudaError_t launch_cell_scores(const float* u, const float* lse, const int32_t* qperm,
                                const int32_t* qoff, const int32_t* koff, float* scores, int P,
                                int g, int N, int Gq, int Gk, cudaStream_t s) {
-    cell_scores_kernel<<<dim3(Gq, P), 256, 0, s>>>(u, lse, qperm, qoff, koff, scores, g, N, Gq, Gk);
+    cell_scores_kernel<<<dim3(Gq, P), kCsThreads, 0, s>>>(u, lse, qperm, qoff, koff, scores, g, N, Gq, Gk);
     return cudaGetLastError();
 }
 
