@@ -1,5 +1,5 @@
-"""The multi-rank path of bench.py on CPU: two gloo ranks (no GPU) run the host logic the
-driver's torchrun launch exercises — rendezvous, the max-over-ranks reduction of the timed
+"""The multi-rank path of bench.py on CPU: two gloo ranks (no GPU) run the host logic that a
+torchrun launch of bench.py exercises — rendezvous, the max-over-ranks reduction of the timed
 region, the barrier, the whole-job value (all ranks' work over the slowest rank's time), the
 per-rank seeding of the inputs, and the reference arm's rule that rank 0 alone runs and prints."""
 import contextlib
