@@ -1,0 +1,80 @@
+"""Parity on the degenerate inputs the method has.
+
+  - a target density below the probes' share (rho < M/N): the route budget rho N^2 - M N is
+    negative, so every query group keeps only its mandatory top cell ([execution]: rho_exec =
+    route density + M/N; every query group keeps at least one cell);
+  - identical keys: every distance of the key k-means ties, all keys fall in group 0 (ties go to
+    the lowest group), the other key groups are empty, the softmax over the keys is uniform, the
+    sparse output equals the dense one and the probe residuals are zero (an empty residual
+    subspace, a zero correction);
+  - identical queries: every query falls in query group 0, the other query groups are empty, and
+    the probe rows come from one group in index order (equal radial keys).
+
+Each runs the whole call on the GPU (fused and stage by stage, bit-identical) and checks it against
+the oracle with the GPU's partition and route handed in (sampled rows and every probe row, max-abs
+2e-2, mean-abs 2e-3), the cell scores and the selection (identical cells), and the group-major
+orders; the labels are also checked against the tie rule directly.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import free_block_sparse_sparsepr_b200 as spr  # noqa: E402
+from synthetic import Workload, video_qkv  # noqa: E402
+from gpu_helpers import sampled_call_parity  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+# d = 128 (tensor-core path), GQA with two query heads per KV head, Gk > rQ (projected coordinates)
+W = Workload("degenerate_n4096", B=1, Hq=4, Hkv=2, T=4, Hg=32, Wg=32, d=128, Gk=96, Gq=80, block=128,
+             rho=0.22, locality=1.0)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    spr.load_library()
+
+
+def _labels(w, Qb, Kb):
+    q, k = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda() for x in (Qb, Kb))
+    with spr.SparsePR.from_workload(w) as h:
+        pv = {n: t.cpu().numpy() for n, t in h.partition_views(h.partition(q, k)).items()}
+        assert h.device_status() == 0
+    return pv
+
+
+def test_density_below_the_probe_share():
+    w = W.replace(rho=0.01)                               # M / N = 64 / 4096 = 1.56%
+    assert oracle.budget_pairs(w.rho, w.N, w.M) < 0
+    rv = sampled_call_parity(w, *video_qkv(w), kv_heads=[0, 1])
+    for z in range(w.B * w.Hkv):
+        cells = np.diff(rv["rowptr"][z])
+        assert cells.max() <= 1                           # the mandatory cell only
+    pv = _labels(w, *video_qkv(w)[:2])
+    for z in range(w.B * w.Hkv):
+        assert np.array_equal(np.diff(rv["rowptr"][z]), (np.diff(pv["qoff"][z]) > 0).astype(np.int32))
+
+
+def test_identical_keys():
+    Qb, Kb, Vb = video_qkv(W)
+    Kb = np.ascontiguousarray(np.broadcast_to(Kb[:, :, :1, :], Kb.shape))
+    sampled_call_parity(W, Qb, Kb, Vb, kv_heads=[0, 1])
+    pv = _labels(W, Qb, Kb)
+    for z in range(W.B * W.Hkv):
+        assert np.all(pv["kgroup"][z] == 0)               # every distance ties: the lowest group
+        assert pv["koff"][z][1] == W.N
+
+
+def test_identical_queries():
+    Qb, Kb, Vb = video_qkv(W)
+    Qb = np.ascontiguousarray(np.broadcast_to(Qb[:, :, :1, :], Qb.shape))
+    sampled_call_parity(W, Qb, Kb, Vb, kv_heads=[0, 1])
+    pv = _labels(W, Qb, Kb)
+    for z in range(W.B * W.Hkv):
+        assert np.all(pv["qgroup"][z] == 0)
+        probe = np.sort(pv["probe"][z])
+        assert np.array_equal(probe, oracle.sample_rows(W.N, W.M))   # one group, index order
