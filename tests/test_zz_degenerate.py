@@ -8,7 +8,10 @@
     sparse output equals the dense one and the probe residuals are zero (an empty residual
     subspace, a zero correction);
   - identical queries: every query falls in query group 0, the other query groups are empty, and
-    the probe rows come from one group in index order (equal radial keys).
+    the probe rows come from one group in index order (equal radial keys);
+  - extreme sizes and group counts: a length below one row tile (N = 100, GQA), a single cell
+    (Gk = Gq = 1: the route keeps everything, the query coordinates are all zero), and as many key
+    groups as keys (N = Gk = 256: groups of one key).
 
 Each runs the whole call on the GPU (fused and stage by stage, bit-identical) and checks it against
 the oracle with the GPU's partition and route handed in (sampled rows and every probe row, max-abs
@@ -78,3 +81,20 @@ def test_identical_queries():
         assert np.all(pv["qgroup"][z] == 0)
         probe = np.sort(pv["probe"][z])
         assert np.array_equal(probe, oracle.sample_rows(W.N, W.M))   # one group, index order
+
+
+SMALL = [
+    Workload("n100_gqa", B=1, Hq=2, Hkv=1, T=1, Hg=10, Wg=10, d=128, Gk=8, Gq=6, block=64, rho=0.4, M=16, r=4),
+    Workload("single_cell_n512", B=1, Hq=2, Hkv=2, T=2, Hg=16, Wg=16, d=64, Gk=1, Gq=1, block=64, rho=0.22, M=32,
+             r=8),
+    Workload("one_key_per_group_n256", B=1, Hq=2, Hkv=2, T=1, Hg=16, Wg=16, d=128, Gk=256, Gq=128, block=128,
+             rho=0.3, M=32, r=8),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_and_extreme_group_counts(w):
+    rv = sampled_call_parity(w, *video_qkv(w))
+    if w.Gk == 1 and w.Gq == 1:
+        for z in range(w.B * w.Hkv):
+            assert int(rv["pairs"][z]) == w.N * w.N          # the one cell holds every pair
