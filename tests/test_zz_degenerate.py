@@ -10,8 +10,10 @@
   - identical queries: every query falls in query group 0, the other query groups are empty, and
     the probe rows come from one group in index order (equal radial keys);
   - extreme sizes and group counts: a length below one row tile (N = 100, GQA), a single cell
-    (Gk = Gq = 1: the route keeps everything, the query coordinates are all zero), and as many key
-    groups as keys (N = Gk = 256: groups of one key).
+    (Gk = Gq = 1: the route keeps everything, the query coordinates are all zero), as many key
+    groups as keys (N = Gk = 256: groups of one key), every row a probe (M = N = 64: the output is
+    the dense attention), no Lloyd round after the seeding assignment (the centroids are the seed
+    rows), and an odd GQA group (three query heads on one KV head).
 
 Each runs the whole call on the GPU (fused and stage by stage, bit-identical) and checks it against
 the oracle with the GPU's partition and route handed in (sampled rows and every probe row, max-abs
@@ -89,6 +91,11 @@ SMALL = [
              r=8),
     Workload("one_key_per_group_n256", B=1, Hq=2, Hkv=2, T=1, Hg=16, Wg=16, d=128, Gk=256, Gq=128, block=128,
              rho=0.3, M=32, r=8),
+    Workload("every_row_a_probe_n64", B=1, Hq=2, Hkv=2, T=1, Hg=8, Wg=8, d=128, Gk=4, Gq=4, block=64, rho=0.5, M=64,
+             r=8),
+    Workload("no_lloyd_rounds_n1024", B=1, Hq=2, Hkv=2, T=4, Hg=16, Wg=16, d=128, Gk=16, Gq=16, block=128,
+             rho=0.25, kmeans_iters=0),
+    Workload("gqa_odd_group_n1024", B=1, Hq=3, Hkv=1, T=4, Hg=16, Wg=16, d=128, Gk=16, Gq=12, block=128, rho=0.3),
 ]
 
 
