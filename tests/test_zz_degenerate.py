@@ -13,7 +13,10 @@
     (Gk = Gq = 1: the route keeps everything, the query coordinates are all zero), as many key
     groups as keys (N = Gk = 256: groups of one key), every row a probe (M = N = 64: the output is
     the dense attention), no Lloyd round after the seeding assignment (the centroids are the seed
-    rows), and an odd GQA group (three query heads on one KV head).
+    rows), and an odd GQA group (three query heads on one KV head);
+  - the other shapes the configuration allows: d = 64 under GQA with an even group (two query heads
+    per attention CTA), the smallest ranks (rK = rQ = 8 with Gk > rQ, r = 1) and the largest
+    (rK = rQ = 64, M = 64, r = 32).
 
 Each runs the whole call on the GPU (fused and stage by stage, bit-identical) and checks it against
 the oracle with the GPU's partition and route handed in (sampled rows and every probe row, max-abs
@@ -96,6 +99,12 @@ SMALL = [
     Workload("no_lloyd_rounds_n1024", B=1, Hq=2, Hkv=2, T=4, Hg=16, Wg=16, d=128, Gk=16, Gq=16, block=128,
              rho=0.25, kmeans_iters=0),
     Workload("gqa_odd_group_n1024", B=1, Hq=3, Hkv=1, T=4, Hg=16, Wg=16, d=128, Gk=16, Gq=12, block=128, rho=0.3),
+    Workload("d64_even_gqa_n2048", B=1, Hq=4, Hkv=2, T=2, Hg=32, Wg=32, d=64, Gk=32, Gq=24, block=64, rho=0.25,
+             M=32, r=8),
+    Workload("low_ranks_n1024", B=1, Hq=2, Hkv=2, T=4, Hg=16, Wg=16, d=128, Gk=32, Gq=16, block=128, rho=0.25,
+             rK=8, rQ=8, M=16, r=1),
+    Workload("max_ranks_n2048", B=1, Hq=2, Hkv=2, T=2, Hg=32, Wg=32, d=128, Gk=64, Gq=48, block=128, rho=0.2,
+             rK=64, rQ=64, M=64, r=32),
 ]
 
 
