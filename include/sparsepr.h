@@ -235,8 +235,10 @@ sparsepr_status sparsepr_partition(sparsepr_handle h, const void* Q, const void*
  * floor(rho_exec*N^2) - M*N: each query group's top cell first, then cells in
  * descending score (ties: lower query group, then lower key group) while the
  * total stays within budget, the crossing cell kept iff its overshoot is
- * smaller than the undershoot without it. `part` may be handle-owned or
- * handed in. *out receives pointers to handle-owned buffers.
+ * smaller than the undershoot without it. A budget below the top cells' cost
+ * (negative when rho_exec < M/N) keeps the top cells only; rho_exec >= 1 keeps
+ * every cell whose query and key groups are both non-empty. `part` may be
+ * handle-owned or handed in. *out receives pointers to handle-owned buffers.
  */
 sparsepr_status sparsepr_route(sparsepr_handle h, const void* Q, const sparsepr_partition_t* part,
                                sparsepr_route_t* out, void* stream);
