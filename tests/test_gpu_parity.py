@@ -11,9 +11,10 @@ torch = pytest.importorskip("torch")
 
 import oracle  # noqa: E402
 import free_block_sparse_sparsepr_b200 as spr  # noqa: E402
-from synthetic import Workload, get_workload  # noqa: E402
+from synthetic import Workload, get_workload, video_qkv  # noqa: E402
 from gpu_helpers import (MAX_ABS, MEAN_ABS, assert_close, bf16_to_f64, err, inputs, kmeans_margin,  # noqa: E402
-                         partition_tensors, route_tensors, selected_from_csr, to_group_major)
+                         partition_tensors, route_tensors, sampled_call_parity, selected_from_csr,
+                         to_group_major)
 
 pytestmark = pytest.mark.gpu
 
@@ -265,6 +266,17 @@ def test_attention_end_to_end(name):
             assert e_gpu <= 1.1 * e_orc + 1e-3, (e_gpu, e_orc)
         mx, mn = err(Of, res["O"])
         assert mn <= 5 * MEAN_ABS, f"end-to-end mean-abs {mn}"
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_call_on_its_own_partition_every_row(name):
+    """The fused call element by element: the GPU's own partition and route handed to the oracle,
+    every row of every query head within max-abs 2e-2 / mean-abs 2e-3 (O_s and O), plus the cell
+    scores, the selection rule on the GPU's scores (identical cells) and the probe rows = the
+    GPU's dense rows exactly. Complements the end-to-end test above, whose partitions may differ
+    from the oracle's at k-means near ties and which therefore compares a mean only."""
+    w = CASES[name]
+    sampled_call_parity(w, *video_qkv(w), kv_heads=range(w.B * w.Hkv), rows_per_head=w.N)
 
 
 def test_full_density_equals_dense():
