@@ -317,11 +317,74 @@ def m_correction_sign(Os, U, A, obar, Rbar, flags=0):
     return _ORIG["correction"](Os, U, A, -obar, Rbar, flags)
 
 
+def m_top_mass_set_strict(z_row, mass=0.9):
+    """Keys tied with the k-th largest logit left out (strict comparison)."""
+    z = np.asarray(z_row, dtype=np.float64)
+    k = osp.top_mass_count(z, mass)
+    return z > np.sort(z)[::-1][k - 1]
+
+
+def m_top_mass_count_right(z_row, mass=0.9):
+    """Cumulative-mass search from the right: one key too many when the mass lands exactly."""
+    z = np.asarray(z_row, dtype=np.float64)
+    c = np.cumsum(np.sort(np.exp(z - z.max()))[::-1])
+    return min(int(np.searchsorted(c, mass * c[-1], side="right")) + 1, len(z))
+
+
+def m_shared_rows_no_half(lo, hi, R=osp.SHARED_ROWS):
+    """Shared-route rows without the half-step offset."""
+    size = hi - lo
+    Rp = min(R, size)
+    return lo + (np.arange(Rp, dtype=np.int64) * size) // Rp
+
+
+def m_shared_support_largest_not_union(Qg, Kh, qperm, qoff, R=osp.SHARED_ROWS, mass=0.9):
+    """The group's support taken as its largest single-row set instead of the union."""
+    union, single = _ORIG["shared_support"](Qg, Kh, qperm, qoff, R, mass)
+    return single.max(axis=1), single
+
+
+def m_shared_support_head0(Qg, Kh, qperm, qoff, R=osp.SHARED_ROWS, mass=0.9):
+    """Every shared row taken from query head 0 (the cycling over the KV group's heads dropped)."""
+    return _ORIG["shared_support"](Qg[:1], Kh, qperm, qoff, R, mass)
+
+
+def m_probe_uniform_no_half(qperm, M):
+    """Uniform probe grid without the half-step offset."""
+    rows = (np.arange(M, dtype=np.int64) * len(qperm)) // M
+    return osp._by_sequence_position(rows, qperm)
+
+
+def m_probe_random_no_salt(qperm, M, seed):
+    """Random probes drawn from the seed without the salt."""
+    return _ORIG["probe_rows_random"](qperm, M, seed ^ osp.PROBE_SEED_SALT)
+
+
+def m_affine_total_denominator(Os, Od):
+    """Explained fraction over the uncentred residual energy."""
+    Os = np.asarray(Os, dtype=np.float64)
+    R = np.asarray(Od, dtype=np.float64) - Os
+    X = np.concatenate([Os, np.ones((Os.shape[0], 1))], axis=1)
+    beta, *_ = np.linalg.lstsq(X, R, rcond=None)
+    sse = float(((R - X @ beta) ** 2).sum())
+    return 1.0 - sse / float((R ** 2).sum()), sse / float((R ** 2).sum())
+
+
+def m_affine_no_intercept(Os, Od):
+    """Affine fit without the constant column (a linear fit)."""
+    Os = np.asarray(Os, dtype=np.float64)
+    R = np.asarray(Od, dtype=np.float64) - Os
+    beta, *_ = np.linalg.lstsq(Os, R, rcond=None)
+    sse = float(((R - Os @ beta) ** 2).sum())
+    return 1.0 - sse / float(((R - R.mean(axis=0)) ** 2).sum()), sse / float((R ** 2).sum())
+
+
 # ---------------------------------------------------------------- cases
 
 P = "test_oracle_partition"
 R = "test_oracle_route_attn_fit"
 D = "test_oracle_steps_direct"
+SS = "test_oracle_shared_support"
 
 CASES = [
     ("sample_rows", m_sample_rows_no_half, [(P, "test_sample_rows_closed_form")]),
@@ -362,6 +425,15 @@ CASES = [
     ("residual_subspace", m_subspace_right_vectors, [(R, "test_residual_subspace_equals_gram_eigenvectors")]),
     ("correction", m_correction_rbar_unprojected, [(R, "test_correction_variants")]),
     ("correction", m_correction_sign, [(R, "test_correction_variants")]),
+    ("top_mass_set", m_top_mass_set_strict, [(SS, "test_top_mass_set_closed_forms")]),
+    ("top_mass_count", m_top_mass_count_right, [(SS, "test_top_mass_set_closed_forms")]),
+    ("shared_rows", m_shared_rows_no_half, [(SS, "test_shared_rows_positions")]),
+    ("shared_support", m_shared_support_largest_not_union, [(SS, "test_shared_support_brute_force")]),
+    ("shared_support", m_shared_support_head0, [(SS, "test_shared_support_brute_force")]),
+    ("probe_rows_uniform", m_probe_uniform_no_half, [(SS, "test_alternative_probe_samplers")]),
+    ("probe_rows_random", m_probe_random_no_salt, [(SS, "test_alternative_probe_samplers")]),
+    ("affine_diagnostics", m_affine_total_denominator, [(SS, "test_affine_diagnostics_planted")]),
+    ("affine_diagnostics", m_affine_no_intercept, [(SS, "test_affine_diagnostics_planted")]),
 ]
 
 
