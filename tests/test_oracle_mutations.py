@@ -379,6 +379,24 @@ def m_affine_no_intercept(Os, Od):
     return 1.0 - sse / float(((R - R.mean(axis=0)) ** 2).sum()), sse / float((R ** 2).sum())
 
 
+def m_call_no_probe_override(Q, K, V, cfg, rows=None, partitions=None, routes=None):
+    """Probe rows of the output left as corrected sparse rows instead of the exact dense rows."""
+    res = _ORIG["sparsepr_attention"](Q, K, V, cfg, rows, partitions, routes)
+    g = Q.shape[1] // K.shape[1]
+    for (b, hq), fit in res["fits"].items():
+        p = res["partitions"][(b, hq // g)].probe
+        o = res["O_sparse"][b, hq, p]
+        res["O"][b, hq, p] = o + osp.correction(o, fit.U, fit.A, fit.obar, fit.Rbar, getattr(cfg, "flags", 0))
+    return res
+
+
+def m_call_rho_exec_without_probes(Q, K, V, cfg, rows=None, partitions=None, routes=None):
+    """Execution density reported without the probes' share M/N."""
+    res = _ORIG["sparsepr_attention"](Q, K, V, cfg, rows, partitions, routes)
+    res["rho_exec"] = res["route_density"]
+    return res
+
+
 # ---------------------------------------------------------------- cases
 
 P = "test_oracle_partition"
@@ -434,6 +452,8 @@ CASES = [
     ("probe_rows_random", m_probe_random_no_salt, [(SS, "test_alternative_probe_samplers")]),
     ("affine_diagnostics", m_affine_total_denominator, [(SS, "test_affine_diagnostics_planted")]),
     ("affine_diagnostics", m_affine_no_intercept, [(SS, "test_affine_diagnostics_planted")]),
+    ("sparsepr_attention", m_call_no_probe_override, [(R, "test_probe_rows_of_output_are_dense_rows_exactly")]),
+    ("sparsepr_attention", m_call_rho_exec_without_probes, [(R, "test_realised_density_and_rho_exec")]),
 ]
 
 
